@@ -1,0 +1,57 @@
+"""The oracle's pins must catch plausible slips (CPU only).
+
+Each case plants one mistake in a copy of the oracle's C source (a dropped term,
+an off-by-one, a reversed order, a wrong index), builds it into a scratch
+directory, and runs the pin suite against that build in a subprocess. The
+suite must fail for every mutant; the unmodified oracle passes it (the pin
+tests themselves).
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "lci_oracle.c")
+
+# (name, original text, planted mistake)
+MUTANTS = [
+    ("score drops all heads but one",
+     "            for (int64_t h = 0; h < H; ++h)\n                for (int64_t d = 0; d < D; ++d)\n                    acc +=",
+     "            for (int64_t h = 0; h < 1; ++h)\n                for (int64_t d = 0; d < D; ++d)\n                    acc +="),
+    ("score reads the query row of the sequence, not of the query",
+     "ld(q_c, dt, (row * H + h) * D + d)", "ld(q_c, dt, (b * H + h) * D + d)"),
+    ("query's own block not visible", "int64_t v = last / bs + 1;", "int64_t v = last / bs;"),
+    ("ties keep the higher id", "return (x->id > y->id) - (x->id < y->id);",
+     "return (x->id < y->id) - (x->id > y->id);"),
+    ("ascending scores", "if (x->score > y->score) return -1;\n    if (x->score < y->score) return 1;",
+     "if (x->score < y->score) return -1;\n    if (x->score > y->score) return 1;"),
+    ("query's own token masked", "if (t > last) break;", "if (t >= last) break;"),
+    ("kv head chosen modulo instead of by group", "            int64_t g = h / G;\n            double* o = out + (r * H_q + h) * hd;\n            for (int64_t d = 0; d < hd; ++d) o[d] = 0.0;\n            if (n == 0) continue;",
+     "            int64_t g = h % H_kv;\n            double* o = out + (r * H_q + h) * hd;\n            for (int64_t d = 0; d < hd; ++d) o[d] = 0.0;\n            if (n == 0) continue;"),
+    ("pool slot and head transposed", "return ((page * H_kv + g) * bs + u) * hd + d;",
+     "return ((page * bs + u) * H_kv + g) * hd + d;"),
+    ("scale dropped", "                logit[t] = scale * dot;\n                if (logit[t] > m) m = logit[t];\n            }\n            double den",
+     "                logit[t] = dot;\n                if (logit[t] > m) m = logit[t];\n            }\n            double den"),
+    ("block mean divides by the block size", "sum / (double)(t1 - t0)", "sum / (double)bs"),
+    ("bf16 widened with the wrong shift", "<< 16;", "<< 15;"),
+    ("block table row stride ignored", "int64_t page = block_table[b * nb_max + j];\n            for (int64_t u = 0; u < bs; ++u) {",
+     "int64_t page = block_table[j];\n            for (int64_t u = 0; u < bs; ++u) {"),
+]
+
+
+@pytest.mark.parametrize("name,orig,bad", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(name, orig, bad, tmp_path):
+    src = open(SRC).read()
+    assert src.count(orig) == 1, f"mutation site not unique: {name}"
+    mut_c = tmp_path / "mutant.c"
+    mut_c.write_text(src.replace(orig, bad))
+    mut_so = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-o", str(mut_so),
+                    str(mut_c), "-lm"], check=True)
+    env = dict(os.environ, LCI_ORACLE_LIB=str(mut_so), OMP_NUM_THREADS="2")
+    res = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                          os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                         cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert res.returncode != 0, f"pins did not catch: {name}\n{res.stdout[-2000:]}"
