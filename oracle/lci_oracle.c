@@ -22,12 +22,12 @@
  *   A2  masked top-k        ids[b,s,:] = the min(topk, vis) causal-visible blocks
  *                           with the largest scores, ranked by (score desc, block
  *                           id asc), padded with -1 (same page, section 4.1;
- *                           "scoring, Top-K, and masking" in page 1's section
- *                           "Operatorizing Index Selection").
+ *                           the score/top-k/mask combination of page 1's
+ *                           section "Operatorizing Index Selection").
  *   A3+A4 sparse attention  exact softmax attention of each query head over the
  *                           tokens of the selected blocks only, gathered from a
  *                           paged KV pool through a block table (page 2 section
- *                           4.1 "exact attention only over those positions";
+ *                           4.1, attention restricted to the chosen positions;
  *                           "Day-0 Adaptation for Trillion-Parameter MoE Models"
  *                           section IV, KV pages and the page table).
  *
@@ -309,8 +309,8 @@ int orc_sparse_attn(const void* q, const void* k_pool, const void* v_pool, int d
  * Full dense attention over every token t <= last of the sequence, with the
  * logits of tokens whose block is not among ids[r][*] set to -infinity before
  * the softmax. For distinct ids this is the same function as orc_sparse_attn,
- * written the long way round ("the sparse path and full attention must undergo
- * layer-by-layer alignment verification", page 3 section IV).
+ * written the long way round: page 3 section IV asks that the sparse path be
+ * checked against full attention.
  */
 int orc_dense_masked(const void* q, const void* k_pool, const void* v_pool, int dt,
                      int64_t B, int64_t S, int64_t H_q, int64_t H_kv, int64_t hd,

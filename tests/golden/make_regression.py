@@ -1,9 +1,9 @@
 """Write tests/golden/oracle_regression.json from the CPU oracle alone.
 
 The pages print no worked example for the index pipeline, so the stored values
-here are a regression set of the oracle itself ("Build a regression set",
-section 6 of "Day-0 Inference Adaptation of Ultra-Large-Scale MoE Models on
-Domestic AI Accelerators"): small seeded cases whose block ids and a digest of
+here are a regression set of the oracle itself (section 6 of "Day-0 Inference Adaptation of Ultra-Large-Scale MoE Models on
+Domestic AI Accelerators" recommends turning problems met into reusable test
+cases): small seeded cases whose block ids and a digest of
 the attention output must not change unless the oracle's definition changes.
 Run from the repository root:  python tests/golden/make_regression.py
 """
