@@ -1,0 +1,419 @@
+#!/usr/bin/env python
+"""Benchmark of the sparse-attention index pipeline on B200.
+
+One step = one pass of the whole hot path over one batch: index_select (block
+scoring fused with the causal-masked top-k) followed by sparse_attn (paged
+gather + exact online-softmax attention), both through the C ABI. The headline
+workload is the decode configuration (B=32 sequences, 32768-token context,
+block 64, 8 indexer heads of dim 128, top-32 blocks, 16 query heads sharing one
+KV head of dim 128, paged KV with a random-permuted block table).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N>1 runs under torchrun, one rank per GPU, each rank on its own batch of 32
+sequences (weak scaling: the sequences are independent, so no data-path
+collective). Timing: per-step CUDA events on the launching stream, the L2
+flushed (a 2x-L2 write) and the queue pre-filled (a short device sleep) before
+every step, max over ranks. Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_indexer_b200.workloads import CONFIGS, generate  # noqa: E402
+
+METRIC = "sparse-attn decode tokens/s (B=32, 32K ctx); prefill Mtok/s; % of roofline"
+HEADLINE = "decode"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default=HEADLINE, choices=sorted(CONFIGS))
+    ap.add_argument("--no-extra", action="store_true", help="skip the other configurations")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def workload_name(cfg) -> str:
+    return (f"{cfg.name} {cfg.dtype}: B={cfg.B} S={cfg.S} ctx={cfg.ctx} q_start={cfg.q_start} "
+            f"block={cfg.bs} NB={cfg.NB} H_i={cfg.H_i} d_c={cfg.d_c} topk={cfg.topk} "
+            f"H_q={cfg.H_q} H_kv={cfg.H_kv} hd={cfg.hd}")
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap"}
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = int(vis.split(",")[device_index]) if vis else device_index
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _sample(self):
+        nv = self._nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+        r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        for bit, name in self.REASONS.items():
+            if r & bit:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                return
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._nv is not None:
+            self._t.join(timeout=1.0)
+            try:
+                self._sample()  # at least one sample right at the end of the timed region
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ the path
+
+class Pipeline:
+    """Device-resident inputs of one workload and the two ABI calls of a step."""
+
+    def __init__(self, cfg, w, device):
+        import long_context_indexer_b200 as lci
+        self.lci, self.cfg = lci, cfg
+        self.host = w
+        self.d = {k: v.to(device) for k, v in w.items()}
+        d = self.d
+        self.k_c = (torch.empty((cfg.B, cfg.NB, cfg.H_i, cfg.d_c), dtype=cfg.torch_dtype,
+                                device=device) if cfg.compress else d["k_c"])
+        self.bt = lci.create_block_table(d["block_table"], d["k_pool"])
+        self.ids = torch.empty((cfg.B, cfg.S, cfg.topk), dtype=torch.int32, device=device)
+        self.out = torch.empty_like(d["q"])
+        ni = lci.index_select_workspace_size(cfg.B, cfg.S, cfg.H_i, cfg.d_c, cfg.NB, cfg.topk)
+        na = lci.sparse_attn_workspace_size(cfg.B, cfg.S, cfg.H_q, cfg.topk, self.bt)
+        self.ws_i = torch.zeros(max(ni, 256), dtype=torch.uint8, device=device)
+        self.ws_a = torch.zeros(max(na, 256), dtype=torch.uint8, device=device)
+        self.launches_per_step = (1 if cfg.compress else 0) + 2
+
+    def index(self):
+        d, c = self.d, self.cfg
+        if c.compress:
+            self.lci.block_compress(d["k_idx"], c.bs, out=self.k_c)
+        self.lci.index_select(d["q_c"], self.k_c, c.bs, d["ctx_len"], d["q_start"], c.topk,
+                              ids=self.ids, ws=self.ws_i)
+
+    def attn(self):
+        d, c = self.d, self.cfg
+        self.lci.sparse_attn(d["q"], d["k_pool"], d["v_pool"], self.bt, self.ids, d["ctx_len"],
+                             d["q_start"], out=self.out, ws=self.ws_a)
+
+    def step(self):
+        self.index()
+        self.attn()
+
+    # Algorithmic work, from the shapes and the produced ids (outside timing):
+    # every byte that must cross HBM at least once (unique k_c and KV blocks,
+    # queries, ids, outputs) and the flops of the definition.
+    def algorithmic(self):
+        c = self.cfg
+        dev = self.ids.device
+        esz = 4 if c.dtype == "f32" else 2
+        K = c.H_i * c.d_c
+        pos = self.d["q_start"].long()[:, None] + torch.arange(c.S, device=dev)[None]
+        ctx = self.d["ctx_len"].long()
+        last = torch.minimum(pos, ctx[:, None] - 1)  # [B,S]
+        vis = torch.where(last >= 0, torch.clamp(last // c.bs + 1, max=c.NB),
+                          torch.zeros_like(last))
+        rows = c.B * c.S
+        kc_unique = int(vis.max(dim=1).values.sum())  # blocks of k_c read per sequence
+        idx_bytes = rows * K * esz + kc_unique * K * esz + rows * c.topk * 4 + 8 * c.B
+        if c.compress:
+            idx_bytes += c.B * c.ctx * K * esz + c.B * c.NB * K * esz
+        ids = self.ids.long()
+        valid = ids >= 0
+        first = ids.clamp(min=0) * c.bs
+        ntok = torch.clamp(last[..., None] - first + 1, min=0, max=c.bs) * valid
+        nsel = int(ntok.sum())  # (query, token) pairs attended
+        used = torch.zeros((c.B, c.NB), dtype=torch.bool, device=dev)
+        used.scatter_(1, ids.clamp(min=0).reshape(c.B, -1), valid.reshape(c.B, -1))
+        blk_tok = torch.clamp(ctx[:, None] - torch.arange(c.NB, device=dev)[None] * c.bs, 0, c.bs)
+        kv_tokens = int((blk_tok * used).sum())  # unique KV tokens gathered
+        kv_bytes = kv_tokens * c.H_kv * c.hd * esz * 2 + int(used.sum()) * 4
+        attn_bytes = kv_bytes + 2 * rows * c.H_q * c.hd * esz + rows * c.topk * 4 + 8 * c.B
+        return {"index_bytes": idx_bytes, "attn_bytes": attn_bytes,
+                "attn_flops": 4.0 * nsel * c.H_q * c.hd, "index_flops": 2.0 * int(vis.sum()) * K,
+                "selected_pairs": nsel, "kv_tokens": kv_tokens}
+
+
+def l2_flush_buffer(device):
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    return torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=device)
+
+
+def timed_steps(pipe, steps, warmup, flush, e2e=False):
+    """Per-step device times (ms) of index, attention and the whole step."""
+    stream = torch.cuda.current_stream()
+    if e2e:
+        pin = {k: pipe.host[k].pin_memory() for k in ("q_c", "q", "ctx_len", "q_start")
+               if k in pipe.host}
+        ids_h = torch.empty(pipe.ids.shape, dtype=torch.int32).pin_memory()
+        out_h = torch.empty(pipe.out.shape, dtype=pipe.out.dtype).pin_memory()
+    evs = []
+    for i in range(warmup + steps):
+        flush.zero_()
+        torch.cuda._sleep(200_000)  # keep the device busy while the step is queued
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record(stream)
+        if e2e:
+            for k, v in pin.items():
+                pipe.d[k].copy_(v, non_blocking=True)
+        pipe.index()
+        ev[1].record(stream)
+        pipe.attn()
+        if e2e:
+            ids_h.copy_(pipe.ids, non_blocking=True)
+            out_h.copy_(pipe.out, non_blocking=True)
+        ev[2].record(stream)
+        if i >= warmup:
+            evs.append(ev)
+    torch.cuda.synchronize()
+    res_i = [e[0].elapsed_time(e[1]) for e in evs]
+    res_a = [e[1].elapsed_time(e[2]) for e in evs]
+    res_s = [e[0].elapsed_time(e[2]) for e in evs]
+    extra = {}
+    if e2e:
+        extra["h2d_bytes_per_step"] = sum(v.numel() * v.element_size() for v in pin.values())
+        extra["d2h_bytes_per_step"] = (ids_h.numel() * 4 + out_h.numel() * out_h.element_size())
+    return res_i, res_a, res_s, extra
+
+
+def measure(cfg, steps, warmup, device, rank=0, seed_offset=0, with_e2e=True):
+    w = generate(cfg, seed=cfg.seed + seed_offset)
+    pipe = Pipeline(cfg, w, device)
+    flush = l2_flush_buffer(device)
+    t_i, t_a, t_s, _ = timed_steps(pipe, steps, warmup, flush)
+    alg = pipe.algorithmic()
+    res = {"pipe": pipe, "t_index_ms": sum(t_i) / len(t_i), "t_attn_ms": sum(t_a) / len(t_a),
+           "t_step_ms": sum(t_s) / len(t_s), "t_total_ms": sum(t_s), "alg": alg}
+    if with_e2e:
+        _, _, e_s, ex = timed_steps(pipe, steps, warmup, flush, e2e=True)
+        res["e2e_total_ms"] = sum(e_s)
+        res["e2e_bytes"] = ex
+    del flush
+    return res
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def oracle_throughput(cfg, min_seconds=10.0, max_rows=None, w=None):
+    """Oracle (fp64 C, OpenMP) tokens/s on a bounded sample of the workload."""
+    import oracle
+    w = generate(cfg) if w is None else w
+    rows_all = cfg.B * cfg.S
+    n = rows_all if max_rows is None else min(rows_all, max_rows)
+    rows = list(range(n))
+    scale = 1.0 / math.sqrt(cfg.hd)
+    k_c = oracle.block_compress(w["k_idx"], cfg.bs).to(cfg.torch_dtype) if cfg.compress else w["k_c"]
+    done, t0 = 0, time.perf_counter()
+    while True:
+        ids = oracle.index_select(w["q_c"], k_c, cfg.bs, w["ctx_len"], w["q_start"], cfg.topk,
+                                  rows=rows)
+        oracle.sparse_attn(w["q"], w["k_pool"], w["v_pool"], w["block_table"], ids, w["ctx_len"],
+                           w["q_start"], scale, rows=rows)
+        done += n
+        el = time.perf_counter() - t0
+        if el >= min_seconds:
+            break
+    return {"value": done / el, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} of {rows_all} query rows of the {cfg.name} workload, repeated "
+                      f"{done // n}x over {el:.1f} s (index_select + sparse_attn, fp64)"}
+
+
+# ------------------------------------------------------------------ main
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return 0
+    cfg = CONFIGS[args.config]
+    w = generate(cfg)
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        r = oracle_throughput(cfg, min_seconds=0.0, max_rows=4, w=w)
+        if i >= args.warmup:
+            per_step.append(r)
+    rows = sum(4 for _ in per_step)
+    tok_s = statistics.median(r["value"] for r in per_step)
+    ms = 1000.0 * min(4, cfg.B * cfg.S) / tok_s
+    line = {"impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": workload_name(cfg), "sample_rows_per_step": 4},
+            "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": per_step[0]["cores"],
+                             "kind": "oracle",
+                             "sample": f"4 of {cfg.B * cfg.S} query rows per step, {rows} rows"},
+            "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    world, rank, local = dist_setup(args)
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    import long_context_indexer_b200 as lci
+    lci.load_library()
+    cfg = CONFIGS[args.config]
+    pk = peaks()
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        res = measure(cfg, args.steps, args.warmup, device, rank, seed_offset=1000 * rank)
+    torch.cuda.synchronize()
+    lci.get_device_status()
+    total_ms = torch.tensor([res["t_total_ms"], res["e2e_total_ms"]], device=device,
+                            dtype=torch.float64)
+    if world > 1:
+        dist.barrier()
+        dist.all_reduce(total_ms, op=dist.ReduceOp.MAX)
+    t_total, e_total = total_ms.tolist()
+    tokens = world * cfg.B * cfg.S * args.steps
+    value = tokens / (t_total / 1e3)
+    e2e_value = tokens / (e_total / 1e3)
+
+    alg = res["alg"]
+    kernels = {
+        "index_select": {"ms": res["t_index_ms"], "bytes": alg["index_bytes"]},
+        "sparse_attn": {"ms": res["t_attn_ms"], "bytes": alg["attn_bytes"]},
+    }
+    dom = max(kernels, key=lambda k: kernels[k]["ms"])
+    ach = kernels[dom]["bytes"] / (kernels[dom]["ms"] * 1e-3) / 1e9
+    roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": ach / pk["hbm_gbs"], "traffic": None, "peak_source": pk["source"]}
+    step_bytes = alg["index_bytes"] + alg["attn_bytes"]
+    step_gbs = step_bytes / (res["t_step_ms"] * 1e-3) / 1e9
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": workload_name(cfg), "global_batch": world * cfg.B,
+                   "seq_len": cfg.ctx, "parallelism": f"dp{world}" if world > 1 else "single",
+                   "l2": "flushed before every step (2x L2 write), per-step CUDA events"},
+        "roofline": roof,
+        "step_roofline": {"bytes": step_bytes, "achieved_gbs": step_gbs,
+                          "frac": step_gbs / pk["hbm_gbs"]},
+        "kernels_ms": {k: v["ms"] for k, v in kernels.items()},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", **res["e2e_bytes"]},
+        "gpu_launches": res["pipe"].launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_throughput(cfg, min_seconds=10.0, w=res["pipe"].host)
+    if rank == 0 and world == 1 and not args.no_extra:
+        extra = {}
+        for name in ("prefill", "long", "1m_decode", "1m_chunk", "tiny"):
+            if name == args.config:
+                continue
+            c = CONFIGS[name]
+            r = measure(c, max(5, args.steps // 5), 3, device, with_e2e=False)
+            a = r["alg"]
+            rows = c.B * c.S
+            extra[name] = {
+                "ms_step": r["t_step_ms"], "ms_index": r["t_index_ms"], "ms_attn": r["t_attn_ms"],
+                "tokens_per_s": rows / (r["t_step_ms"] * 1e-3),
+                "index_gbs": a["index_bytes"] / (r["t_index_ms"] * 1e-3) / 1e9,
+                "index_tflops": a["index_flops"] / (r["t_index_ms"] * 1e-3) / 1e12,
+                "attn_gbs": a["attn_bytes"] / (r["t_attn_ms"] * 1e-3) / 1e9,
+                "attn_tflops": a["attn_flops"] / (r["t_attn_ms"] * 1e-3) / 1e12,
+            }
+            del r
+            torch.cuda.empty_cache()
+        line["other_configs"] = extra
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

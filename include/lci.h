@@ -1,0 +1,204 @@
+/*
+ * lci.h -- C ABI of the B200 sparse-attention index pipeline (liblci.so).
+ *
+ * The library implements one layer of index-selected sparse attention for long
+ * contexts, as described by three web pages:
+ *   [GPU-stack] "Day-0 Inference Adaptation for Ultra-Large MoE Models on
+ *               Domestic GPUs: A Software Stack Perspective"
+ *   [AI-acc]    "Day-0 Inference Adaptation of Ultra-Large-Scale MoE Models on
+ *               Domestic AI Accelerators"
+ *   [Hetero]    "Day-0 Adaptation for Trillion-Parameter MoE Models: A
+ *               Comprehensive Guide to Heterogeneous Compute Deployment"
+ *
+ * Pipeline: compressed block keys k_c are scored against compressed queries
+ * q_c (summed over indexer heads), every query keeps the top-k causal-visible
+ * blocks, and exact softmax attention runs over the tokens of those blocks,
+ * gathered from a paged KV pool through a block table. Prefill (many queries
+ * per sequence) and decode (one query per sequence) share one representation:
+ * int32 block ids in rank order plus the block table.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers named d_* and all tensor arguments are DEVICE pointers on the
+ *   current CUDA device; the caller allocates and owns them. The library keeps
+ *   no reference to them after a call returns (except the block table object,
+ *   which records the table pointer it is given; see below).
+ * - Layouts are dense row-major, innermost index last, with no padding.
+ *   Floating tensors of one call share one element type (lci_dtype).
+ * - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *   stream. Every launch is asynchronous on it. No entry point synchronises,
+ *   except lci_get_device_status.
+ * - Host-detectable argument errors return a status before anything is
+ *   launched; lci_last_error() then describes the problem. Launch calls make
+ *   no device allocation: scratch memory is the caller's workspace.
+ * - Device-side checks (block ids outside [-1, nb_max), table entries outside
+ *   [0, num_pages)) never trap: the offending item is skipped, a sticky device
+ *   status word is set, and lci_get_device_status reports it.
+ * - Query position: p = d_q_start[b] + s for query s of sequence b. The last
+ *   attendable token is last = min(p, d_ctx_len[b] - 1). Block j is causal-
+ *   visible when j * block_size <= last (so vis = min(nb_max, last/bs + 1)).
+ */
+#ifndef LCI_H
+#define LCI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LCI_API __attribute__((visibility("default")))
+#else
+#define LCI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LCI_OK = 0,
+    LCI_ERR_INVALID_ARG = 1,   /* null pointer, bad size or inconsistent shapes */
+    LCI_ERR_UNSUPPORTED = 2,   /* valid arguments outside what the kernels cover */
+    LCI_ERR_WORKSPACE = 3,     /* workspace missing, misaligned or too small */
+    LCI_ERR_CUDA = 4,          /* a CUDA runtime call failed (see lci_last_error) */
+    LCI_ERR_DEVICE_BOUNDS = 5, /* a device-side bounds check fired (sticky word) */
+    LCI_ERR_TIMEOUT = 6        /* reserved: a bounded device wait gave up */
+} lci_status;
+
+typedef enum { LCI_F32 = 0, LCI_BF16 = 1 } lci_dtype;
+
+/* Which kernel family runs. AUTO: DECODE when S == 1, PREFILL otherwise.
+ * Both produce identical block ids for identical inputs ([GPU-stack],
+ * "Separate Paths for Prefill and Decode": two schedules, one representation). */
+typedef enum { LCI_PHASE_AUTO = 0, LCI_PHASE_PREFILL = 1, LCI_PHASE_DECODE = 2 } lci_phase;
+
+typedef struct lci_block_table lci_block_table; /* opaque, host-side */
+
+/* Library version string ("major.minor.patch"). */
+LCI_API const char* lci_version(void);
+
+/* Static description of a status code. */
+LCI_API const char* lci_status_string(lci_status status);
+
+/* Message of the last failing call on this host thread ("" when none). */
+LCI_API const char* lci_last_error(void);
+
+/*
+ * Block table of a paged KV cache ([GPU-stack] "Reorganizing KV Cache Layout";
+ * [Hetero] §II and §IV, KV pages addressed through a page table).
+ *
+ *   d_table      [batch][max_blocks] int32, device. Entry (b, j) is the pool
+ *                page that holds logical block j (tokens j*block_size ..
+ *                (j+1)*block_size-1) of sequence b. The object records this
+ *                pointer without copying; the caller keeps the memory alive and
+ *                may update its contents between calls.
+ *   num_pages    pages in each KV pool.
+ *   block_size   tokens per page.
+ *   num_kv_heads, head_dim, kv_dtype: shape and type of the pools
+ *                K, V = [num_pages][num_kv_heads][block_size][head_dim].
+ * Allocates only the host object. Returns LCI_ERR_INVALID_ARG on a null
+ * pointer or a non-positive size.
+ */
+LCI_API lci_status lci_create_block_table(const int32_t* d_table, int32_t batch, int32_t max_blocks,
+                                  int32_t num_pages, int32_t block_size, int32_t num_kv_heads,
+                                  int32_t head_dim, lci_dtype kv_dtype, lci_block_table** out);
+
+/* Frees the host object (never the caller's table memory). NULL is a no-op. */
+LCI_API lci_status lci_destroy_block_table(lci_block_table* table);
+
+/*
+ * Bounds-checks every table entry against [0, num_pages) on the device.
+ * Violations set the sticky device status word (see lci_get_device_status).
+ */
+LCI_API lci_status lci_validate_block_table(const lci_block_table* table, void* stream);
+
+/*
+ * A0 -- block compression ([GPU-stack] "Adapting Sparse Attention", the
+ * representation-generation stage; [AI-acc] §4.1, k_comp):
+ *   k_c[b][j][h][d] = mean over the tokens t of block j of k_idx[b][t][h][d]
+ * with block j = tokens [j*block_size, min(tokens, (j+1)*block_size)).
+ *   k_idx  [batch][tokens][heads][dim], device, dtype
+ *   k_c    [batch][ceil(tokens/block_size)][heads][dim], device, dtype (output)
+ * Sums in fp32, divides by the token count, rounds once to dtype.
+ */
+LCI_API lci_status lci_block_compress(const void* k_idx, lci_dtype dtype, int32_t batch, int32_t tokens,
+                              int32_t heads, int32_t dim, int32_t block_size, void* k_c,
+                              void* stream);
+
+/*
+ * Workspace bytes lci_index_select needs for these sizes (0 is possible).
+ */
+LCI_API lci_status lci_index_select_workspace_size(int32_t batch, int32_t S, int32_t H_i, int32_t d_c,
+                                           int32_t nb_max, int32_t topk, lci_phase phase,
+                                           size_t* bytes);
+
+/*
+ * A1 + A2 -- block scoring fused with the causal-masked top-k
+ * ([GPU-stack] "Operatorizing Index Selection": scoring, top-k and masking in
+ * one operator; [AI-acc] §4.1, matmul of compressed queries and keys followed
+ * by an on-device top-k that avoids a full sort):
+ *   score[b][s][j] = sum_h sum_d q_c[b][s][h][d] * k_c[b][j][h][d]   (j < vis)
+ *   d_ids[b][s][0 .. min(topk, vis)) = visible block ids ranked by
+ *       (score descending, block id ascending); the rest of the row is -1.
+ *   q_c        [batch][S][H_i][d_c], device, dtype
+ *   k_c        [batch][nb_max][H_i][d_c], device, dtype
+ *   d_ctx_len  [batch] int32, d_q_start [batch] int32, device
+ *   d_ids      [batch][S][topk] int32, device (output)
+ *   workspace  >= lci_index_select_workspace_size bytes, 256-byte aligned.
+ *              Its first bytes hold arrival counters that must be zero before
+ *              the first call; every call leaves them zero again. Calls that
+ *              share a workspace must not overlap in time.
+ * Scores are accumulated in fp32. Limits: 1 <= topk <= 256,
+ * nb_max <= 16384, H_i*d_c <= 8192 and a multiple of 8 (bf16) or 4 (f32).
+ */
+LCI_API lci_status lci_index_select(const void* q_c, const void* k_c, lci_dtype dtype, int32_t batch,
+                            int32_t S, int32_t H_i, int32_t d_c, int32_t block_size,
+                            int32_t nb_max, const int32_t* d_ctx_len, const int32_t* d_q_start,
+                            int32_t topk, lci_phase phase, int32_t* d_ids, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/*
+ * Workspace bytes lci_sparse_attn needs for these sizes (0 is possible).
+ */
+LCI_API lci_status lci_sparse_attn_workspace_size(int32_t batch, int32_t S, int32_t H_q, int32_t topk,
+                                          const lci_block_table* table, lci_phase phase,
+                                          size_t* bytes);
+
+/*
+ * A3 + A4 -- paged gather and exact sparse attention ([AI-acc] §4.1, exact
+ * attention over the selected positions only; [Hetero] §IV, gather of the
+ * selected KV pages, then a compute-heavy prefill or memory-heavy decode
+ * kernel). For query head h (KV head g = h / (H_q / num_kv_heads)):
+ *   T   = { t : t / block_size is one of d_ids[b][s][*], t <= last }
+ *   out = sum_{t in T} softmax_t(scale * q . K_t) V_t ,  K_t, V_t read at
+ *         pool[table[b][t / block_size]][g][t % block_size][:]
+ * An empty T gives a zero row. Rows of d_ids may be in any order, may hold -1
+ * entries anywhere, and must not repeat a block.
+ *   q        [batch][S][H_q][head_dim], device, dtype = the table's kv_dtype
+ *   k_pool, v_pool  [num_pages][num_kv_heads][block_size][head_dim], device
+ *   d_ids    [batch][S][topk] int32, device
+ *   scale    softmax scale; <= 0 selects 1/sqrt(head_dim)
+ *   out      [batch][S][H_q][head_dim], device, dtype (output)
+ *   workspace >= lci_sparse_attn_workspace_size bytes, 256-byte aligned; same
+ *             zero-on-first-use counter rule as lci_index_select.
+ * Softmax and accumulation are fp32; bf16 inputs feed the tensor cores.
+ * Limits: H_q a multiple of num_kv_heads, head_dim a multiple of 32 and
+ * <= 256, topk <= 256.
+ */
+LCI_API lci_status lci_sparse_attn(const void* q, int32_t batch, int32_t S, int32_t H_q,
+                           const void* k_pool, const void* v_pool, const lci_block_table* table,
+                           const int32_t* d_ids, int32_t topk, const int32_t* d_ctx_len,
+                           const int32_t* d_q_start, float scale, lci_phase phase, void* out,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the sticky device status
+ * word of the current device: LCI_OK, or LCI_ERR_DEVICE_BOUNDS when a device
+ * bounds check fired since the last call.
+ */
+LCI_API lci_status lci_get_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LCI_H */

@@ -1,0 +1,13 @@
+"""lci -- B200-native sparse-attention index pipeline.
+
+The CUDA library is ``liblci.so`` (C ABI in ``include/lci.h``); ``lci`` is its
+thin ctypes binding and ``workloads`` the seeded synthetic input generator.
+Importing the package loads nothing; the library is loaded on first use.
+"""
+from .lci import (BlockTable, LciError, block_compress, create_block_table, get_device_status,
+                  index_select, index_select_workspace_size, load_library, sparse_attn,
+                  sparse_attn_workspace_size, version)
+
+__all__ = ["BlockTable", "LciError", "block_compress", "create_block_table", "get_device_status",
+           "index_select", "index_select_workspace_size", "load_library", "sparse_attn",
+           "sparse_attn_workspace_size", "version"]

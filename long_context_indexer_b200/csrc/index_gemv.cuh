@@ -1,0 +1,91 @@
+// index_gemv.cuh -- block scoring fused with the causal-masked top-k, one query
+// row at a time (the decode schedule; also the generic path for any S).
+//
+// Grid (rows, chunks). Each CTA scores one chunk of the row's causal-visible
+// blocks: k_c rows stream from HBM with 16-byte loads, every warp dots them
+// against the query row staged in shared memory and reduces with shuffles. The
+// fp32 scores go to the workspace (L2-resident, 4 bytes per 2 KiB block key).
+// The last CTA of the row to arrive (atomic counter, no spin-wait) runs the
+// exact CTA radix select over the row's scores and writes the block ids, then
+// resets the counter for the next call.
+#pragma once
+
+#include "common.cuh"
+#include "topk_select.cuh"
+
+namespace lci {
+
+template <typename T> struct ElemsPer16B;
+template <> struct ElemsPer16B<float> { static constexpr int v = 4; };
+template <> struct ElemsPer16B<__nv_bfloat16> { static constexpr int v = 8; };
+
+__device__ __forceinline__ float dot_chunk(const uint4& raw, const float* q, float) {
+    return __uint_as_float(raw.x) * q[0] + __uint_as_float(raw.y) * q[1] +
+           __uint_as_float(raw.z) * q[2] + __uint_as_float(raw.w) * q[3];
+}
+
+__device__ __forceinline__ float dot_chunk(const uint4& raw, const float* q, __nv_bfloat16) {
+    const float2 a = bf16x2_to_f32(raw.x), b = bf16x2_to_f32(raw.y);
+    const float2 c = bf16x2_to_f32(raw.z), d = bf16x2_to_f32(raw.w);
+    return a.x * q[0] + a.y * q[1] + b.x * q[2] + b.y * q[3] + c.x * q[4] + c.y * q[5] +
+           d.x * q[6] + d.y * q[7];
+}
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+template <typename T, int NT>
+__global__ void __launch_bounds__(NT) index_gemv_select_kernel(
+    const T* __restrict__ q_c, const T* __restrict__ k_c, int S, int K, int nb_max, int bs,
+    const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ q_start, int topk,
+    int chunk_blocks, int nchunks, float* __restrict__ scores,
+    unsigned int* __restrict__ counters, int32_t* __restrict__ ids) {
+    extern __shared__ __align__(16) unsigned char dyn_smem[];
+    __shared__ SelectSmem sel;
+    __shared__ int s_last;
+    constexpr int NW = NT / 32;
+    constexpr int E = ElemsPer16B<T>::v;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int row = blockIdx.x, chunk = blockIdx.y;
+    const int b = row / S, s = row - b * S;
+    const long long p = (long long)__ldg(&q_start[b]) + s;
+    const int vis = visible_blocks(p, __ldg(&ctx_len[b]), bs, nb_max);
+    const int j0 = chunk * chunk_blocks;
+    const int j1 = min(j0 + chunk_blocks, vis);
+
+    if (j0 < j1) {
+        float* qs = reinterpret_cast<float*>(dyn_smem);
+        const T* qrow = q_c + (size_t)row * K;
+        for (int i = tid; i < K; i += NT) qs[i] = to_f32(qrow[i]);
+        __syncthreads();
+        const int nvec = K / E;
+        for (int j = j0 + warp; j < j1; j += NW) {
+            const uint4* kr = reinterpret_cast<const uint4*>(k_c + ((size_t)b * nb_max + j) * K);
+            float acc = 0.f;
+            for (int c = lane; c < nvec; c += 32) acc += dot_chunk(ld_stream(kr + c), qs + c * E, T());
+            acc = warp_sum(acc);
+            if (lane == 0) scores[(size_t)row * nb_max + j] = acc;
+        }
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        const unsigned prev = atomicAdd(&counters[row], 1u);
+        s_last = (prev == (unsigned)(nchunks - 1));
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    if (tid == 0) counters[row] = 0u;
+    uint32_t* keys = reinterpret_cast<uint32_t*>(dyn_smem);
+    for (int i = tid; i < vis; i += NT) keys[i] = score_key(__ldcg(&scores[(size_t)row * nb_max + i]));
+    __syncthreads();
+    cta_topk_from_keys<NT>(keys, vis, topk, ids + (size_t)row * topk, sel);
+}
+
+}  // namespace lci

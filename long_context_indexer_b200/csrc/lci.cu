@@ -1,0 +1,344 @@
+// lci.cu -- C ABI of the sparse-attention index pipeline (see include/lci.h).
+//
+// Host side only: argument checks, workspace layout, kernel selection and
+// launches. Every step of the computation runs in the kernels included below.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <new>
+#include <string>
+
+#include "../../include/lci.h"
+#include "attn_simt.cuh"
+#include "common.cuh"
+#include "compress.cuh"
+#include "index_gemv.cuh"
+#include "topk_select.cuh"
+
+struct lci_block_table {
+    const int32_t* d_table;
+    int32_t batch, max_blocks, num_pages, block_size, num_kv_heads, head_dim;
+    lci_dtype dtype;
+};
+
+namespace {
+
+thread_local std::string t_last_error;
+
+lci_status fail(lci_status st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    t_last_error = buf;
+    return st;
+}
+
+lci_status ok() {
+    t_last_error.clear();
+    return LCI_OK;
+}
+
+lci_status check_launch(const char* what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(LCI_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return ok();
+}
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool dtype_ok(lci_dtype d) { return d == LCI_F32 || d == LCI_BF16; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+lci_phase resolve_phase(lci_phase ph, int32_t S) {
+    if (ph == LCI_PHASE_AUTO) return S == 1 ? LCI_PHASE_DECODE : LCI_PHASE_PREFILL;
+    return ph;
+}
+
+// ------------------------------------------------------------ index_select
+
+constexpr int kIndexThreads = 256;
+constexpr int kMaxNbMax = 16384;
+constexpr int kMaxIndexK = 8192;
+
+struct IndexPlan {
+    int chunk_blocks, nchunks;
+    size_t off_counters, off_scores, bytes;
+    size_t smem;
+};
+
+IndexPlan plan_index(int32_t batch, int32_t S, int32_t K, int32_t nb_max) {
+    IndexPlan pl{};
+    const long long rows = (long long)batch * S;
+    // Enough CTAs to cover the 148 SMs several times over, chunks of 8..32 blocks.
+    int chunk = 32;
+    while (chunk > 8 && rows * ((nb_max + chunk - 1) / chunk) < 4 * 148) chunk >>= 1;
+    pl.chunk_blocks = chunk;
+    pl.nchunks = (nb_max + chunk - 1) / chunk;
+    pl.off_counters = 0;
+    pl.off_scores = align_up((size_t)rows * sizeof(unsigned int));
+    pl.bytes = pl.off_scores + align_up((size_t)rows * nb_max * sizeof(float));
+    const size_t qbytes = (size_t)K * sizeof(float);
+    const size_t kbytes = (size_t)nb_max * sizeof(uint32_t);
+    pl.smem = qbytes > kbytes ? qbytes : kbytes;
+    return pl;
+}
+
+lci_status check_index_args(int32_t batch, int32_t S, int32_t H_i, int32_t d_c, int32_t nb_max,
+                            int32_t topk, lci_dtype dtype) {
+    if (batch <= 0 || S <= 0 || H_i <= 0 || d_c <= 0 || nb_max <= 0)
+        return fail(LCI_ERR_INVALID_ARG, "index_select: sizes must be positive "
+                    "(batch=%d S=%d H_i=%d d_c=%d nb_max=%d)", batch, S, H_i, d_c, nb_max);
+    if (topk <= 0) return fail(LCI_ERR_INVALID_ARG, "index_select: topk must be positive (%d)", topk);
+    if (!dtype_ok(dtype)) return fail(LCI_ERR_INVALID_ARG, "index_select: unknown dtype %d", (int)dtype);
+    if (topk > lci::kMaxTopk)
+        return fail(LCI_ERR_UNSUPPORTED, "index_select: topk %d above %d", topk, lci::kMaxTopk);
+    if (nb_max > kMaxNbMax)
+        return fail(LCI_ERR_UNSUPPORTED, "index_select: nb_max %d above %d", nb_max, kMaxNbMax);
+    const long long K = (long long)H_i * d_c;
+    const int vec = dtype == LCI_BF16 ? 8 : 4;
+    if (K > kMaxIndexK || K % vec != 0)
+        return fail(LCI_ERR_UNSUPPORTED, "index_select: H_i*d_c=%lld must be <= %d and a multiple "
+                    "of %d", K, kMaxIndexK, vec);
+    return LCI_OK;
+}
+
+template <typename T>
+lci_status launch_index_gemv(const void* q_c, const void* k_c, int32_t batch, int32_t S, int32_t K,
+                             int32_t bs, int32_t nb_max, const int32_t* ctx_len,
+                             const int32_t* q_start, int32_t topk, int32_t* ids, void* ws,
+                             const IndexPlan& pl, cudaStream_t st) {
+    auto kern = lci::index_gemv_select_kernel<T, kIndexThreads>;
+    if (pl.smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)pl.smem);
+        if (e != cudaSuccess) return fail(LCI_ERR_CUDA, "index_select: %s", cudaGetErrorString(e));
+    }
+    char* w = static_cast<char*>(ws);
+    dim3 grid((unsigned)(batch * S), (unsigned)pl.nchunks);
+    kern<<<grid, kIndexThreads, pl.smem, st>>>(
+        static_cast<const T*>(q_c), static_cast<const T*>(k_c), S, K, nb_max, bs, ctx_len, q_start,
+        topk, pl.chunk_blocks, pl.nchunks, reinterpret_cast<float*>(w + pl.off_scores),
+        reinterpret_cast<unsigned int*>(w + pl.off_counters), ids);
+    return check_launch("index_select");
+}
+
+// ------------------------------------------------------------ sparse_attn
+
+lci_status check_attn_args(int32_t batch, int32_t S, int32_t H_q, const lci_block_table* t,
+                           int32_t topk) {
+    if (!t) return fail(LCI_ERR_INVALID_ARG, "sparse_attn: null block table");
+    if (batch <= 0 || S <= 0 || H_q <= 0 || topk <= 0)
+        return fail(LCI_ERR_INVALID_ARG, "sparse_attn: sizes must be positive (batch=%d S=%d H_q=%d "
+                    "topk=%d)", batch, S, H_q, topk);
+    if (batch > t->batch)
+        return fail(LCI_ERR_INVALID_ARG, "sparse_attn: batch %d exceeds the table's %d", batch,
+                    t->batch);
+    if (H_q % t->num_kv_heads != 0)
+        return fail(LCI_ERR_INVALID_ARG, "sparse_attn: H_q %d not a multiple of num_kv_heads %d",
+                    H_q, t->num_kv_heads);
+    if (topk > lci::kMaxTopk)
+        return fail(LCI_ERR_UNSUPPORTED, "sparse_attn: topk %d above %d", topk, lci::kMaxTopk);
+    if (t->head_dim % 32 != 0 || t->head_dim > 32 * lci::kSimtMaxHdPerLane)
+        return fail(LCI_ERR_UNSUPPORTED, "sparse_attn: head_dim %d must be a multiple of 32 and "
+                    "<= %d", t->head_dim, 32 * lci::kSimtMaxHdPerLane);
+    return LCI_OK;
+}
+
+template <typename T>
+lci_status launch_attn_simt(const void* q, int32_t batch, int32_t S, int32_t H_q,
+                            const void* k_pool, const void* v_pool, const lci_block_table* t,
+                            const int32_t* ids, int32_t topk, const int32_t* ctx_len,
+                            const int32_t* q_start, float scale, void* out, cudaStream_t st) {
+    const int G = H_q / t->num_kv_heads;
+    const int warps = G < 16 ? G : 16;
+    dim3 grid((unsigned)(batch * S), (unsigned)t->num_kv_heads);
+    const float scale_log2 = scale * 1.4426950408889634f;
+    lci::sparse_attn_simt_kernel<T><<<grid, warps * 32, 0, st>>>(
+        static_cast<const T*>(q), static_cast<const T*>(k_pool), static_cast<const T*>(v_pool),
+        t->d_table, t->max_blocks, t->num_pages, t->num_kv_heads, t->block_size, t->head_dim, S,
+        H_q, ids, topk, ctx_len, q_start, scale_log2, static_cast<T*>(out));
+    return check_launch("sparse_attn");
+}
+
+__global__ void validate_table_kernel(const int32_t* __restrict__ table, long long n,
+                                      int num_pages) {
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int v = table[i];
+        if (v < 0 || v >= num_pages) lci::raise_status(lci::kStatusBadPage);
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lci_version(void) { return "0.1.0"; }
+
+const char* lci_status_string(lci_status s) {
+    switch (s) {
+        case LCI_OK: return "ok";
+        case LCI_ERR_INVALID_ARG: return "invalid argument";
+        case LCI_ERR_UNSUPPORTED: return "unsupported configuration";
+        case LCI_ERR_WORKSPACE: return "workspace missing or too small";
+        case LCI_ERR_CUDA: return "CUDA error";
+        case LCI_ERR_DEVICE_BOUNDS: return "device bounds check fired";
+        case LCI_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+const char* lci_last_error(void) { return t_last_error.c_str(); }
+
+lci_status lci_create_block_table(const int32_t* d_table, int32_t batch, int32_t max_blocks,
+                                  int32_t num_pages, int32_t block_size, int32_t num_kv_heads,
+                                  int32_t head_dim, lci_dtype kv_dtype, lci_block_table** out) {
+    if (!out) return fail(LCI_ERR_INVALID_ARG, "create_block_table: null output pointer");
+    *out = nullptr;
+    if (!d_table) return fail(LCI_ERR_INVALID_ARG, "create_block_table: null table pointer");
+    if (batch <= 0 || max_blocks <= 0 || num_pages <= 0 || block_size <= 0 || num_kv_heads <= 0 ||
+        head_dim <= 0)
+        return fail(LCI_ERR_INVALID_ARG, "create_block_table: sizes must be positive");
+    if (!dtype_ok(kv_dtype)) return fail(LCI_ERR_INVALID_ARG, "create_block_table: unknown dtype");
+    lci_block_table* t = new (std::nothrow) lci_block_table;
+    if (!t) return fail(LCI_ERR_INVALID_ARG, "create_block_table: host allocation failed");
+    *t = lci_block_table{d_table, batch, max_blocks, num_pages, block_size, num_kv_heads, head_dim,
+                         kv_dtype};
+    *out = t;
+    return ok();
+}
+
+lci_status lci_destroy_block_table(lci_block_table* table) {
+    delete table;
+    return ok();
+}
+
+lci_status lci_validate_block_table(const lci_block_table* t, void* stream) {
+    if (!t) return fail(LCI_ERR_INVALID_ARG, "validate_block_table: null table");
+    const long long n = (long long)t->batch * t->max_blocks;
+    const int blocks = (int)((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184);
+    validate_table_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(t->d_table, n,
+                                                                                  t->num_pages);
+    return check_launch("validate_block_table");
+}
+
+lci_status lci_block_compress(const void* k_idx, lci_dtype dtype, int32_t batch, int32_t tokens,
+                              int32_t heads, int32_t dim, int32_t block_size, void* k_c,
+                              void* stream) {
+    if (!k_idx || !k_c) return fail(LCI_ERR_INVALID_ARG, "block_compress: null pointer");
+    if (batch <= 0 || tokens <= 0 || heads <= 0 || dim <= 0 || block_size <= 0)
+        return fail(LCI_ERR_INVALID_ARG, "block_compress: sizes must be positive");
+    if (!dtype_ok(dtype)) return fail(LCI_ERR_INVALID_ARG, "block_compress: unknown dtype");
+    const int NB = (tokens + block_size - 1) / block_size;
+    const int HD = heads * dim;
+    const long long total = (long long)batch * NB * HD;
+    const int threads = 256;
+    const long long want = (total + threads - 1) / threads;
+    const int blocks = (int)(want < 148 * 16 ? want : 148 * 16);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dtype == LCI_F32)
+        lci::block_compress_kernel<float><<<blocks, threads, 0, st>>>(
+            static_cast<const float*>(k_idx), batch, tokens, HD, block_size, NB,
+            static_cast<float*>(k_c));
+    else
+        lci::block_compress_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(k_idx), batch, tokens, HD, block_size, NB,
+            static_cast<__nv_bfloat16*>(k_c));
+    return check_launch("block_compress");
+}
+
+lci_status lci_index_select_workspace_size(int32_t batch, int32_t S, int32_t H_i, int32_t d_c,
+                                           int32_t nb_max, int32_t topk, lci_phase phase,
+                                           size_t* bytes) {
+    if (!bytes) return fail(LCI_ERR_INVALID_ARG, "index_select_workspace_size: null output");
+    lci_status st = check_index_args(batch, S, H_i, d_c, nb_max, topk, LCI_BF16);
+    if (st != LCI_OK && st != LCI_ERR_UNSUPPORTED) return st;
+    (void)phase;
+    *bytes = plan_index(batch, S, H_i * d_c, nb_max).bytes;
+    return ok();
+}
+
+lci_status lci_index_select(const void* q_c, const void* k_c, lci_dtype dtype, int32_t batch,
+                            int32_t S, int32_t H_i, int32_t d_c, int32_t block_size,
+                            int32_t nb_max, const int32_t* d_ctx_len, const int32_t* d_q_start,
+                            int32_t topk, lci_phase phase, int32_t* d_ids, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+    if (!q_c || !k_c || !d_ctx_len || !d_q_start || !d_ids)
+        return fail(LCI_ERR_INVALID_ARG, "index_select: null pointer argument");
+    if (block_size <= 0) return fail(LCI_ERR_INVALID_ARG, "index_select: block_size must be positive");
+    lci_status st = check_index_args(batch, S, H_i, d_c, nb_max, topk, dtype);
+    if (st != LCI_OK) return st;
+    if (phase != LCI_PHASE_AUTO && phase != LCI_PHASE_PREFILL && phase != LCI_PHASE_DECODE)
+        return fail(LCI_ERR_INVALID_ARG, "index_select: unknown phase %d", (int)phase);
+    if (!aligned16(q_c) || !aligned16(k_c))
+        return fail(LCI_ERR_INVALID_ARG, "index_select: q_c and k_c must be 16-byte aligned");
+    const int K = H_i * d_c;
+    const IndexPlan pl = plan_index(batch, S, K, nb_max);
+    if (!workspace || workspace_bytes < pl.bytes ||
+        (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+        return fail(LCI_ERR_WORKSPACE, "index_select: workspace needs %zu bytes, 256-byte aligned "
+                    "(got %zu at %p)", pl.bytes, workspace_bytes, workspace);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    (void)resolve_phase(phase, S);
+    if (dtype == LCI_F32)
+        return launch_index_gemv<float>(q_c, k_c, batch, S, K, block_size, nb_max, d_ctx_len,
+                                        d_q_start, topk, d_ids, workspace, pl, cs);
+    return launch_index_gemv<__nv_bfloat16>(q_c, k_c, batch, S, K, block_size, nb_max, d_ctx_len,
+                                            d_q_start, topk, d_ids, workspace, pl, cs);
+}
+
+lci_status lci_sparse_attn_workspace_size(int32_t batch, int32_t S, int32_t H_q, int32_t topk,
+                                          const lci_block_table* table, lci_phase phase,
+                                          size_t* bytes) {
+    if (!bytes) return fail(LCI_ERR_INVALID_ARG, "sparse_attn_workspace_size: null output");
+    lci_status st = check_attn_args(batch, S, H_q, table, topk);
+    if (st != LCI_OK) return st;
+    (void)phase;
+    *bytes = 0;
+    return ok();
+}
+
+lci_status lci_sparse_attn(const void* q, int32_t batch, int32_t S, int32_t H_q,
+                           const void* k_pool, const void* v_pool, const lci_block_table* table,
+                           const int32_t* d_ids, int32_t topk, const int32_t* d_ctx_len,
+                           const int32_t* d_q_start, float scale, lci_phase phase, void* out,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+    if (!q || !k_pool || !v_pool || !d_ids || !d_ctx_len || !d_q_start || !out)
+        return fail(LCI_ERR_INVALID_ARG, "sparse_attn: null pointer argument");
+    lci_status st = check_attn_args(batch, S, H_q, table, topk);
+    if (st != LCI_OK) return st;
+    if (phase != LCI_PHASE_AUTO && phase != LCI_PHASE_PREFILL && phase != LCI_PHASE_DECODE)
+        return fail(LCI_ERR_INVALID_ARG, "sparse_attn: unknown phase %d", (int)phase);
+    if (!(scale > 0.f)) scale = 1.0f / std::sqrt((float)table->head_dim);
+    if (!std::isfinite(scale)) return fail(LCI_ERR_INVALID_ARG, "sparse_attn: non-finite scale");
+    (void)workspace;
+    (void)workspace_bytes;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (table->dtype == LCI_F32)
+        return launch_attn_simt<float>(q, batch, S, H_q, k_pool, v_pool, table, d_ids, topk,
+                                       d_ctx_len, d_q_start, scale, out, cs);
+    return launch_attn_simt<__nv_bfloat16>(q, batch, S, H_q, k_pool, v_pool, table, d_ids, topk,
+                                           d_ctx_len, d_q_start, scale, out, cs);
+}
+
+lci_status lci_get_device_status(void* stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(LCI_ERR_CUDA, "get_device_status: %s", cudaGetErrorString(e));
+    unsigned int v = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&v, lci::g_device_status, sizeof v);
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(lci::g_device_status, &zero, sizeof zero);
+    if (e != cudaSuccess) return fail(LCI_ERR_CUDA, "get_device_status: %s", cudaGetErrorString(e));
+    if (v != 0)
+        return fail(LCI_ERR_DEVICE_BOUNDS, "device bounds check fired (flags 0x%x:%s%s)", v,
+                    (v & lci::kStatusBadBlockId) ? " block id" : "",
+                    (v & lci::kStatusBadPage) ? " page" : "");
+    return ok();
+}
+
+}  // extern "C"

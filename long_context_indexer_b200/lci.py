@@ -1,0 +1,270 @@
+"""Thin Python binding of liblci.so (include/lci.h).
+
+Argument marshalling only: every function checks the torch tensors it is given
+(device, dtype, contiguity, shapes), takes their device pointers and the
+current CUDA stream, and calls the C entry point of the same name. Outputs and
+workspaces are torch allocations; the computation runs entirely in the
+library's CUDA kernels. There is no fallback: if liblci.so is missing or fails
+to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Dict, Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "liblci.so")
+
+LCI_OK = 0
+STATUS_NAMES = {0: "LCI_OK", 1: "LCI_ERR_INVALID_ARG", 2: "LCI_ERR_UNSUPPORTED",
+                3: "LCI_ERR_WORKSPACE", 4: "LCI_ERR_CUDA", 5: "LCI_ERR_DEVICE_BOUNDS",
+                6: "LCI_ERR_TIMEOUT"}
+LCI_F32, LCI_BF16 = 0, 1
+PHASES = {"auto": 0, "prefill": 1, "decode": 2}
+
+# Every entry point of include/lci.h: name -> (restype, argtypes)
+_vp, _i32, _sz, _f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_float
+_st = ctypes.c_int
+SIGNATURES = {
+    "lci_version": (ctypes.c_char_p, []),
+    "lci_status_string": (ctypes.c_char_p, [_st]),
+    "lci_last_error": (ctypes.c_char_p, []),
+    "lci_create_block_table": (_st, [_vp, _i32, _i32, _i32, _i32, _i32, _i32, _st,
+                                     ctypes.POINTER(_vp)]),
+    "lci_destroy_block_table": (_st, [_vp]),
+    "lci_validate_block_table": (_st, [_vp, _vp]),
+    "lci_block_compress": (_st, [_vp, _st, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
+    "lci_index_select_workspace_size": (_st, [_i32, _i32, _i32, _i32, _i32, _i32, _st,
+                                              ctypes.POINTER(_sz)]),
+    "lci_index_select": (_st, [_vp, _vp, _st, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _i32,
+                               _st, _vp, _vp, _sz, _vp]),
+    "lci_sparse_attn_workspace_size": (_st, [_i32, _i32, _i32, _i32, _vp, _st,
+                                             ctypes.POINTER(_sz)]),
+    "lci_sparse_attn": (_st, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _f32,
+                              _st, _vp, _vp, _sz, _vp]),
+    "lci_get_device_status": (_st, [_vp]),
+}
+
+_lib = None
+_lock = threading.Lock()
+
+
+class LciError(RuntimeError):
+    def __init__(self, status: int, where: str, message: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {message}")
+
+
+def load_library() -> ctypes.CDLL:
+    """Load liblci.so (built by long_context_indexer_b200.build); raise if absent."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"liblci.so not found at {LIB_PATH}; build it with "
+                                   "`python -m long_context_indexer_b200.build`")
+            lib = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def _check(status: int, where: str) -> None:
+    if status != LCI_OK:
+        msg = load_library().lci_last_error().decode(errors="replace")
+        raise LciError(status, where, msg)
+
+
+def version() -> str:
+    return load_library().lci_version().decode()
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return LCI_F32
+    if t.dtype == torch.bfloat16:
+        return LCI_BF16
+    raise TypeError(f"lci: unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _dev(t: torch.Tensor, name: str, dtype: Optional[torch.dtype] = None, ndim: Optional[int] = None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"lci: {name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"lci: {name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"lci: {name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"lci: {name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"lci: {name} must have {ndim} dims, got {t.dim()}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+# ---------------------------------------------------------------- workspaces
+
+_ws: Dict[Tuple[int, str], torch.Tensor] = {}
+
+
+def workspace(device: torch.device, nbytes: int, tag: str) -> torch.Tensor:
+    """A zero-initialised, 256-byte aligned device buffer of at least nbytes.
+
+    The library keeps the counter region of a workspace at zero between calls,
+    so a buffer is zero-filled once, when it is first allocated or grown.
+    """
+    key = (torch.device(device).index or 0, tag)
+    buf = _ws.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+        _ws[key] = buf
+    return buf
+
+
+# ---------------------------------------------------------------- block table
+
+class BlockTable:
+    """Owns an lci_block_table handle; keeps the table tensor alive."""
+
+    def __init__(self, table: torch.Tensor, num_pages: int, block_size: int, num_kv_heads: int,
+                 head_dim: int, dtype: torch.dtype):
+        ptr = _dev(table, "block_table", torch.int32, 2)
+        self.table = table
+        self.batch, self.max_blocks = table.shape
+        self.num_pages, self.block_size = int(num_pages), int(block_size)
+        self.num_kv_heads, self.head_dim = int(num_kv_heads), int(head_dim)
+        self.dtype = dtype
+        handle = ctypes.c_void_p()
+        lib = load_library()
+        _check(lib.lci_create_block_table(ptr, self.batch, self.max_blocks, self.num_pages,
+                                          self.block_size, self.num_kv_heads, self.head_dim,
+                                          _dtype_code(torch.empty(0, dtype=dtype)),
+                                          ctypes.byref(handle)), "lci_create_block_table")
+        self._handle = handle
+        self._lib = lib
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        return self._handle
+
+    def validate(self, stream=None) -> None:
+        _check(self._lib.lci_validate_block_table(self._handle, _stream(stream)),
+               "lci_validate_block_table")
+
+    def close(self) -> None:
+        if getattr(self, "_handle", None):
+            self._lib.lci_destroy_block_table(self._handle)
+            self._handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def create_block_table(table: torch.Tensor, k_pool: torch.Tensor) -> BlockTable:
+    """Block table over pools shaped [num_pages, H_kv, block_size, head_dim]."""
+    P, H_kv, bs, hd = k_pool.shape
+    return BlockTable(table, P, bs, H_kv, hd, k_pool.dtype)
+
+
+# ---------------------------------------------------------------- entry points
+
+def block_compress(k_idx: torch.Tensor, block_size: int, out: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """A0: [B, T, H, D] per-token indexer keys -> [B, ceil(T/bs), H, D] block means."""
+    B, T, H, D = k_idx.shape
+    NB = (T + block_size - 1) // block_size
+    if out is None:
+        out = torch.empty((B, NB, H, D), dtype=k_idx.dtype, device=k_idx.device)
+    _check(load_library().lci_block_compress(_dev(k_idx, "k_idx", None, 4), _dtype_code(k_idx), B, T,
+                                             H, D, block_size, _dev(out, "out", k_idx.dtype, 4),
+                                             _stream(stream)), "lci_block_compress")
+    return out
+
+
+def index_select_workspace_size(B, S, H_i, d_c, nb_max, topk, phase="auto") -> int:
+    n = ctypes.c_size_t()
+    _check(load_library().lci_index_select_workspace_size(B, S, H_i, d_c, nb_max, topk,
+                                                          PHASES[phase], ctypes.byref(n)),
+           "lci_index_select_workspace_size")
+    return n.value
+
+
+def index_select(q_c: torch.Tensor, k_c: torch.Tensor, block_size: int, ctx_len: torch.Tensor,
+                 q_start: torch.Tensor, topk: int, phase: str = "auto",
+                 ids: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    """A1+A2: ids [B, S, topk] int32, ranked (score desc, id asc), -1 padded."""
+    B, S, H_i, d_c = q_c.shape
+    nb_max = k_c.shape[1]
+    if k_c.shape[0] != B or k_c.shape[2:] != q_c.shape[2:] or k_c.dtype != q_c.dtype:
+        raise ValueError("lci: k_c must be [B, nb_max, H_i, d_c] with q_c's dtype")
+    if ids is None:
+        ids = torch.empty((B, S, topk), dtype=torch.int32, device=q_c.device)
+    need = index_select_workspace_size(B, S, H_i, d_c, nb_max, topk, phase)
+    if ws is None:
+        ws = workspace(q_c.device, need, "index_select")
+    _check(load_library().lci_index_select(
+        _dev(q_c, "q_c", None, 4), _dev(k_c, "k_c", q_c.dtype, 4), _dtype_code(q_c), B, S, H_i, d_c,
+        block_size, nb_max, _dev(ctx_len, "ctx_len", torch.int32, 1),
+        _dev(q_start, "q_start", torch.int32, 1), topk, PHASES[phase],
+        _dev(ids, "ids", torch.int32, 3), _dev(ws, "workspace"), ws.numel() * ws.element_size(),
+        _stream(stream)), "lci_index_select")
+    return ids
+
+
+def sparse_attn_workspace_size(B, S, H_q, topk, table: BlockTable, phase="auto") -> int:
+    n = ctypes.c_size_t()
+    _check(load_library().lci_sparse_attn_workspace_size(B, S, H_q, topk, table.handle,
+                                                         PHASES[phase], ctypes.byref(n)),
+           "lci_sparse_attn_workspace_size")
+    return n.value
+
+
+def sparse_attn(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, table: BlockTable,
+                ids: torch.Tensor, ctx_len: torch.Tensor, q_start: torch.Tensor,
+                scale: float = 0.0, phase: str = "auto", out: Optional[torch.Tensor] = None,
+                ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """A3+A4: exact softmax attention over the selected blocks. out [B, S, H_q, hd]."""
+    B, S, H_q, hd = q.shape
+    topk = ids.shape[-1]
+    if tuple(ids.shape) != (B, S, topk):
+        raise ValueError("lci: ids must be [B, S, topk]")
+    if tuple(k_pool.shape) != (table.num_pages, table.num_kv_heads, table.block_size,
+                               table.head_dim) or v_pool.shape != k_pool.shape:
+        raise ValueError("lci: pools do not match the block table")
+    if q.dtype != table.dtype or k_pool.dtype != q.dtype or v_pool.dtype != q.dtype:
+        raise TypeError("lci: q and the pools must share the block table's dtype")
+    if hd != table.head_dim:
+        raise ValueError("lci: q's head_dim differs from the block table's")
+    if out is None:
+        out = torch.empty_like(q)
+    need = sparse_attn_workspace_size(B, S, H_q, topk, table, phase)
+    if ws is None:
+        ws = workspace(q.device, need, "sparse_attn")
+    _check(load_library().lci_sparse_attn(
+        _dev(q, "q", None, 4), B, S, H_q, _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
+        table.handle, _dev(ids, "ids", torch.int32, 3), topk, _dev(ctx_len, "ctx_len", torch.int32, 1),
+        _dev(q_start, "q_start", torch.int32, 1), float(scale), PHASES[phase],
+        _dev(out, "out", q.dtype, 4), _dev(ws, "workspace"), ws.numel() * ws.element_size(),
+        _stream(stream)), "lci_sparse_attn")
+    return out
+
+
+def get_device_status(stream=None) -> None:
+    """Synchronise the stream; raise LciError if a device bounds check fired."""
+    _check(load_library().lci_get_device_status(_stream(stream)), "lci_get_device_status")

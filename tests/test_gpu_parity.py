@@ -1,0 +1,217 @@
+"""CUDA path (through the C ABI) against the CPU oracle, element by element.
+
+Block ids must match bit for bit (order and -1 padding included); outputs must
+match within max-abs 2e-2 (bf16) or 1e-4 (fp32). The five measured
+configurations run at full size, with the oracle computing every id row where
+that takes seconds and sampled rows (first, last, block boundaries, random)
+where it does not.
+"""
+import random
+
+import pytest
+import torch
+
+import long_context_indexer_b200 as lci
+import oracle
+from long_context_indexer_b200.workloads import CONFIGS, generate
+from tests.gpu_common import TOL, assert_out_close, oracle_k_c, oracle_rows, run_gpu, upload
+
+pytestmark = pytest.mark.gpu
+
+
+def _sample_rows(cfg, n_random=24, seed=0):
+    S, B = cfg.S, cfg.B
+    rows = set()
+    for b in range(B):
+        for s in (0, 1, cfg.bs - 1, cfg.bs, cfg.bs + 1, S // 2, S - 2, S - 1):
+            if 0 <= s < S:
+                rows.add(b * S + s)
+    rng = random.Random(seed)
+    rows.update(rng.randrange(B * S) for _ in range(n_random))
+    return sorted(rows)
+
+
+# ------------------------------------------------------------ full configs
+
+def test_tiny_fp32_end_to_end():
+    cfg = CONFIGS["tiny"]
+    w = generate(cfg)
+    k_c, ids, out = run_gpu(cfg, upload(w))
+    assert torch.equal(k_c.cpu().double(), oracle.block_compress(w["k_idx"], cfg.bs))
+    ref_ids, ref_out = oracle_rows(cfg, w)
+    assert torch.equal(ids.cpu().reshape(-1, cfg.topk), ref_ids)
+    assert_out_close(out.reshape(-1, cfg.H_q, cfg.hd), ref_out, torch.float32, "tiny")
+
+
+@pytest.mark.parametrize("name", ["decode", "long", "1m_decode"])
+def test_decode_configs_all_rows(name):
+    cfg = CONFIGS[name]
+    w = generate(cfg)
+    _, ids, out = run_gpu(cfg, upload(w))
+    ref_ids, ref_out = oracle_rows(cfg, w)
+    assert torch.equal(ids.cpu().reshape(-1, cfg.topk), ref_ids)
+    assert_out_close(out.reshape(-1, cfg.H_q, cfg.hd), ref_out, torch.bfloat16, name)
+
+
+def test_prefill_config():
+    cfg = CONFIGS["prefill"]
+    w = generate(cfg)
+    _, ids, out = run_gpu(cfg, upload(w))
+    # every id row (8192 x 128 blocks) ...
+    ref_ids = oracle.index_select(w["q_c"], w["k_c"], cfg.bs, w["ctx_len"], w["q_start"], cfg.topk)
+    assert torch.equal(ids.cpu().reshape(-1, cfg.topk), ref_ids)
+    # ... and the attention output on sampled rows
+    rows = _sample_rows(cfg, 40)
+    _, ref_out = oracle_rows(cfg, w, rows=rows)
+    got = out.reshape(-1, cfg.H_q, cfg.hd)[rows]
+    assert_out_close(got, ref_out, torch.bfloat16, "prefill")
+    assert torch.isfinite(out).all()
+
+
+def test_1m_chunk_config():
+    cfg = CONFIGS["1m_chunk"]
+    w = generate(cfg)
+    _, ids, out = run_gpu(cfg, upload(w))
+    rows = _sample_rows(cfg, 24)
+    ref_ids, ref_out = oracle_rows(cfg, w, rows=rows)
+    assert torch.equal(ids.cpu().reshape(-1, cfg.topk)[rows], ref_ids)
+    assert_out_close(out.reshape(-1, cfg.H_q, cfg.hd)[rows], ref_out, torch.bfloat16, "1m_chunk")
+    assert torch.isfinite(out).all()
+    # every row's ids are distinct visible blocks (a property that holds at any size)
+    ids_all = ids.cpu().reshape(-1, cfg.topk)
+    assert (ids_all >= 0).all() and (ids_all < cfg.NB).all()
+    srt = ids_all.sort(dim=1).values
+    assert (srt[:, 1:] != srt[:, :-1]).all()
+
+
+# ------------------------------------------------------------ small cases, edges
+
+SMALL = CONFIGS["decode"].replace(name="small", B=3, S=1, ctx=1000, q_start=999, bs=64, topk=4,
+                                  H_q=8, H_kv=2, hd=128, H_i=2, d_c=64, spare_pages=5)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("S,q0,ctx,topk", [(1, 999, 1000, 4), (37, 950, 1000, 3), (70, 0, 70, 2),
+                                           (5, 1200, 1000, 32), (300, 10, 900, 1)])
+def test_small_ragged_cases(dtype, S, q0, ctx, topk):
+    cfg = SMALL.replace(dtype=dtype, S=S, q_start=q0, ctx=ctx, topk=topk)
+    w = generate(cfg)
+    # ragged per-sequence lengths and start positions
+    w["ctx_len"] = torch.tensor([ctx, max(1, ctx // 2), 1], dtype=torch.int32)[: cfg.B]
+    w["q_start"] = torch.tensor([q0, max(0, q0 - 333), 0], dtype=torch.int32)[: cfg.B]
+    _, ids, out = run_gpu(cfg, upload(w))
+    ref_ids, ref_out = oracle_rows(cfg, w)
+    assert torch.equal(ids.cpu().reshape(-1, topk), ref_ids)
+    assert_out_close(out.reshape(-1, cfg.H_q, cfg.hd), ref_out, cfg.torch_dtype, "ragged")
+
+
+def test_empty_context_gives_no_ids_and_zero_output():
+    cfg = SMALL
+    w = generate(cfg)
+    w["ctx_len"] = torch.tensor([0, 0, 5], dtype=torch.int32)
+    _, ids, out = run_gpu(cfg, upload(w))
+    assert (ids[:2] == -1).all()
+    assert (out[:2] == 0).all()
+    assert ids[2, 0, 0].item() == 0 and (ids[2, 0, 1:] == -1).all()
+
+
+def test_ties_break_to_lower_block_id():
+    cfg = SMALL.replace(S=4, q_start=996)
+    w = generate(cfg)
+    w["q_c"].zero_()
+    _, ids, _ = run_gpu(cfg, upload(w))
+    assert (ids.cpu() == torch.arange(cfg.topk, dtype=torch.int32)).all()
+    # partial ties: only a few distinct score values
+    w = generate(cfg)
+    w["q_c"] = (w["q_c"] > 1).to(w["q_c"].dtype) * 0.0625
+    w["k_c"] = (w["k_c"] > 0).to(w["k_c"].dtype) * 0.0625
+    _, ids, _ = run_gpu(cfg, upload(w))
+    ref_ids, _ = oracle_rows(cfg, w)
+    assert torch.equal(ids.cpu().reshape(-1, cfg.topk), ref_ids)
+
+
+def test_extreme_grid_values_are_exact():
+    cfg = SMALL.replace(H_i=8, d_c=128, topk=6, S=2, q_start=998)
+    w = generate(cfg)
+    w["q_c"].fill_(2.0)
+    sign = torch.where(torch.rand(w["k_c"].shape, generator=torch.Generator().manual_seed(5)) < 0.5,
+                       -2.0, 2.0)
+    w["k_c"] = sign.to(w["k_c"].dtype)
+    _, ids, _ = run_gpu(cfg, upload(w))
+    ref_ids, _ = oracle_rows(cfg, w)
+    assert torch.equal(ids.cpu().reshape(-1, cfg.topk), ref_ids)
+
+
+def test_decode_matches_prefill_rows():
+    """The shared representation: decode at position p equals prefill row p."""
+    cfg = SMALL.replace(S=48, q_start=900, ctx=948, B=2)
+    w = generate(cfg)
+    d = upload(w)
+    _, ids_p, out_p = run_gpu(cfg, d, phase="prefill")
+    for s in (0, 17, 47):
+        d1 = dict(d)
+        d1["q_c"] = d["q_c"][:, s:s + 1].contiguous()
+        d1["q"] = d["q"][:, s:s + 1].contiguous()
+        d1["q_start"] = d["q_start"] + s
+        _, ids_d, out_d = run_gpu(cfg.replace(S=1), d1, phase="decode")
+        assert torch.equal(ids_d[:, 0], ids_p[:, s])
+        assert (out_d[:, 0].float() - out_p[:, s].float()).abs().max().item() <= TOL[torch.bfloat16]
+
+
+def test_phases_agree_and_runs_are_deterministic():
+    cfg = SMALL.replace(S=40, q_start=500)
+    d = upload(generate(cfg))
+    res = [run_gpu(cfg, d, phase=ph) for ph in ("auto", "prefill", "decode", "auto")]
+    for r in res[1:]:
+        assert torch.equal(r[1], res[0][1])
+    assert torch.equal(res[3][2], res[0][2])
+
+
+def test_page_permutation_gives_identical_output():
+    cfg = SMALL.replace(S=3, q_start=990)
+    w = generate(cfg)
+    d = upload(w)
+    _, ids, out = run_gpu(cfg, d)
+    P = cfg.num_pages
+    perm = torch.randperm(P, generator=torch.Generator().manual_seed(7))
+    k2 = torch.empty_like(w["k_pool"])
+    v2 = torch.empty_like(w["v_pool"])
+    k2[perm] = w["k_pool"]
+    v2[perm] = w["v_pool"]
+    d2 = dict(d, k_pool=k2.cuda(), v_pool=v2.cuda(),
+              block_table=perm[w["block_table"].long()].to(torch.int32).cuda())
+    _, ids2, out2 = run_gpu(cfg, d2)
+    assert torch.equal(ids, ids2)
+    assert torch.equal(out, out2)
+
+
+def test_explicit_scale():
+    cfg = SMALL.replace(S=2, q_start=998)
+    w = generate(cfg)
+    _, _, out = run_gpu(cfg, upload(w), scale=0.02)
+    _, ref = oracle_rows(cfg, w, scale=0.02)
+    assert_out_close(out.reshape(-1, cfg.H_q, cfg.hd), ref, torch.bfloat16, "scale")
+
+
+def test_device_bounds_checks_report_without_trapping():
+    cfg = SMALL
+    w = generate(cfg)
+    d = upload(w)
+    bt = lci.create_block_table(d["block_table"], d["k_pool"])
+    bad_ids = torch.tensor([[[0, cfg.NB, -1, 3]], [[-5, 1, 2, -1]], [[0, 1, 2, 3]]],
+                           dtype=torch.int32, device="cuda")
+    lci.sparse_attn(d["q"], d["k_pool"], d["v_pool"], bt, bad_ids, d["ctx_len"], d["q_start"])
+    with pytest.raises(lci.LciError) as e:
+        lci.get_device_status()
+    assert e.value.status == 5
+    lci.get_device_status()  # cleared
+    bad_table = d["block_table"].clone()
+    bad_table[1, 3] = cfg.num_pages
+    bt2 = lci.create_block_table(bad_table, d["k_pool"])
+    bt2.validate()
+    with pytest.raises(lci.LciError):
+        lci.get_device_status()
+    ok_ids = torch.tensor([[[0, 1, 2, 4]]] * 3, dtype=torch.int32, device="cuda")
+    lci.sparse_attn(d["q"], d["k_pool"], d["v_pool"], bt2, ok_ids, d["ctx_len"], d["q_start"])
+    with pytest.raises(lci.LciError):
+        lci.get_device_status()
