@@ -144,9 +144,12 @@ LCI_API lci_status lci_index_select_workspace_size(int32_t batch, int32_t S, int
  *   d_ctx_len  [batch] int32, d_q_start [batch] int32, device
  *   d_ids      [batch][S][topk] int32, device (output)
  *   workspace  >= lci_index_select_workspace_size bytes, 256-byte aligned.
- *              Its first bytes hold arrival counters that must be zero before
- *              the first call; every call leaves them zero again. Calls that
- *              share a workspace must not overlap in time.
+ *              It holds arrival counters whose position depends on the sizes
+ *              (batch, S, nb_max). Zero-fill a workspace before its first call;
+ *              every call leaves its counters at zero again, so later calls
+ *              with the same sizes need no clearing. Zero it again before using
+ *              it with other sizes. Calls that share a workspace must not
+ *              overlap in time.
  * Scores are accumulated in fp32. Limits: 1 <= topk <= 256,
  * nb_max <= 16384, H_i*d_c <= 8192 and a multiple of 8 (bf16) or 4 (f32).
  */
@@ -178,8 +181,8 @@ LCI_API lci_status lci_sparse_attn_workspace_size(int32_t batch, int32_t S, int3
  *   d_ids    [batch][S][topk] int32, device
  *   scale    softmax scale; <= 0 selects 1/sqrt(head_dim)
  *   out      [batch][S][H_q][head_dim], device, dtype (output)
- *   workspace >= lci_sparse_attn_workspace_size bytes, 256-byte aligned; same
- *             zero-on-first-use counter rule as lci_index_select.
+ *   workspace >= lci_sparse_attn_workspace_size bytes, 256-byte aligned; the
+ *             same zero-fill rule as lci_index_select (per set of sizes).
  * Softmax and accumulation are fp32; bf16 inputs feed the tensor cores.
  * Limits: H_q a multiple of num_kv_heads, head_dim a multiple of 32 and
  * <= 256, topk <= 256.

@@ -1,0 +1,356 @@
+// attn_decode.cuh -- paged gather + exact sparse attention on tensor cores
+// (bf16 in, fp32 softmax and accumulation), head_dim 128, up to 16 query heads
+// per KV head, block_size a multiple of 64.
+//
+// Work: one "pair" = (query row, KV head g). Its selected blocks are cut into
+// 64-token tiles ("units"); the units of a pair are split over `nsplit` CTAs
+// that form one thread-block cluster.
+//
+// Per CTA: one producer warp walks the CTA's units, resolves block id -> page
+// through the block table and issues TMA tensor loads of the K and V tiles
+// (two 64x64 boxes each, 128-byte swizzle) into a 3-stage shared-memory ring
+// guarded by mbarriers. Four consumer warps each take 16 tokens of every tile:
+// S = Q K^T with mma.m16n8k16 (the 16 rows are the query heads of the group),
+// an online softmax in fp32 (exp2, running max and sum), then O += P V.
+//
+// Fragment layout: the head-dim order inside each 32-dim slice is permuted
+// identically for Q and K, the token order inside each 8-token group is the
+// permutation pi(x) = x ^ (4 * (x & 1)) for both the S columns and the V rows,
+// and the output columns of P V are permuted so that each thread ends with 16
+// contiguous dims. Together with the swizzle this makes every 16-byte shared
+// load bank-conflict free and needs no ldmatrix.
+//
+// Combine: the four warps merge through shared memory into a CTA partial
+// (max, sum, unnormalised O); the CTAs of a cluster then merge their partials
+// through distributed shared memory, each CTA finishing a slice of the output.
+// No global workspace and no atomics.
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace lci {
+
+namespace dec {
+constexpr int kHD = 128;           // head dim
+constexpr int kTile = 64;          // tokens per unit
+constexpr int kStages = 3;         // shared-memory ring depth
+constexpr int kConsumers = 4;      // consumer warps, 16 tokens each
+constexpr int kThreads = (kConsumers + 1) * 32;
+constexpr int kBox = 64 * 64 * 2;  // one 64x64 bf16 box = 8 KiB
+constexpr int kStageBytes = 4 * kBox;  // K: 2 boxes, V: 2 boxes
+constexpr int kMaxSplit = 8;
+constexpr int kRows = 16;          // query heads per MMA (padded)
+// shared memory: stages, then barriers and metadata
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256;
+}  // namespace dec
+
+__device__ __forceinline__ int tok_perm(int x) { return x ^ ((x & 1) << 2); }
+
+// Byte offset of (row r, 16-byte chunk c of the 128-dim row) inside one K or V
+// tile stored as two 64x64 boxes with the 128-byte swizzle.
+__device__ __forceinline__ uint32_t tile_off(int r, int c) {
+    return (uint32_t)((c >> 3) * dec::kBox + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+__global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+    const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ table, int nb_max,
+    int num_pages, int H_kv, int bs, int S, int H_q, const int32_t* __restrict__ ids, int topk,
+    const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ q_start, float scale_log2,
+    __nv_bfloat16* __restrict__ out, int nsplit) {
+    using namespace dec;
+    namespace cg = cooperative_groups;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+    uint64_t* empty_bar = full_bar + kStages;
+    int* info = reinterpret_cast<int*>(empty_bar + kStages);  // t0 of the unit, or -1
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int pair = blockIdx.x, split = blockIdx.y;
+    const int row = pair / H_kv, g = pair - row * H_kv;
+    const int G = H_q / H_kv;
+    const int b = row / S, s = row - b * S;
+    const int tiles_per_block = bs / kTile;
+    const int nunits = topk * tiles_per_block;
+    const int per = (nunits + nsplit - 1) / nsplit;
+    const int u0 = split * per;
+    const int u1 = min(nunits, u0 + per);
+
+    if (tid == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&full_bar[i], 1);
+            mbar_init(&empty_bar[i], kConsumers);
+        }
+        fence_mbar_init();
+    }
+    if (warp == kConsumers && lane == 0) {
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
+    __syncthreads();
+
+    // Per-thread fragment coordinates.
+    const int g8 = lane >> 2, q4 = lane & 3;
+
+    // Query rows of this pair (independent of the previous kernel's output).
+    uint4 qa[4], qb[4];
+    if (warp < kConsumers) {
+        const int ha = g8, hb = g8 + 8;
+        const __nv_bfloat16* qrow = q + ((size_t)row * H_q + (size_t)g * G) * kHD;
+#pragma unroll
+        for (int sl = 0; sl < 4; ++sl) {
+            const int d0 = 32 * sl + 8 * q4;
+            qa[sl] = ha < G ? *reinterpret_cast<const uint4*>(qrow + (size_t)ha * kHD + d0)
+                            : make_uint4(0, 0, 0, 0);
+            qb[sl] = hb < G ? *reinterpret_cast<const uint4*>(qrow + (size_t)hb * kHD + d0)
+                            : make_uint4(0, 0, 0, 0);
+        }
+    }
+
+    // Block ids come from the previous kernel on the stream.
+    pdl_wait();
+    const long long p = (long long)q_start[b] + s;
+    const long long ctx = ctx_len[b];
+    const long long last = p < ctx - 1 ? p : ctx - 1;
+
+    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+    float o[2][8][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[h][i][e] = 0.f;
+
+    if (warp == kConsumers) {
+        // ---------------- producer ----------------
+        if (lane == 0) {
+            const int32_t* row_ids = ids + (size_t)row * topk;
+            for (int u = u0, it = 0; u < u1; ++u, ++it) {
+                const int st = it % kStages;
+                if (it >= kStages && !mbar_wait(&empty_bar[st], ((it / kStages) - 1) & 1)) break;
+                const int i = u / tiles_per_block, sub = u - i * tiles_per_block;
+                const int j = row_ids[i];
+                int t0 = -1, page = -1;
+                if (j >= 0 && j < nb_max) {
+                    page = table[(size_t)b * nb_max + j];
+                    if (page < 0 || page >= num_pages) {
+                        raise_status(kStatusBadPage);
+                        page = -1;
+                    } else {
+                        t0 = j * bs + sub * kTile;
+                        if ((long long)t0 > last) t0 = -1;
+                    }
+                } else if (j != -1) {
+                    raise_status(kStatusBadBlockId);
+                }
+                info[st] = t0;
+                if (t0 < 0) {
+                    mbar_arrive(&full_bar[st]);
+                } else {
+                    unsigned char* dst = smem + st * kStageBytes;
+                    const int y = (page * H_kv + g) * bs + sub * kTile;
+                    mbar_arrive_expect_tx(&full_bar[st], kStageBytes);
+                    tma_load_2d(dst, &tm_k, 0, y, &full_bar[st]);
+                    tma_load_2d(dst + kBox, &tm_k, 64, y, &full_bar[st]);
+                    tma_load_2d(dst + 2 * kBox, &tm_v, 0, y, &full_bar[st]);
+                    tma_load_2d(dst + 3 * kBox, &tm_v, 64, y, &full_bar[st]);
+                }
+            }
+        }
+    } else {
+        // ---------------- consumers ----------------
+        const int w = warp;
+        for (int u = u0, it = 0; u < u1; ++u, ++it) {
+            const int st = it % kStages;
+            const bool ok = mbar_wait(&full_bar[st], (it / kStages) & 1);
+            const int t0 = info[st];
+            const long long wt0 = (long long)t0 + 16 * w;  // first token of this warp
+            if (ok && t0 >= 0 && wt0 <= last) {
+                const uint32_t kbase = smem_u32(smem + st * kStageBytes);
+                const uint32_t vbase = kbase + 2 * kBox;
+                // S = Q K^T over this warp's 16 tokens (two n-tiles of 8)
+                float sacc[2][4];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) sacc[j][e] = 0.f;
+                    const int tr = 16 * w + 8 * j + tok_perm(g8);
+#pragma unroll
+                    for (int sl = 0; sl < 4; ++sl) {
+                        const uint4 kk = lds128(kbase + tile_off(tr, 4 * sl + q4));
+                        mma_bf16_16816(sacc[j], qa[sl].x, qb[sl].x, qa[sl].y, qb[sl].y, kk.x, kk.y);
+                        mma_bf16_16816(sacc[j], qa[sl].z, qb[sl].z, qa[sl].w, qb[sl].w, kk.z, kk.w);
+                    }
+                }
+                // tokens of the C-fragment columns: n = 2*q4, 2*q4+1 of each n-tile
+                const int c0 = tok_perm(2 * q4), c1 = tok_perm(2 * q4 + 1);
+                const bool partial = wt0 + 15 > last;
+                float x[2][4];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const long long ta = wt0 + 8 * j + c0, tb = wt0 + 8 * j + c1;
+                    x[j][0] = (partial && ta > last) ? -INFINITY : sacc[j][0] * scale_log2;
+                    x[j][1] = (partial && tb > last) ? -INFINITY : sacc[j][1] * scale_log2;
+                    x[j][2] = (partial && ta > last) ? -INFINITY : sacc[j][2] * scale_log2;
+                    x[j][3] = (partial && tb > last) ? -INFINITY : sacc[j][3] * scale_log2;
+                }
+                float mx_a = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+                float mx_b = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
+                mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
+                mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
+                mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
+                mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
+                const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
+                const float base_a = mn_a == -INFINITY ? 0.f : mn_a;
+                const float base_b = mn_b == -INFINITY ? 0.f : mn_b;
+                const float corr_a = exp2f(m_a - base_a), corr_b = exp2f(m_b - base_b);
+                m_a = mn_a;
+                m_b = mn_b;
+                float pr[2][4];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    pr[j][0] = exp2f(x[j][0] - base_a);
+                    pr[j][1] = exp2f(x[j][1] - base_a);
+                    pr[j][2] = exp2f(x[j][2] - base_b);
+                    pr[j][3] = exp2f(x[j][3] - base_b);
+                }
+                l_a = l_a * corr_a + (pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1]);
+                l_b = l_b * corr_b + (pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3]);
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        o[h][i][0] *= corr_a;
+                        o[h][i][1] *= corr_a;
+                        o[h][i][2] *= corr_b;
+                        o[h][i][3] *= corr_b;
+                    }
+                const uint32_t pa0 = pack_bf16x2(pr[0][0], pr[0][1]);
+                const uint32_t pa1 = pack_bf16x2(pr[0][2], pr[0][3]);
+                const uint32_t pa2 = pack_bf16x2(pr[1][0], pr[1][1]);
+                const uint32_t pa3 = pack_bf16x2(pr[1][2], pr[1][3]);
+                // V rows of the k positions 2q4, 2q4+1, 2q4+8, 2q4+9
+                const int r0 = 16 * w + c0, r1 = 16 * w + c1, r2 = r0 + 8, r3 = r1 + 8;
+                // masked tokens must not reach the MMA (their V may be unset memory)
+                const bool z0 = partial && wt0 + c0 > last, z1 = partial && wt0 + c1 > last;
+                const bool z2 = partial && wt0 + 8 + c0 > last, z3 = partial && wt0 + 8 + c1 > last;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint4 va = lds128(vbase + tile_off(r0, 8 * h + g8));
+                    uint4 vb = lds128(vbase + tile_off(r1, 8 * h + g8));
+                    uint4 vc = lds128(vbase + tile_off(r2, 8 * h + g8));
+                    uint4 vd = lds128(vbase + tile_off(r3, 8 * h + g8));
+                    if (z0) va = make_uint4(0, 0, 0, 0);
+                    if (z1) vb = make_uint4(0, 0, 0, 0);
+                    if (z2) vc = make_uint4(0, 0, 0, 0);
+                    if (z3) vd = make_uint4(0, 0, 0, 0);
+                    const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
+                    const uint32_t wc[4] = {vc.x, vc.y, vc.z, vc.w}, wd[4] = {vd.x, vd.y, vd.z, vd.w};
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const uint32_t sel = (i & 1) ? 0x7632u : 0x5410u;
+                        const uint32_t b0 = __byte_perm(wa[i >> 1], wb[i >> 1], sel);
+                        const uint32_t b1 = __byte_perm(wc[i >> 1], wd[i >> 1], sel);
+                        mma_bf16_16816(o[h][i], pa0, pa1, pa2, pa3, b0, b1);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty_bar[st]);
+        }
+    }
+    __syncthreads();  // every stage consumed: the ring memory is free
+
+    // ---------------- combine the four warps ----------------
+    // Warp partials: m, l [4][16]; O [4][16][128] fp32 (32 KiB in the ring).
+    float* wo = reinterpret_cast<float*>(smem);
+    float* wm = wo + kConsumers * kRows * kHD;
+    float* wl = wm + kConsumers * kRows;
+    if (warp < kConsumers) {
+        l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+        l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+        l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+        l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+        if (q4 == 0) {
+            wm[warp * kRows + g8] = m_a;
+            wm[warp * kRows + g8 + 8] = m_b;
+            wl[warp * kRows + g8] = l_a;
+            wl[warp * kRows + g8 + 8] = l_b;
+        }
+        float* oa = wo + (warp * kRows + g8) * kHD;
+        float* ob = oa + 8 * kHD;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int da = 64 * h + 16 * q4 + i, db = da + 8;
+                oa[da] = o[h][i][0];
+                oa[db] = o[h][i][1];
+                ob[da] = o[h][i][2];
+                ob[db] = o[h][i][3];
+            }
+    }
+    __syncthreads();
+    // CTA partial: cm, cl [16], co [16][128] (after the warp partials).
+    float* co = wl + kConsumers * kRows;
+    float* cm = co + kRows * kHD;
+    float* cl = cm + kRows;
+    for (int e = tid; e < kRows * kHD; e += kThreads) {
+        const int r = e / kHD;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w2 = 0; w2 < kConsumers; ++w2) M = fmaxf(M, wm[w2 * kRows + r]);
+        const float base = M == -INFINITY ? 0.f : M;
+        float acc = 0.f, L = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < kConsumers; ++w2) {
+            const float f = exp2f(wm[w2 * kRows + r] - base);
+            acc += f * wo[(w2 * kRows + r) * kHD + (e - r * kHD)];
+            L += f * wl[w2 * kRows + r];
+        }
+        co[e] = acc;
+        if ((e - r * kHD) == 0) {
+            cm[r] = M;
+            cl[r] = L;
+        }
+    }
+
+    __nv_bfloat16* orow = out + ((size_t)row * H_q + (size_t)g * G) * kHD;
+    if (nsplit == 1) {
+        __syncthreads();
+        for (int e = tid; e < G * kHD; e += kThreads) {
+            const int r = e / kHD;
+            const float L = cl[r];
+            orow[e] = __float2bfloat16_rn(L > 0.f ? co[e] / L : 0.f);
+        }
+        return;
+    }
+    // ---------------- combine the CTAs of the cluster (DSMEM) ----------------
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    const int nel = G * kHD;
+    const int chunk = (nel + nsplit - 1) / nsplit;
+    const int e0 = split * chunk, e1 = min(nel, e0 + chunk);
+    for (int e = e0 + tid; e < e1; e += kThreads) {
+        const int r = e / kHD;
+        float M = -INFINITY;
+        for (int c = 0; c < nsplit; ++c) M = fmaxf(M, cluster.map_shared_rank(cm, c)[r]);
+        const float base = M == -INFINITY ? 0.f : M;
+        float acc = 0.f, L = 0.f;
+        for (int c = 0; c < nsplit; ++c) {
+            const float f = exp2f(cluster.map_shared_rank(cm, c)[r] - base);
+            acc += f * cluster.map_shared_rank(co, c)[e];
+            L += f * cluster.map_shared_rank(cl, c)[r];
+        }
+        orow[e] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
+    }
+    cluster.sync();  // keep this CTA's partial alive until every reader is done
+}
+
+}  // namespace lci

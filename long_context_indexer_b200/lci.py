@@ -122,8 +122,11 @@ _ws: Dict[Tuple[int, str], torch.Tensor] = {}
 def workspace(device: torch.device, nbytes: int, tag: str) -> torch.Tensor:
     """A zero-initialised, 256-byte aligned device buffer of at least nbytes.
 
-    The library keeps the counter region of a workspace at zero between calls,
-    so a buffer is zero-filled once, when it is first allocated or grown.
+    Workspaces hold arrival counters that the library leaves at zero after
+    every call, but only in the layout of the shape they were used with. So a
+    cached buffer is keyed by ``tag``, which callers make unique per layout
+    (entry point and the sizes the layout depends on), and is zero-filled once
+    when first allocated.
     """
     key = (torch.device(device).index or 0, tag)
     buf = _ws.get(key)
@@ -217,7 +220,7 @@ def index_select(q_c: torch.Tensor, k_c: torch.Tensor, block_size: int, ctx_len:
         ids = torch.empty((B, S, topk), dtype=torch.int32, device=q_c.device)
     need = index_select_workspace_size(B, S, H_i, d_c, nb_max, topk, phase)
     if ws is None:
-        ws = workspace(q_c.device, need, "index_select")
+        ws = workspace(q_c.device, need, f"index_select:{B}x{S}x{nb_max}:{H_i * d_c}")
     _check(load_library().lci_index_select(
         _dev(q_c, "q_c", None, 4), _dev(k_c, "k_c", q_c.dtype, 4), _dtype_code(q_c), B, S, H_i, d_c,
         block_size, nb_max, _dev(ctx_len, "ctx_len", torch.int32, 1),
@@ -255,7 +258,8 @@ def sparse_attn(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, tab
         out = torch.empty_like(q)
     need = sparse_attn_workspace_size(B, S, H_q, topk, table, phase)
     if ws is None:
-        ws = workspace(q.device, need, "sparse_attn")
+        ws = workspace(q.device, need, f"sparse_attn:{B}x{S}x{H_q}x{topk}:{table.max_blocks}:"
+                                       f"{table.num_kv_heads}x{table.block_size}")
     _check(load_library().lci_sparse_attn(
         _dev(q, "q", None, 4), B, S, H_q, _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
         table.handle, _dev(ids, "ids", torch.int32, 3), topk, _dev(ctx_len, "ctx_len", torch.int32, 1),

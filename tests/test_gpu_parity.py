@@ -211,7 +211,7 @@ def test_device_bounds_checks_report_without_trapping():
     bt2.validate()
     with pytest.raises(lci.LciError):
         lci.get_device_status()
-    ok_ids = torch.tensor([[[0, 1, 2, 4]]] * 3, dtype=torch.int32, device="cuda")
+    ok_ids = torch.tensor([[[0, 1, 2, 3]]] * 3, dtype=torch.int32, device="cuda")
     lci.sparse_attn(d["q"], d["k_pool"], d["v_pool"], bt2, ok_ids, d["ctx_len"], d["q_start"])
     with pytest.raises(lci.LciError):
         lci.get_device_status()
