@@ -11,6 +11,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "ptx.cuh"
 #include "topk_select.cuh"
 
 namespace lci {
@@ -51,6 +52,9 @@ __global__ void __launch_bounds__(NT) index_gemv_select_kernel(
     constexpr int NW = NT / 32;
     constexpr int E = ElemsPer16B<T>::v;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // Let the attention kernel that follows on the stream start its prologue;
+    // it waits for this grid's results before reading the block ids.
+    pdl_trigger();
     const int row = blockIdx.x, chunk = blockIdx.y;
     const int b = row / S, s = row - b * S;
     const long long p = (long long)__ldg(&q_start[b]) + s;

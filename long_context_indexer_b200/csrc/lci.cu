@@ -2,15 +2,19 @@
 //
 // Host side only: argument checks, workspace layout, kernel selection and
 // launches. Every step of the computation runs in the kernels included below.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <mutex>
 #include <new>
 #include <string>
 
 #include "../../include/lci.h"
+#include "attn_decode.cuh"
 #include "attn_simt.cuh"
 #include "common.cuh"
 #include "compress.cuh"
@@ -163,6 +167,103 @@ lci_status launch_attn_simt(const void* q, int32_t batch, int32_t S, int32_t H_q
         static_cast<const T*>(q), static_cast<const T*>(k_pool), static_cast<const T*>(v_pool),
         t->d_table, t->max_blocks, t->num_pages, t->num_kv_heads, t->block_size, t->head_dim, S,
         H_q, ids, topk, ctx_len, q_start, scale_log2, static_cast<T*>(out));
+    return check_launch("sparse_attn");
+}
+
+// ---- TMA tensor maps (driver entry point fetched through the runtime) ----
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// A KV pool [P][H_kv][bs][128] bf16 seen as a 2D tensor of P*H_kv*bs rows of
+// 128 elements, read in 64x64 boxes with the 128-byte swizzle.
+lci_status encode_pool_map(CUtensorMap* map, const void* pool, long long rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return fail(LCI_ERR_CUDA, "sparse_attn: cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[2] = {(cuuint64_t)lci::dec::kHD, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)lci::dec::kHD * 2};
+    cuuint32_t box[2] = {64, 64};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pool), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(LCI_ERR_CUDA, "sparse_attn: tensor map encode failed (%d)", (int)r);
+    return LCI_OK;
+}
+
+bool decode_kernel_fits(const lci_block_table* t, int32_t H_q, const void* k_pool,
+                        const void* v_pool) {
+    const int G = H_q / t->num_kv_heads;
+    const long long rows = (long long)t->num_pages * t->num_kv_heads * t->block_size;
+    return t->dtype == LCI_BF16 && t->head_dim == lci::dec::kHD && t->block_size % 64 == 0 &&
+           G <= lci::dec::kRows && aligned16(k_pool) && aligned16(v_pool) && rows < (1ll << 31);
+}
+
+int decode_splits(long long pairs, int units) {
+    long long want = (2 * 148 + pairs - 1) / pairs;
+    if (want > lci::dec::kMaxSplit) want = lci::dec::kMaxSplit;
+    if (want > units) want = units;
+    return want < 1 ? 1 : (int)want;
+}
+
+lci_status launch_attn_decode(const void* q, int32_t batch, int32_t S, int32_t H_q,
+                              const void* k_pool, const void* v_pool, const lci_block_table* t,
+                              const int32_t* ids, int32_t topk, const int32_t* ctx_len,
+                              const int32_t* q_start, float scale, void* out, cudaStream_t st) {
+    const long long rows = (long long)t->num_pages * t->num_kv_heads * t->block_size;
+    CUtensorMap tm_k, tm_v;
+    lci_status s = encode_pool_map(&tm_k, k_pool, rows);
+    if (s != LCI_OK) return s;
+    s = encode_pool_map(&tm_v, v_pool, rows);
+    if (s != LCI_OK) return s;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(lci::sparse_attn_decode_kernel,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        lci::dec::kSmemBytes);
+    });
+    if (attr_err != cudaSuccess)
+        return fail(LCI_ERR_CUDA, "sparse_attn: %s", cudaGetErrorString(attr_err));
+    const long long pairs = (long long)batch * S * t->num_kv_heads;
+    const int units = topk * (t->block_size / 64);
+    const int nsplit = decode_splits(pairs, units);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)pairs, (unsigned)nsplit, 1);
+    cfg.blockDim = dim3(lci::dec::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = lci::dec::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attrs[2];
+    int na = 0;
+    if (nsplit > 1) {
+        attrs[na].id = cudaLaunchAttributeClusterDimension;
+        attrs[na].val.clusterDim.x = 1;
+        attrs[na].val.clusterDim.y = (unsigned)nsplit;
+        attrs[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+    cfg.attrs = attrs;
+    cfg.numAttrs = na;
+    const float scale_log2 = scale * 1.4426950408889634f;
+    cudaError_t e = cudaLaunchKernelEx(
+        &cfg, lci::sparse_attn_decode_kernel, tm_k, tm_v, static_cast<const __nv_bfloat16*>(q),
+        t->d_table, t->max_blocks, t->num_pages, t->num_kv_heads, t->block_size, S, H_q, ids, topk,
+        ctx_len, q_start, scale_log2, static_cast<__nv_bfloat16*>(out), nsplit);
+    if (e != cudaSuccess) return fail(LCI_ERR_CUDA, "sparse_attn: %s", cudaGetErrorString(e));
     return check_launch("sparse_attn");
 }
 
@@ -320,6 +421,9 @@ lci_status lci_sparse_attn(const void* q, int32_t batch, int32_t S, int32_t H_q,
     (void)workspace;
     (void)workspace_bytes;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (decode_kernel_fits(table, H_q, k_pool, v_pool))
+        return launch_attn_decode(q, batch, S, H_q, k_pool, v_pool, table, d_ids, topk, d_ctx_len,
+                                  d_q_start, scale, out, cs);
     if (table->dtype == LCI_F32)
         return launch_attn_simt<float>(q, batch, S, H_q, k_pool, v_pool, table, d_ids, topk,
                                        d_ctx_len, d_q_start, scale, out, cs);

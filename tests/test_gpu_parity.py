@@ -215,3 +215,21 @@ def test_device_bounds_checks_report_without_trapping():
     lci.sparse_attn(d["q"], d["k_pool"], d["v_pool"], bt2, ok_ids, d["ctx_len"], d["q_start"])
     with pytest.raises(lci.LciError):
         lci.get_device_status()
+
+
+@pytest.mark.parametrize("S,q0", [(1, 999), (24, 976)])
+def test_unwritten_cache_slots_never_reach_the_output(S, q0):
+    """Pool slots past ctx_len (unwritten cache memory) are loaded with their
+    64-token tile but masked; NaN there must not leak into the output."""
+    cfg = SMALL.replace(S=S, q_start=q0, ctx=1000)
+    w = generate(cfg)
+    bs = cfg.bs
+    for b in range(cfg.B):
+        last_block = (cfg.ctx - 1) // bs
+        page = int(w["block_table"][b, last_block])
+        w["k_pool"][page, :, cfg.ctx % bs:] = float("nan")
+        w["v_pool"][page, :, cfg.ctx % bs:] = float("nan")
+    _, ids, out = run_gpu(cfg, upload(w))
+    ref_ids, ref_out = oracle_rows(cfg, w)
+    assert torch.equal(ids.cpu().reshape(-1, cfg.topk), ref_ids)
+    assert_out_close(out.reshape(-1, cfg.H_q, cfg.hd), ref_out, torch.bfloat16, "nan-tail")
