@@ -129,37 +129,54 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
 
     if (warp == kConsumers) {
         // ---------------- producer ----------------
-        if (lane == 0) {
-            const int32_t* row_ids = ids + (size_t)row * topk;
-            for (int u = u0, it = 0; u < u1; ++u, ++it) {
-                const int st = it % kStages;
-                if (it >= kStages && !mbar_wait(&empty_bar[st], ((it / kStages) - 1) & 1)) break;
+        // Lanes resolve 32 units at a time (block id -> page -> TMA row), so the
+        // dependent id and table loads overlap; lane 0 then issues the copies.
+        const int32_t* row_ids = ids + (size_t)row * topk;
+        bool alive = true;
+        for (int base = u0; base < u1 && alive; base += 32) {
+            const int u = base + lane;
+            int t0 = -1, y = 0;
+            if (u < u1) {
                 const int i = u / tiles_per_block, sub = u - i * tiles_per_block;
                 const int j = row_ids[i];
-                int t0 = -1, page = -1;
                 if (j >= 0 && j < nb_max) {
-                    page = table[(size_t)b * nb_max + j];
+                    const int page = table[(size_t)b * nb_max + j];
                     if (page < 0 || page >= num_pages) {
                         raise_status(kStatusBadPage);
-                        page = -1;
-                    } else {
+                    } else if ((long long)j * bs + sub * kTile <= last) {
                         t0 = j * bs + sub * kTile;
-                        if ((long long)t0 > last) t0 = -1;
+                        y = (page * H_kv + g) * bs + sub * kTile;
                     }
                 } else if (j != -1) {
                     raise_status(kStatusBadBlockId);
                 }
-                info[st] = t0;
-                if (t0 < 0) {
-                    mbar_arrive(&full_bar[st]);
-                } else {
-                    unsigned char* dst = smem + st * kStageBytes;
-                    const int y = (page * H_kv + g) * bs + sub * kTile;
-                    mbar_arrive_expect_tx(&full_bar[st], kStageBytes);
-                    tma_load_2d(dst, &tm_k, 0, y, &full_bar[st]);
-                    tma_load_2d(dst + kBox, &tm_k, 64, y, &full_bar[st]);
-                    tma_load_2d(dst + 2 * kBox, &tm_v, 0, y, &full_bar[st]);
-                    tma_load_2d(dst + 3 * kBox, &tm_v, 64, y, &full_bar[st]);
+            }
+            const int n = min(32, u1 - base);
+            for (int k = 0; k < n; ++k) {
+                const int tk = __shfl_sync(0xffffffffu, t0, k);
+                const int yk = __shfl_sync(0xffffffffu, y, k);
+                const int it = base - u0 + k;
+                const int st = it % kStages;
+                int ok = 1;
+                if (lane == 0) {
+                    if (it >= kStages) ok = mbar_wait(&empty_bar[st], ((it / kStages) - 1) & 1);
+                    if (ok) {
+                        info[st] = tk;
+                        if (tk < 0) {
+                            mbar_arrive(&full_bar[st]);
+                        } else {
+                            unsigned char* dst = smem + st * kStageBytes;
+                            mbar_arrive_expect_tx(&full_bar[st], kStageBytes);
+                            tma_load_2d(dst, &tm_k, 0, yk, &full_bar[st]);
+                            tma_load_2d(dst + kBox, &tm_k, 64, yk, &full_bar[st]);
+                            tma_load_2d(dst + 2 * kBox, &tm_v, 0, yk, &full_bar[st]);
+                            tma_load_2d(dst + 3 * kBox, &tm_v, 64, yk, &full_bar[st]);
+                        }
+                    }
+                }
+                if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                    alive = false;
+                    break;
                 }
             }
         }
@@ -301,32 +318,36 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
     float* co = wl + kConsumers * kRows;
     float* cm = co + kRows * kHD;
     float* cl = cm + kRows;
-    for (int e = tid; e < kRows * kHD; e += kThreads) {
-        const int r = e / kHD;
+    float* wf = cl + kRows;  // [kConsumers][16] merge weights of the warps
+    if (tid < kRows) {
         float M = -INFINITY;
 #pragma unroll
-        for (int w2 = 0; w2 < kConsumers; ++w2) M = fmaxf(M, wm[w2 * kRows + r]);
+        for (int w2 = 0; w2 < kConsumers; ++w2) M = fmaxf(M, wm[w2 * kRows + tid]);
         const float base = M == -INFINITY ? 0.f : M;
-        float acc = 0.f, L = 0.f;
+        float L = 0.f;
 #pragma unroll
         for (int w2 = 0; w2 < kConsumers; ++w2) {
-            const float f = exp2f(wm[w2 * kRows + r] - base);
-            acc += f * wo[(w2 * kRows + r) * kHD + (e - r * kHD)];
-            L += f * wl[w2 * kRows + r];
+            const float f = exp2f(wm[w2 * kRows + tid] - base);
+            wf[w2 * kRows + tid] = f;
+            L += f * wl[w2 * kRows + tid];
         }
+        cm[tid] = M;
+        cl[tid] = L;
+    }
+    __syncthreads();
+    for (int e = tid; e < kRows * kHD; e += kThreads) {
+        const int r = e / kHD;
+        float acc = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < kConsumers; ++w2) acc += wf[w2 * kRows + r] * wo[w2 * kRows * kHD + e];
         co[e] = acc;
-        if ((e - r * kHD) == 0) {
-            cm[r] = M;
-            cl[r] = L;
-        }
     }
 
     __nv_bfloat16* orow = out + ((size_t)row * H_q + (size_t)g * G) * kHD;
     if (nsplit == 1) {
         __syncthreads();
         for (int e = tid; e < G * kHD; e += kThreads) {
-            const int r = e / kHD;
-            const float L = cl[r];
+            const float L = cl[e / kHD];
             orow[e] = __float2bfloat16_rn(L > 0.f ? co[e] / L : 0.f);
         }
         return;
@@ -334,21 +355,39 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
     // ---------------- combine the CTAs of the cluster (DSMEM) ----------------
     cg::cluster_group cluster = cg::this_cluster();
     cluster.sync();
+    float* xf = wf + kConsumers * kRows;  // [kMaxSplit][16] merge weights of the CTAs
+    float* xl = xf + kMaxSplit * kRows;   // [16] 1 / merged sum
+    if (tid < kRows) {
+        float mc[kMaxSplit];
+        float M = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kMaxSplit; ++c) {
+            mc[c] = c < nsplit ? cluster.map_shared_rank(cm, c)[tid] : -INFINITY;
+            M = fmaxf(M, mc[c]);
+        }
+        const float base = M == -INFINITY ? 0.f : M;
+        float L = 0.f;
+#pragma unroll
+        for (int c = 0; c < kMaxSplit; ++c) {
+            const float f = c < nsplit ? exp2f(mc[c] - base) : 0.f;
+            xf[c * kRows + tid] = f;
+            if (c < nsplit) L += f * cluster.map_shared_rank(cl, c)[tid];
+        }
+        xl[tid] = L > 0.f ? 1.f / L : 0.f;
+    }
+    __syncthreads();
     const int nel = G * kHD;
     const int chunk = (nel + nsplit - 1) / nsplit;
     const int e0 = split * chunk, e1 = min(nel, e0 + chunk);
     for (int e = e0 + tid; e < e1; e += kThreads) {
         const int r = e / kHD;
-        float M = -INFINITY;
-        for (int c = 0; c < nsplit; ++c) M = fmaxf(M, cluster.map_shared_rank(cm, c)[r]);
-        const float base = M == -INFINITY ? 0.f : M;
-        float acc = 0.f, L = 0.f;
-        for (int c = 0; c < nsplit; ++c) {
-            const float f = exp2f(cluster.map_shared_rank(cm, c)[r] - base);
-            acc += f * cluster.map_shared_rank(co, c)[e];
-            L += f * cluster.map_shared_rank(cl, c)[r];
-        }
-        orow[e] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
+        float v[kMaxSplit];
+#pragma unroll
+        for (int c = 0; c < kMaxSplit; ++c) v[c] = c < nsplit ? cluster.map_shared_rank(co, c)[e] : 0.f;
+        float acc = 0.f;
+#pragma unroll
+        for (int c = 0; c < kMaxSplit; ++c) acc += xf[c * kRows + r] * v[c];
+        orow[e] = __float2bfloat16_rn(acc * xl[r]);
     }
     cluster.sync();  // keep this CTA's partial alive until every reader is done
 }

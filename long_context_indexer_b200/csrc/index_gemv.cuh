@@ -32,22 +32,17 @@ __device__ __forceinline__ float dot_chunk(const uint4& raw, const float* q, __n
            d.x * q[6] + d.y * q[7];
 }
 
-__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
-
 template <typename T, int NT>
 __global__ void __launch_bounds__(NT) index_gemv_select_kernel(
     const T* __restrict__ q_c, const T* __restrict__ k_c, int S, int K, int nb_max, int bs,
     const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ q_start, int topk,
     int chunk_blocks, int nchunks, float* __restrict__ scores,
     unsigned int* __restrict__ counters, int32_t* __restrict__ ids) {
-    extern __shared__ __align__(16) unsigned char dyn_smem[];
+    // Dynamic shared memory: [k_c chunk: chunk_blocks * K * sizeof(T)][q row: K floats];
+    // after scoring, the first nb_max * 4 bytes hold the row's radix keys.
+    extern __shared__ __align__(128) unsigned char dyn_smem[];
     __shared__ SelectSmem sel;
+    __shared__ uint64_t bar;
     __shared__ int s_last;
     constexpr int NW = NT / 32;
     constexpr int E = ElemsPer16B<T>::v;
@@ -61,17 +56,31 @@ __global__ void __launch_bounds__(NT) index_gemv_select_kernel(
     const int vis = visible_blocks(p, __ldg(&ctx_len[b]), bs, nb_max);
     const int j0 = chunk * chunk_blocks;
     const int j1 = min(j0 + chunk_blocks, vis);
+    const size_t row_bytes = (size_t)K * sizeof(T);
 
     if (j0 < j1) {
-        float* qs = reinterpret_cast<float*>(dyn_smem);
+        unsigned char* tile = dyn_smem;
+        float* qs = reinterpret_cast<float*>(dyn_smem + (size_t)chunk_blocks * row_bytes);
+        if (tid == 0) {
+            mbar_init(&bar, 1);
+            fence_mbar_init();
+            // The chunk's block keys are one contiguous range of k_c.
+            const uint32_t bytes = (uint32_t)((j1 - j0) * row_bytes);
+            const unsigned char* src =
+                reinterpret_cast<const unsigned char*>(k_c + ((size_t)b * nb_max + j0) * K);
+            mbar_arrive_expect_tx(&bar, bytes);
+            for (uint32_t off = 0; off < bytes; off += 16384u)
+                bulk_load(tile + off, src + off, min(16384u, bytes - off), &bar);
+        }
         const T* qrow = q_c + (size_t)row * K;
         for (int i = tid; i < K; i += NT) qs[i] = to_f32(qrow[i]);
         __syncthreads();
+        const bool ok = mbar_wait(&bar, 0);
         const int nvec = K / E;
-        for (int j = j0 + warp; j < j1; j += NW) {
-            const uint4* kr = reinterpret_cast<const uint4*>(k_c + ((size_t)b * nb_max + j) * K);
+        for (int j = j0 + warp; ok && j < j1; j += NW) {
+            const uint4* kr = reinterpret_cast<const uint4*>(tile + (size_t)(j - j0) * row_bytes);
             float acc = 0.f;
-            for (int c = lane; c < nvec; c += 32) acc += dot_chunk(ld_stream(kr + c), qs + c * E, T());
+            for (int c = lane; c < nvec; c += 32) acc += dot_chunk(kr[c], qs + c * E, T());
             acc = warp_sum(acc);
             if (lane == 0) scores[(size_t)row * nb_max + j] = acc;
         }

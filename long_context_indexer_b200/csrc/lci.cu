@@ -56,6 +56,7 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool dtype_ok(lci_dtype d) { return d == LCI_F32 || d == LCI_BF16; }
+size_t dtype_size(lci_dtype d) { return d == LCI_F32 ? 4 : 2; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -69,6 +70,7 @@ lci_phase resolve_phase(lci_phase ph, int32_t S) {
 constexpr int kIndexThreads = 256;
 constexpr int kMaxNbMax = 16384;
 constexpr int kMaxIndexK = 8192;
+constexpr int kIndexMaxSmem = 65536 + 1024;
 
 struct IndexPlan {
     int chunk_blocks, nchunks;
@@ -76,20 +78,23 @@ struct IndexPlan {
     size_t smem;
 };
 
-IndexPlan plan_index(int32_t batch, int32_t S, int32_t K, int32_t nb_max) {
+IndexPlan plan_index(int32_t batch, int32_t S, int32_t K, int32_t nb_max, size_t esz) {
     IndexPlan pl{};
     const long long rows = (long long)batch * S;
-    // Enough CTAs to cover the 148 SMs several times over, chunks of 8..32 blocks.
+    const size_t row_bytes = (size_t)K * esz;
+    // Chunks of at most 32 blocks and 32 KiB of block keys, halved while the
+    // grid would not cover the 148 SMs about four times.
     int chunk = 32;
-    while (chunk > 8 && rows * ((nb_max + chunk - 1) / chunk) < 4 * 148) chunk >>= 1;
+    while (chunk > 1 && (size_t)chunk * row_bytes > 32768) chunk >>= 1;
+    while (chunk > 4 && rows * ((nb_max + chunk - 1) / chunk) < 4 * 148) chunk >>= 1;
     pl.chunk_blocks = chunk;
     pl.nchunks = (nb_max + chunk - 1) / chunk;
     pl.off_counters = 0;
     pl.off_scores = align_up((size_t)rows * sizeof(unsigned int));
     pl.bytes = pl.off_scores + align_up((size_t)rows * nb_max * sizeof(float));
-    const size_t qbytes = (size_t)K * sizeof(float);
-    const size_t kbytes = (size_t)nb_max * sizeof(uint32_t);
-    pl.smem = qbytes > kbytes ? qbytes : kbytes;
+    const size_t stage = (size_t)chunk * row_bytes + (size_t)K * sizeof(float);
+    const size_t keys = (size_t)nb_max * sizeof(uint32_t);
+    pl.smem = stage > keys ? stage : keys;
     return pl;
 }
 
@@ -118,11 +123,18 @@ lci_status launch_index_gemv(const void* q_c, const void* k_c, int32_t batch, in
                              const int32_t* q_start, int32_t topk, int32_t* ids, void* ws,
                              const IndexPlan& pl, cudaStream_t st) {
     auto kern = lci::index_gemv_select_kernel<T, kIndexThreads>;
-    if (pl.smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)pl.smem);
-        if (e != cudaSuccess) return fail(LCI_ERR_CUDA, "index_select: %s", cudaGetErrorString(e));
-    }
+    // Largest dynamic shared memory any plan asks for: 32 KiB of block keys
+    // plus an 8192-float query row, or 16384 radix keys.
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [kern] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        kIndexMaxSmem);
+    });
+    if (attr_err != cudaSuccess)
+        return fail(LCI_ERR_CUDA, "index_select: %s", cudaGetErrorString(attr_err));
+    if (pl.smem > (size_t)kIndexMaxSmem)
+        return fail(LCI_ERR_UNSUPPORTED, "index_select: needs %zu bytes of shared memory", pl.smem);
     char* w = static_cast<char*>(ws);
     dim3 grid((unsigned)(batch * S), (unsigned)pl.nchunks);
     kern<<<grid, kIndexThreads, pl.smem, st>>>(
@@ -361,7 +373,7 @@ lci_status lci_index_select_workspace_size(int32_t batch, int32_t S, int32_t H_i
     lci_status st = check_index_args(batch, S, H_i, d_c, nb_max, topk, LCI_BF16);
     if (st != LCI_OK && st != LCI_ERR_UNSUPPORTED) return st;
     (void)phase;
-    *bytes = plan_index(batch, S, H_i * d_c, nb_max).bytes;
+    *bytes = plan_index(batch, S, H_i * d_c, nb_max, 2).bytes;
     return ok();
 }
 
@@ -380,7 +392,7 @@ lci_status lci_index_select(const void* q_c, const void* k_c, lci_dtype dtype, i
     if (!aligned16(q_c) || !aligned16(k_c))
         return fail(LCI_ERR_INVALID_ARG, "index_select: q_c and k_c must be 16-byte aligned");
     const int K = H_i * d_c;
-    const IndexPlan pl = plan_index(batch, S, K, nb_max);
+    const IndexPlan pl = plan_index(batch, S, K, nb_max, dtype_size(dtype));
     if (!workspace || workspace_bytes < pl.bytes ||
         (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
         return fail(LCI_ERR_WORKSPACE, "index_select: workspace needs %zu bytes, 256-byte aligned "
