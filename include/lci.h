@@ -194,6 +194,37 @@ LCI_API lci_status lci_sparse_attn(const void* q, int32_t batch, int32_t S, int3
                            void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * lci_index_select without any device allocation. The reference pages have no
+ * counterpart; this entry point exists for callers that are not allowed to
+ * allocate device memory or to hold a workspace of their own: for example code
+ * running inside a host framework that owns every device allocation (a plugin
+ * or an engine with a pre-planned memory arena) and so cannot call cudaMalloc
+ * or keep a separate scratch buffer per call site.
+ *
+ * Same arguments, layouts, results and limits as lci_index_select, minus the
+ * workspace; it always runs the one-row-at-a-time kernel (the decode schedule)
+ * whatever the phase. Its scratch is one fixed array of
+ * LCI_NOALLOC_SCRATCH_BYTES bytes inside the library, which every GPU that
+ * loads the library holds until the process exits. Sizes whose scratch would
+ * exceed it (about batch*S*(4*nb_max + 4) bytes plus alignment) return
+ * LCI_ERR_WORKSPACE before anything is launched.
+ * The first call on each device looks up the array's device address (with that
+ * device current); make that first call before any stream capture. Each call
+ * clears the array's arrival counters on `stream` before its kernel runs (the
+ * array keeps the previous call's contents otherwise). All calls on a device
+ * share the one array: calls that may overlap on the GPU (other streams, other
+ * host threads) race and corrupt each other's results. The caller still passes
+ * and owns all inputs and outputs. No cudaMalloc or cudaFree is ever called.
+ */
+#define LCI_NOALLOC_SCRATCH_BYTES (8u << 20)
+LCI_API lci_status lci_index_select_noalloc(const void* q_c, const void* k_c, lci_dtype dtype,
+                                            int32_t batch, int32_t S, int32_t H_i, int32_t d_c,
+                                            int32_t block_size, int32_t nb_max,
+                                            const int32_t* d_ctx_len, const int32_t* d_q_start,
+                                            int32_t topk, lci_phase phase, int32_t* d_ids,
+                                            void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the sticky device status
  * word of the current device: LCI_OK, or LCI_ERR_DEVICE_BOUNDS when a device
  * bounds check fired since the last call.

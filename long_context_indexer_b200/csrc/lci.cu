@@ -443,6 +443,78 @@ lci_status lci_sparse_attn(const void* q, int32_t batch, int32_t S, int32_t H_q,
                                            d_ctx_len, d_q_start, scale, out, cs);
 }
 
+}  // extern "C"
+
+// ---- index selection without device allocation ----
+//
+// The scratch of lci_index_select_noalloc: one file-scope device array per GPU
+// that loads the library. Host code never passes its name to a kernel (on the
+// host it is only a stand-in symbol); the device address comes from
+// cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LCI_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+std::once_flag g_noalloc_once[kNoAllocMaxDevices];
+void* g_noalloc_ptr[kNoAllocMaxDevices];
+cudaError_t g_noalloc_err[kNoAllocMaxDevices];
+
+lci_status noalloc_scratch(void** out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(LCI_ERR_CUDA, "index_select_noalloc: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kNoAllocMaxDevices)
+        return fail(LCI_ERR_UNSUPPORTED, "index_select_noalloc: device %d above %d", dev,
+                    kNoAllocMaxDevices - 1);
+    std::call_once(g_noalloc_once[dev], [dev] {
+        g_noalloc_err[dev] = cudaGetSymbolAddress(&g_noalloc_ptr[dev], g_noalloc_scratch);
+    });
+    if (g_noalloc_err[dev] != cudaSuccess)
+        return fail(LCI_ERR_CUDA, "index_select_noalloc: scratch address lookup failed: %s",
+                    cudaGetErrorString(g_noalloc_err[dev]));
+    *out = g_noalloc_ptr[dev];
+    return LCI_OK;
+}
+}  // namespace
+
+extern "C" lci_status lci_index_select_noalloc(const void* q_c, const void* k_c, lci_dtype dtype,
+                                               int32_t batch, int32_t S, int32_t H_i, int32_t d_c,
+                                               int32_t block_size, int32_t nb_max,
+                                               const int32_t* d_ctx_len, const int32_t* d_q_start,
+                                               int32_t topk, lci_phase phase, int32_t* d_ids,
+                                               void* stream) {
+    if (!q_c || !k_c || !d_ctx_len || !d_q_start || !d_ids)
+        return fail(LCI_ERR_INVALID_ARG, "index_select_noalloc: null pointer argument");
+    if (block_size <= 0)
+        return fail(LCI_ERR_INVALID_ARG, "index_select_noalloc: block_size must be positive");
+    lci_status st = check_index_args(batch, S, H_i, d_c, nb_max, topk, dtype);
+    if (st != LCI_OK) return st;
+    if (phase != LCI_PHASE_AUTO && phase != LCI_PHASE_PREFILL && phase != LCI_PHASE_DECODE)
+        return fail(LCI_ERR_INVALID_ARG, "index_select_noalloc: unknown phase %d", (int)phase);
+    if (!aligned16(q_c) || !aligned16(k_c))
+        return fail(LCI_ERR_INVALID_ARG, "index_select_noalloc: q_c and k_c must be 16-byte aligned");
+    const int K = H_i * d_c;
+    const IndexPlan pl = plan_index(batch, S, K, nb_max, dtype_size(dtype));
+    if (pl.bytes > (size_t)LCI_NOALLOC_SCRATCH_BYTES)
+        return fail(LCI_ERR_WORKSPACE, "index_select_noalloc: these sizes need %zu bytes of scratch; "
+                    "the built-in scratch holds %u", pl.bytes, (unsigned)LCI_NOALLOC_SCRATCH_BYTES);
+    void* scratch = nullptr;
+    st = noalloc_scratch(&scratch);
+    if (st != LCI_OK) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    // The arrival counters must start at zero; the array holds the last call's data.
+    cudaError_t e = cudaMemsetAsync(static_cast<char*>(scratch) + pl.off_counters, 0,
+                                    (size_t)batch * S * sizeof(unsigned int), cs);
+    if (e != cudaSuccess) return fail(LCI_ERR_CUDA, "index_select_noalloc: %s", cudaGetErrorString(e));
+    if (dtype == LCI_F32)
+        return launch_index_gemv<float>(q_c, k_c, batch, S, K, block_size, nb_max, d_ctx_len,
+                                        d_q_start, topk, d_ids, scratch, pl, cs);
+    return launch_index_gemv<__nv_bfloat16>(q_c, k_c, batch, S, K, block_size, nb_max, d_ctx_len,
+                                            d_q_start, topk, d_ids, scratch, pl, cs);
+}
+
+extern "C" {
+
 lci_status lci_get_device_status(void* stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(LCI_ERR_CUDA, "get_device_status: %s", cudaGetErrorString(e));

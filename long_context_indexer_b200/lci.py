@@ -47,6 +47,8 @@ SIGNATURES = {
     "lci_sparse_attn": (_st, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _f32,
                               _st, _vp, _vp, _sz, _vp]),
     "lci_get_device_status": (_st, [_vp]),
+    "lci_index_select_noalloc": (_st, [_vp, _vp, _st, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp,
+                                       _i32, _st, _vp, _vp]),
 }
 
 _lib = None
@@ -227,6 +229,26 @@ def index_select(q_c: torch.Tensor, k_c: torch.Tensor, block_size: int, ctx_len:
         _dev(q_start, "q_start", torch.int32, 1), topk, PHASES[phase],
         _dev(ids, "ids", torch.int32, 3), _dev(ws, "workspace"), ws.numel() * ws.element_size(),
         _stream(stream)), "lci_index_select")
+    return ids
+
+
+def index_select_noalloc(q_c: torch.Tensor, k_c: torch.Tensor, block_size: int,
+                         ctx_len: torch.Tensor, q_start: torch.Tensor, topk: int,
+                         phase: str = "auto", ids: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """index_select through lci_index_select_noalloc: no workspace, no device
+    allocation inside the library (its scratch is a fixed array in liblci.so)."""
+    B, S, H_i, d_c = q_c.shape
+    nb_max = k_c.shape[1]
+    if k_c.shape[0] != B or k_c.shape[2:] != q_c.shape[2:] or k_c.dtype != q_c.dtype:
+        raise ValueError("lci: k_c must be [B, nb_max, H_i, d_c] with q_c's dtype")
+    if ids is None:
+        ids = torch.empty((B, S, topk), dtype=torch.int32, device=q_c.device)
+    _check(load_library().lci_index_select_noalloc(
+        _dev(q_c, "q_c", None, 4), _dev(k_c, "k_c", q_c.dtype, 4), _dtype_code(q_c), B, S, H_i, d_c,
+        block_size, nb_max, _dev(ctx_len, "ctx_len", torch.int32, 1),
+        _dev(q_start, "q_start", torch.int32, 1), topk, PHASES[phase],
+        _dev(ids, "ids", torch.int32, 3), _stream(stream)), "lci_index_select_noalloc")
     return ids
 
 
