@@ -112,11 +112,18 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
         }
     }
 
-    // Block ids come from the previous kernel on the stream.
-    pdl_wait();
+    // Positions and the block table are inputs of the step; warm the table row
+    // into L2 so the page lookups after the wait hit it.
     const long long p = (long long)q_start[b] + s;
     const long long ctx = ctx_len[b];
     const long long last = p < ctx - 1 ? p : ctx - 1;
+    if (warp == kConsumers) {
+        const int32_t* trow = table + (size_t)b * nb_max;
+        const int nlines = min(nb_max, 8192) / 32;  // 128-byte lines of the row
+        for (int l = lane; l < nlines; l += 32) prefetch_l2(trow + l * 32);
+    }
+    // Block ids come from the previous kernel on the stream.
+    pdl_wait();
 
     float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
     float o[2][8][4];
@@ -285,10 +292,20 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
     __syncthreads();  // every stage consumed: the ring memory is free
 
     // ---------------- combine the four warps ----------------
-    // Warp partials: m, l [4][16]; O [4][16][128] fp32 (32 KiB in the ring).
-    float* wo = reinterpret_cast<float*>(smem);
-    float* wm = wo + kConsumers * kRows * kHD;
-    float* wl = wm + kConsumers * kRows;
+    // Partials stay in the accumulator fragment layout: slot o = 32*h + 4*i + e
+    // of lane l holds head (l>>2) + 8*(e>>1), dim 64*h + 16*(l&3) + 8*(e&1) + i.
+    // Every exchange below is a conflict-free [slot][lane] access.
+    constexpr int kSlots = 64;                 // fp32 accumulators per thread
+    constexpr int kElems = kSlots * 32;        // = 16 heads x 128 dims
+    float* wo = reinterpret_cast<float*>(smem);          // [kConsumers][kSlots][32]
+    float* wm = wo + kConsumers * kElems;                 // [kConsumers][16]
+    float* wl = wm + kConsumers * kRows;                  // [kConsumers][16]
+    float* wf = wl + kConsumers * kRows;                  // [kConsumers][16] weights
+    float* cm = wf + kConsumers * kRows;                  // [16] CTA max
+    float* cl = cm + kRows;                               // [16] CTA sum
+    float* co = cl + kRows;                               // [kSlots][32] CTA partial
+    float* xf = co + kElems;                              // [kMaxSplit][16]
+    float* xl = xf + kMaxSplit * kRows;                   // [16]
     if (warp < kConsumers) {
         l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
         l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
@@ -300,25 +317,15 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
             wl[warp * kRows + g8] = l_a;
             wl[warp * kRows + g8 + 8] = l_b;
         }
-        float* oa = wo + (warp * kRows + g8) * kHD;
-        float* ob = oa + 8 * kHD;
+        float* dst = wo + warp * kElems + lane;
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int da = 64 * h + 16 * q4 + i, db = da + 8;
-                oa[da] = o[h][i][0];
-                oa[db] = o[h][i][1];
-                ob[da] = o[h][i][2];
-                ob[db] = o[h][i][3];
-            }
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) dst[(32 * h + 4 * i + e) * 32] = o[h][i][e];
     }
     __syncthreads();
-    // CTA partial: cm, cl [16], co [16][128] (after the warp partials).
-    float* co = wl + kConsumers * kRows;
-    float* cm = co + kRows * kHD;
-    float* cl = cm + kRows;
-    float* wf = cl + kRows;  // [kConsumers][16] merge weights of the warps
     if (tid < kRows) {
         float M = -INFINITY;
 #pragma unroll
@@ -335,28 +342,28 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
         cl[tid] = L;
     }
     __syncthreads();
-    for (int e = tid; e < kRows * kHD; e += kThreads) {
-        const int r = e / kHD;
+    __nv_bfloat16* orow = out + ((size_t)row * H_q + (size_t)g * G) * kHD;
+    for (int sidx = tid; sidx < kElems; sidx += kThreads) {
+        const int ln = sidx & 31, oi = sidx >> 5, e = oi & 3;
+        const int head = (ln >> 2) + 8 * (e >> 1);
         float acc = 0.f;
 #pragma unroll
-        for (int w2 = 0; w2 < kConsumers; ++w2) acc += wf[w2 * kRows + r] * wo[w2 * kRows * kHD + e];
-        co[e] = acc;
-    }
-
-    __nv_bfloat16* orow = out + ((size_t)row * H_q + (size_t)g * G) * kHD;
-    if (nsplit == 1) {
-        __syncthreads();
-        for (int e = tid; e < G * kHD; e += kThreads) {
-            const float L = cl[e / kHD];
-            orow[e] = __float2bfloat16_rn(L > 0.f ? co[e] / L : 0.f);
+        for (int w2 = 0; w2 < kConsumers; ++w2) acc += wf[w2 * kRows + head] * wo[w2 * kElems + sidx];
+        if (nsplit == 1) {
+            if (head < G) {
+                const int dim = 64 * (oi >> 5) + 16 * (ln & 3) + 8 * (e & 1) + ((oi >> 2) & 7);
+                const float L = cl[head];
+                orow[head * kHD + dim] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
+            }
+        } else {
+            co[sidx] = acc;
         }
-        return;
     }
+    if (nsplit == 1) return;
+
     // ---------------- combine the CTAs of the cluster (DSMEM) ----------------
     cg::cluster_group cluster = cg::this_cluster();
     cluster.sync();
-    float* xf = wf + kConsumers * kRows;  // [kMaxSplit][16] merge weights of the CTAs
-    float* xl = xf + kMaxSplit * kRows;   // [16] 1 / merged sum
     if (tid < kRows) {
         float mc[kMaxSplit];
         float M = -INFINITY;
@@ -376,18 +383,21 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
         xl[tid] = L > 0.f ? 1.f / L : 0.f;
     }
     __syncthreads();
-    const int nel = G * kHD;
-    const int chunk = (nel + nsplit - 1) / nsplit;
-    const int e0 = split * chunk, e1 = min(nel, e0 + chunk);
-    for (int e = e0 + tid; e < e1; e += kThreads) {
-        const int r = e / kHD;
+    const int chunk = (kElems + nsplit - 1) / nsplit;
+    const int e0 = split * chunk, e1 = min(kElems, e0 + chunk);
+    for (int sidx = e0 + tid; sidx < e1; sidx += kThreads) {
+        const int ln = sidx & 31, oi = sidx >> 5, e = oi & 3;
+        const int head = (ln >> 2) + 8 * (e >> 1);
         float v[kMaxSplit];
 #pragma unroll
-        for (int c = 0; c < kMaxSplit; ++c) v[c] = c < nsplit ? cluster.map_shared_rank(co, c)[e] : 0.f;
+        for (int c = 0; c < kMaxSplit; ++c) v[c] = c < nsplit ? cluster.map_shared_rank(co, c)[sidx] : 0.f;
         float acc = 0.f;
 #pragma unroll
-        for (int c = 0; c < kMaxSplit; ++c) acc += xf[c * kRows + r] * v[c];
-        orow[e] = __float2bfloat16_rn(acc * xl[r]);
+        for (int c = 0; c < kMaxSplit; ++c) acc += xf[c * kRows + head] * v[c];
+        if (head < G) {
+            const int dim = 64 * (oi >> 5) + 16 * (ln & 3) + 8 * (e & 1) + ((oi >> 2) & 7);
+            orow[head * kHD + dim] = __float2bfloat16_rn(acc * xl[head]);
+        }
     }
     cluster.sync();  // keep this CTA's partial alive until every reader is done
 }

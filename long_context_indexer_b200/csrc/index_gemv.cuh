@@ -32,18 +32,23 @@ __device__ __forceinline__ float dot_chunk(const uint4& raw, const float* q, __n
            d.x * q[6] + d.y * q[7];
 }
 
-template <typename T, int NT>
+// KV > 0: every block key is KV*32 16-byte chunks (2 KiB for KV = 4) and lane l
+// always owns chunks l + 32*c, so its slice of the query row lives in
+// registers. KV == 0: any size, query row staged in shared memory.
+template <typename T, int NT, int KV>
 __global__ void __launch_bounds__(NT) index_gemv_select_kernel(
     const T* __restrict__ q_c, const T* __restrict__ k_c, int S, int K, int nb_max, int bs,
     const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ q_start, int topk,
     int chunk_blocks, int nchunks, float* __restrict__ scores,
-    unsigned int* __restrict__ counters, int32_t* __restrict__ ids) {
-    // Dynamic shared memory: [k_c chunk: chunk_blocks * K * sizeof(T)][q row: K floats];
-    // after scoring, the first nb_max * 4 bytes hold the row's radix keys.
+    uint32_t* __restrict__ chunk_max, unsigned int* __restrict__ counters,
+    int32_t* __restrict__ ids) {
+    // Dynamic shared memory: [k_c chunk: chunk_blocks * K * sizeof(T)]
+    // [query row: K floats, only when KV == 0]; the last CTA of a row reuses it
+    // for the select's scratch.
     extern __shared__ __align__(128) unsigned char dyn_smem[];
-    __shared__ SelectSmem sel;
     __shared__ uint64_t bar;
     __shared__ int s_last;
+    __shared__ uint32_t s_max;
     constexpr int NW = NT / 32;
     constexpr int E = ElemsPer16B<T>::v;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -57,10 +62,11 @@ __global__ void __launch_bounds__(NT) index_gemv_select_kernel(
     const int j0 = chunk * chunk_blocks;
     const int j1 = min(j0 + chunk_blocks, vis);
     const size_t row_bytes = (size_t)K * sizeof(T);
+    float* row_scores = scores + (size_t)row * nb_max;
 
+    if (tid == 0) s_max = 0u;  // below every real key
     if (j0 < j1) {
         unsigned char* tile = dyn_smem;
-        float* qs = reinterpret_cast<float*>(dyn_smem + (size_t)chunk_blocks * row_bytes);
         if (tid == 0) {
             mbar_init(&bar, 1);
             fence_mbar_init();
@@ -73,18 +79,49 @@ __global__ void __launch_bounds__(NT) index_gemv_select_kernel(
                 bulk_load(tile + off, src + off, min(16384u, bytes - off), &bar);
         }
         const T* qrow = q_c + (size_t)row * K;
-        for (int i = tid; i < K; i += NT) qs[i] = to_f32(qrow[i]);
-        __syncthreads();
-        const bool ok = mbar_wait(&bar, 0);
-        const int nvec = K / E;
-        for (int j = j0 + warp; ok && j < j1; j += NW) {
-            const uint4* kr = reinterpret_cast<const uint4*>(tile + (size_t)(j - j0) * row_bytes);
-            float acc = 0.f;
-            for (int c = lane; c < nvec; c += 32) acc += dot_chunk(kr[c], qs + c * E, T());
-            acc = warp_sum(acc);
-            if (lane == 0) scores[(size_t)row * nb_max + j] = acc;
+        if constexpr (KV > 0) {
+            // this lane's query slice: chunks lane + 32*c, E elements each
+            float qv[KV][E];
+#pragma unroll
+            for (int c = 0; c < KV; ++c) {
+                const uint4 raw = *reinterpret_cast<const uint4*>(qrow + (lane + 32 * c) * E);
+                const T* e8 = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+                for (int e = 0; e < E; ++e) qv[c][e] = to_f32(e8[e]);
+            }
+            __syncthreads();
+            const bool ok = mbar_wait(&bar, 0);
+            for (int j = j0 + warp; ok && j < j1; j += NW) {
+                const uint4* kr = reinterpret_cast<const uint4*>(tile + (size_t)(j - j0) * row_bytes);
+                float acc = 0.f;
+#pragma unroll
+                for (int c = 0; c < KV; ++c) acc += dot_chunk(kr[lane + 32 * c], qv[c], T());
+                acc = warp_sum(acc);
+                if (lane == 0) {
+                    row_scores[j] = acc;
+                    atomicMax(&s_max, score_key(acc));
+                }
+            }
+        } else {
+            float* qs = reinterpret_cast<float*>(dyn_smem + (size_t)chunk_blocks * row_bytes);
+            for (int i = tid; i < K; i += NT) qs[i] = to_f32(qrow[i]);
+            __syncthreads();
+            const bool ok = mbar_wait(&bar, 0);
+            const int nvec = K / E;
+            for (int j = j0 + warp; ok && j < j1; j += NW) {
+                const uint4* kr = reinterpret_cast<const uint4*>(tile + (size_t)(j - j0) * row_bytes);
+                float acc = 0.f;
+                for (int c = lane; c < nvec; c += 32) acc += dot_chunk(kr[c], qs + c * E, T());
+                acc = warp_sum(acc);
+                if (lane == 0) {
+                    row_scores[j] = acc;
+                    atomicMax(&s_max, score_key(acc));
+                }
+            }
         }
     }
+    __syncthreads();
+    if (tid == 0 && j0 < j1) chunk_max[(size_t)row * nchunks + chunk] = s_max;
     __threadfence();
     __syncthreads();
     if (tid == 0) {
@@ -95,10 +132,9 @@ __global__ void __launch_bounds__(NT) index_gemv_select_kernel(
     if (!s_last) return;
     __threadfence();
     if (tid == 0) counters[row] = 0u;
-    uint32_t* keys = reinterpret_cast<uint32_t*>(dyn_smem);
-    for (int i = tid; i < vis; i += NT) keys[i] = score_key(__ldcg(&scores[(size_t)row * nb_max + i]));
-    __syncthreads();
-    cta_topk_from_keys<NT>(keys, vis, topk, ids + (size_t)row * topk, sel);
+    SelectSmem& sel = *reinterpret_cast<SelectSmem*>(dyn_smem);
+    cta_topk_select<NT>(row_scores, chunk_max + (size_t)row * nchunks, vis, chunk_blocks, topk,
+                        ids + (size_t)row * topk, sel);
 }
 
 }  // namespace lci

@@ -74,7 +74,8 @@ constexpr int kIndexMaxSmem = 65536 + 1024;
 
 struct IndexPlan {
     int chunk_blocks, nchunks;
-    size_t off_counters, off_scores, bytes;
+    bool qreg;  // 2 KiB block keys: query slice in registers
+    size_t off_counters, off_scores, off_chunk_max, bytes;
     size_t smem;
 };
 
@@ -91,10 +92,12 @@ IndexPlan plan_index(int32_t batch, int32_t S, int32_t K, int32_t nb_max, size_t
     pl.nchunks = (nb_max + chunk - 1) / chunk;
     pl.off_counters = 0;
     pl.off_scores = align_up((size_t)rows * sizeof(unsigned int));
-    pl.bytes = pl.off_scores + align_up((size_t)rows * nb_max * sizeof(float));
-    const size_t stage = (size_t)chunk * row_bytes + (size_t)K * sizeof(float);
-    const size_t keys = (size_t)nb_max * sizeof(uint32_t);
-    pl.smem = stage > keys ? stage : keys;
+    pl.off_chunk_max = pl.off_scores + align_up((size_t)rows * nb_max * sizeof(float));
+    pl.bytes = pl.off_chunk_max + align_up((size_t)rows * pl.nchunks * sizeof(uint32_t));
+    pl.qreg = row_bytes == 2048;
+    const size_t stage = (size_t)chunk * row_bytes + (pl.qreg ? 0 : (size_t)K * sizeof(float));
+    const size_t sel = sizeof(lci::SelectSmem);
+    pl.smem = stage > sel ? stage : sel;
     return pl;
 }
 
@@ -122,14 +125,20 @@ lci_status launch_index_gemv(const void* q_c, const void* k_c, int32_t batch, in
                              int32_t bs, int32_t nb_max, const int32_t* ctx_len,
                              const int32_t* q_start, int32_t topk, int32_t* ids, void* ws,
                              const IndexPlan& pl, cudaStream_t st) {
-    auto kern = lci::index_gemv_select_kernel<T, kIndexThreads>;
+    constexpr int KV = 2048 / (16 * 32);
+    auto kern = pl.qreg ? lci::index_gemv_select_kernel<T, kIndexThreads, KV>
+                        : lci::index_gemv_select_kernel<T, kIndexThreads, 0>;
     // Largest dynamic shared memory any plan asks for: 32 KiB of block keys
-    // plus an 8192-float query row, or 16384 radix keys.
+    // plus an 8192-float query row.
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [kern] {
-        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        kIndexMaxSmem);
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(lci::index_gemv_select_kernel<T, kIndexThreads, KV>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kIndexMaxSmem);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(lci::index_gemv_select_kernel<T, kIndexThreads, 0>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            kIndexMaxSmem);
     });
     if (attr_err != cudaSuccess)
         return fail(LCI_ERR_CUDA, "index_select: %s", cudaGetErrorString(attr_err));
@@ -140,6 +149,7 @@ lci_status launch_index_gemv(const void* q_c, const void* k_c, int32_t batch, in
     kern<<<grid, kIndexThreads, pl.smem, st>>>(
         static_cast<const T*>(q_c), static_cast<const T*>(k_c), S, K, nb_max, bs, ctx_len, q_start,
         topk, pl.chunk_blocks, pl.nchunks, reinterpret_cast<float*>(w + pl.off_scores),
+        reinterpret_cast<uint32_t*>(w + pl.off_chunk_max),
         reinterpret_cast<unsigned int*>(w + pl.off_counters), ids);
     return check_launch("index_select");
 }
