@@ -16,6 +16,8 @@
 //     key; keys in higher bins are in; keys of that boundary bin are ranked
 //     exactly (key desc, block id asc) among themselves.
 //  3. The k winners are ranked and written in order, padded with -1.
+// Ranks are computed a warp per element: 32 lanes compare at once and a
+// ballot counts the elements ranked ahead.
 // If the candidates overflow the shared buffers (long rows of equal scores), a
 // four-pass radix select over all scores, read from global memory, takes over.
 #pragma once
@@ -65,20 +67,38 @@ __device__ __forceinline__ int block_incl_scan(int v, int* warp_tot) {
     return v + off;
 }
 
+// Rank of every element e of keys/ids[0..m) among the same m elements, by
+// (key desc, id asc): one warp per element, lanes compare 32 elements at once
+// and a ballot counts the ones ranked ahead. Calls f(e, rank) from lane 0.
+template <int NT, typename F>
+__device__ __forceinline__ void warp_ranks(const uint32_t* keys, const int32_t* ids, int m, F f) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int e = warp; e < m; e += NT / 32) {
+        const uint32_t ke = keys[e];
+        const int ie = ids[e];
+        int rank = 0;
+        for (int base = 0; base < m; base += 32) {
+            const int j = base + lane;
+            bool ahead = false;
+            if (j < m) {
+                const uint32_t kj = keys[j];
+                ahead = (kj > ke) || (kj == ke && ids[j] < ie);
+            }
+            rank += __popc(__ballot_sync(0xffffffffu, ahead));
+        }
+        if (lane == 0) f(e, rank);
+    }
+}
+
 // Top k of the m candidates cand_key/cand_id[0..m) (k <= m, k <= kMaxTopk,
 // m <= kCandCap). Leaves the k winners, unordered, in win_key/win_id.
 template <int NT>
 __device__ void select_candidates(int m, int k, SelectSmem& sm) {
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int tid = threadIdx.x;
     for (int i = tid; i < kSelBins; i += NT) sm.hist[i] = 0u;
     if (tid < 8) sm.bcast[tid] = 0;
     __syncthreads();
-    for (int base = 0; base < m; base += NT) {
-        const int i = base + tid;
-        const uint32_t bin = i < m ? sm.cand_key[i] >> kSelShift : 0xffffffffu;
-        const unsigned peers = __match_any_sync(0xffffffffu, bin);
-        if (i < m && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[bin], (unsigned)__popc(peers));
-    }
+    for (int i = tid; i < m; i += NT) atomicAdd(&sm.hist[sm.cand_key[i] >> kSelShift], 1u);
     __syncthreads();
     // thread t owns bins 2047-8t .. 2040-8t (descending)
     int c[8], lsum = 0;
@@ -124,19 +144,12 @@ __device__ void select_candidates(int m, int k, SelectSmem& sm) {
     }
     __syncthreads();
     const int nb = min(sm.bcast[4], kMaxBoundary);  // never clipped: nb <= m <= kCandCap
-    for (int e = tid; e < nb; e += NT) {
-        const uint32_t ke = sm.bnd_key[e];
-        const int ie = sm.bnd_id[e];
-        int rank = 0;
-        for (int f = 0; f < nb; ++f) {
-            const uint32_t kf = sm.bnd_key[f];
-            rank += (kf > ke) || (kf == ke && sm.bnd_id[f] < ie);
-        }
+    warp_ranks<NT>(sm.bnd_key, sm.bnd_id, nb, [&](int e, int rank) {
         if (rank < need && above + rank < kMaxTopk) {
-            sm.win_key[above + rank] = ke;
-            sm.win_id[above + rank] = ie;
+            sm.win_key[above + rank] = sm.bnd_key[e];
+            sm.win_id[above + rank] = sm.bnd_id[e];
         }
-    }
+    });
     __syncthreads();
 }
 
@@ -289,16 +302,7 @@ __device__ void cta_topk_select(const float* scores, const uint32_t* chunk_max, 
     else
         radix_select_global<NT>(scores, n, k, sm);
     // 3. rank the k winners (key desc, id asc) and write them in order
-    for (int e = tid; e < k; e += NT) {
-        const uint32_t ke = sm.win_key[e];
-        const int ie = sm.win_id[e];
-        int rank = 0;
-        for (int f = 0; f < k; ++f) {
-            const uint32_t kf = sm.win_key[f];
-            rank += (kf > ke) || (kf == ke && sm.win_id[f] < ie);
-        }
-        out[rank] = ie;
-    }
+    warp_ranks<NT>(sm.win_key, sm.win_id, k, [&](int e, int rank) { out[rank] = sm.win_id[e]; });
     for (int i = k + tid; i < topk; i += NT) out[i] = -1;
 }
 
