@@ -1,0 +1,338 @@
+// index_prefill.cuh -- block scoring fused with the causal-masked top-k on the
+// 5th-generation tensor cores (tcgen05 + TMEM), for many queries per sequence.
+//
+// score[s, j] = q_c[s, :] . k_c[j, :] is a dense [S x NB] GEMM over
+// K = H_i * d_c ([AI-acc] §4.1, matmul of compressed queries and keys). Each
+// CTA owns a 128-query m-tile and a range of 256-block n-tiles:
+//
+//   warp 0      TMA producer: 64-wide K slices of q_c (128 rows) and k_c
+//               (256 rows), 128-byte swizzle, into a 4-stage ring;
+//   warp 1      one thread issues tcgen05.mma (M=128, N=256, K=16, bf16 ->
+//               fp32) into one of two TMEM accumulators (2 x 256 columns) and
+//               commits stage releases / accumulator-ready signals;
+//   warps 2..5  epilogue: thread r owns query row r (TMEM lane r). It reads
+//               its 256 scores with tcgen05.ld, drops blocks that are not
+//               causal-visible, and keeps a running exact top-k in registers
+//               behind a threshold test. Scores never reach global memory
+//               ([GPU-stack] "Operatorizing Index Selection": scoring, top-k
+//               and masking fused in one pass).
+//
+// n-tiles beyond the last visible block of the m-tile are skipped. When an
+// m-tile's n-tiles are split over several CTAs, each writes its per-row
+// candidates (key, id) to the workspace and the last CTA to arrive (atomic
+// counter, no spin-wait) merges them. Ties break to the lower block id.
+#pragma once
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace lci {
+
+namespace pre {
+constexpr int kBM = 128, kBN = 256, kBK = 64;
+constexpr int kStages = 4;
+constexpr int kThreads = 192;
+constexpr int kABytes = kBM * kBK * 2;   // 16 KiB
+constexpr int kBBytes = kBN * kBK * 2;   // 32 KiB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kTmemCols = 2 * kBN;       // two accumulators
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+// instruction descriptor: D fp32, A/B bf16, both K-major, N = 256, M = 128
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
+                            ((uint32_t)(kBM >> 4) << 24);
+}  // namespace pre
+
+// Shared-memory matrix descriptor of a K-major tile written by TMA with the
+// 128-byte swizzle: 8-row groups 1024 bytes apart, sm_100 descriptor version.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
+    return (uint64_t)((smem_addr >> 4) & 0x3fff) | ((uint64_t)1 << 16) /* LBO (unused) */ |
+           ((uint64_t)(1024 >> 4) << 32) /* SBO */ | ((uint64_t)1 << 46) /* version */ |
+           ((uint64_t)2 << 61) /* SWIZZLE_128B */;
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Sorted (key desc) running top-KT list held in registers. A new element with
+// a key equal to an entry comes later in block order, so it ranks behind it.
+template <int KT>
+struct RowTopK {
+    uint32_t key[KT];
+    int32_t id[KT];
+    __device__ __forceinline__ void init() {
+#pragma unroll
+        for (int i = 0; i < KT; ++i) {
+            key[i] = 0u;  // below every real key
+            id[i] = -1;
+        }
+    }
+    __device__ __forceinline__ uint32_t threshold() const { return key[KT - 1]; }
+    // Insert (k, j) when k > threshold(): shift the smaller entries down.
+    __device__ __forceinline__ void insert(uint32_t k, int32_t j) {
+#pragma unroll
+        for (int i = KT - 1; i > 0; --i) {
+            const bool take_prev = k > key[i - 1];
+            const bool here = !take_prev && k > key[i];
+            key[i] = take_prev ? key[i - 1] : (here ? k : key[i]);
+            id[i] = take_prev ? id[i - 1] : (here ? j : id[i]);
+        }
+        if (k > key[0]) {
+            key[0] = k;
+            id[0] = j;
+        }
+    }
+};
+
+template <int KT>
+__global__ void __launch_bounds__(pre::kThreads, 1) index_prefill_tc_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, int S,
+    int nb_max, int bs, const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ q_start,
+    int topk, int ksteps, int m_tiles, int n_split, uint32_t* __restrict__ part_key,
+    int32_t* __restrict__ part_id, unsigned int* __restrict__ counters,
+    int32_t* __restrict__ ids) {
+    using namespace pre;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+    uint64_t* empty_bar = full_bar + kStages;
+    uint64_t* tfull_bar = empty_bar + kStages;
+    uint64_t* tempty_bar = tfull_bar + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + 2);
+    int* s_last = reinterpret_cast<int*>(tmem_slot + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ns = blockIdx.x, mt = blockIdx.y, b = blockIdx.z;
+    const int row0 = mt * kBM;
+
+    // Visible n-tiles of this m-tile (causal), and this CTA's share of them.
+    const long long ctx = ctx_len[b];
+    const long long p_last = (long long)q_start[b] + min(S - 1, row0 + kBM - 1);
+    const int vis_max = visible_blocks(p_last, ctx, bs, nb_max);
+    const int n_tiles = (vis_max + kBN - 1) / kBN;
+    const int per = (n_tiles + n_split - 1) / n_split;
+    const int t_lo = ns * per;
+    const int t_hi = min(n_tiles, t_lo + per);
+    const int my_tiles = max(0, t_hi - t_lo);
+
+    if (tid == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&full_bar[i], 1);
+            mbar_init(&empty_bar[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull_bar[i], 1);
+            mbar_init(&tempty_bar[i], 4);  // one arrive per epilogue warp
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) {  // the whole warp allocates the two accumulators
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            int it = 0;
+            for (int t = 0; t < my_tiles; ++t) {
+                const int n0 = (t_lo + t) * kBN;
+                for (int ks = 0; ks < ksteps; ++ks, ++it) {
+                    const int st = it % kStages;
+                    if (it >= kStages && !mbar_wait(&empty_bar[st], ((it / kStages) - 1) & 1)) break;
+                    unsigned char* a = smem + st * kStageBytes;
+                    mbar_arrive_expect_tx(&full_bar[st], kStageBytes);
+                    tma_load_2d(a, &tm_q, ks * kBK, b * S + row0, &full_bar[st]);
+                    tma_load_2d(a + kABytes, &tm_k, ks * kBK, b * nb_max + n0, &full_bar[st]);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            int it = 0;
+            bool ok = true;
+            for (int t = 0; t < my_tiles && ok; ++t) {
+                const int buf = t & 1;
+                if (t >= 2) ok = mbar_wait(&tempty_bar[buf], ((t >> 1) - 1) & 1);
+                tc_fence_after();
+                const uint32_t d = tmem_base + (uint32_t)(buf * kBN);
+                for (int ks = 0; ks < ksteps && ok; ++ks, ++it) {
+                    const int st = it % kStages;
+                    ok = mbar_wait(&full_bar[st], (it / kStages) & 1);
+                    tc_fence_after();
+                    const uint32_t a = smem_u32(smem + st * kStageBytes);
+                    const uint64_t ad = sw128_desc(a), bd = sw128_desc(a + kABytes);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)  // +32 bytes per K=16 step
+                        tc_mma(d, ad + 2 * kk, bd + 2 * kk, kIdesc, (ks | kk) != 0);
+                    tc_commit(&empty_bar[st]);  // the stage is free once these MMAs finish
+                }
+                tc_commit(&tfull_bar[buf]);  // accumulator ready
+            }
+        }
+    } else {
+        // ---------------- epilogue: one query row per thread ----------------
+        const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+        const int r = quarter * 32 + lane;
+        const int s = row0 + r;
+        const long long p = (long long)q_start[b] + s;
+        const int vis = s < S ? visible_blocks(p, ctx, bs, nb_max) : 0;
+        RowTopK<KT> top;
+        top.init();
+        for (int t = 0; t < my_tiles; ++t) {
+            const int buf = t & 1;
+            const bool ok = mbar_wait(&tfull_bar[buf], (t >> 1) & 1);
+            tc_fence_after();
+            const int n0 = (t_lo + t) * kBN;
+            if (ok) {
+#pragma unroll 1
+                for (int c = 0; c < kBN / 32; ++c) {
+                    float v[32];
+                    tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kBN + c * 32), v);
+                    const int jb = n0 + c * 32;
+                    if (jb >= vis) continue;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const uint32_t key = score_key(v[i]);
+                        if (jb + i < vis && key > top.threshold()) top.insert(key, jb + i);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+        }
+        // ---------------- output ----------------
+        if (n_split == 1) {
+            if (s < S) {
+                int32_t* orow = ids + ((size_t)b * S + s) * topk;
+#pragma unroll
+                for (int i = 0; i < KT; ++i)
+                    if (i < topk) orow[i] = top.id[i];
+            }
+        } else {
+            const size_t prow = (((size_t)b * m_tiles + mt) * kBM + r) * n_split + ns;
+#pragma unroll
+            for (int i = 0; i < KT; ++i) {
+                if (i < topk) {
+                    part_key[prow * topk + i] = top.key[i];
+                    part_id[prow * topk + i] = top.id[i];
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(kTmemCols)
+                     : "memory");
+    }
+    if (n_split == 1) return;
+
+    // ---------------- merge the split candidates (last CTA of the m-tile) ----------------
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        unsigned int* ctr = counters + (size_t)b * m_tiles + mt;
+        const unsigned prev = atomicAdd(ctr, 1u);
+        *s_last = prev == (unsigned)(n_split - 1);
+        if (*s_last) *ctr = 0u;  // ready for the next call
+    }
+    __syncthreads();
+    if (!*s_last) return;
+    __threadfence();
+    // Copy the m-tile's candidate lists [128 rows][n_split][topk] into the
+    // (idle) stage memory with coalesced loads, then merge per row.
+    const int per_row = n_split * topk;
+    const size_t base = ((size_t)b * m_tiles + mt) * kBM * per_row;
+    uint32_t* mk = reinterpret_cast<uint32_t*>(smem);
+    int32_t* mi = reinterpret_cast<int32_t*>(smem) + kBM * per_row;
+#pragma unroll 4
+    for (int e = tid; e < kBM * per_row; e += kThreads) {
+        mk[e] = __ldcg(part_key + base + e);
+        mi[e] = __ldcg(part_id + base + e);
+    }
+    __syncthreads();
+    if (warp < 2) return;
+    const int r = (warp & 3) * 32 + lane;
+    const int s = row0 + r;
+    if (s >= S) return;
+    const uint32_t* rk = mk + r * per_row;
+    const int32_t* ri = mi + r * per_row;
+    // k-way merge of the n_split sorted lists: (key desc, id asc)
+    int head[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) head[q] = 0;
+    int32_t* orow = ids + ((size_t)b * S + s) * topk;
+    for (int i = 0; i < topk; ++i) {
+        int best = -1;
+        uint32_t bk = 0;
+        int32_t bi = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            if (q >= n_split || head[q] >= topk) continue;
+            const uint32_t kq = rk[q * topk + head[q]];
+            const int32_t iq = ri[q * topk + head[q]];
+            if (iq < 0) continue;  // sentinel: that list is exhausted
+            if (best < 0 || kq > bk || (kq == bk && iq < bi)) {
+                best = q;
+                bk = kq;
+                bi = iq;
+            }
+        }
+        orow[i] = best < 0 ? -1 : bi;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) head[q] += (q == best);
+    }
+}
+
+}  // namespace lci

@@ -19,6 +19,7 @@
 #include "common.cuh"
 #include "compress.cuh"
 #include "index_gemv.cuh"
+#include "index_prefill.cuh"
 #include "topk_select.cuh"
 
 struct lci_block_table {
@@ -224,6 +225,95 @@ lci_status encode_pool_map(CUtensorMap* map, const void* pool, long long rows) {
     return LCI_OK;
 }
 
+// Tensor-core schedule for many queries per sequence (index_prefill.cuh).
+struct PrefillPlan {
+    int m_tiles, n_split, kt, ksteps;
+    size_t off_counters, off_key, off_id, bytes;
+};
+
+PrefillPlan plan_prefill(int32_t batch, int32_t S, int32_t K, int32_t nb_max, int32_t topk) {
+    PrefillPlan pl{};
+    pl.m_tiles = (S + lci::pre::kBM - 1) / lci::pre::kBM;
+    pl.ksteps = K / lci::pre::kBK;
+    pl.kt = topk <= 16 ? 16 : (topk <= 32 ? 32 : 64);
+    const int n_tiles = (nb_max + lci::pre::kBN - 1) / lci::pre::kBN;
+    // about one CTA per SM; the merge copies n_split * topk candidates per row
+    // of a 128-row tile into the 192 KiB of stage memory
+    long long split = 148 / ((long long)batch * pl.m_tiles);
+    split = split < 1 ? 1 : split;
+    split = split > 8 ? 8 : split;
+    split = split > n_tiles ? n_tiles : split;
+    while (split > 1 && (long long)lci::pre::kBM * split * topk * 8 > 4 * lci::pre::kStageBytes) --split;
+    pl.n_split = (int)split;
+    const long long cand = (long long)batch * pl.m_tiles * lci::pre::kBM * pl.n_split * topk;
+    pl.off_counters = 0;
+    pl.off_key = align_up((size_t)batch * pl.m_tiles * sizeof(unsigned int));
+    pl.off_id = pl.off_key + align_up((size_t)cand * sizeof(uint32_t));
+    pl.bytes = pl.off_id + align_up((size_t)cand * sizeof(int32_t));
+    return pl;
+}
+
+bool prefill_path(lci_dtype dtype, lci_phase phase, int32_t S, int32_t K, int32_t topk,
+                  const void* q_c, const void* k_c) {
+    const lci_phase ph = resolve_phase(phase, S);
+    const bool wants = phase == LCI_PHASE_PREFILL || (ph == LCI_PHASE_PREFILL && S >= 32);
+    return wants && dtype == LCI_BF16 && K % lci::pre::kBK == 0 && topk <= 64 && aligned16(q_c) &&
+           aligned16(k_c);
+}
+
+lci_status encode_rows_map(CUtensorMap* map, const void* base, long long rows, int K, int box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return fail(LCI_ERR_CUDA, "index_select: cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {(cuuint32_t)lci::pre::kBK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(LCI_ERR_CUDA, "index_select: tensor map encode failed (%d)", (int)r);
+    return LCI_OK;
+}
+
+template <int KT>
+lci_status launch_prefill_kt(const CUtensorMap& tq, const CUtensorMap& tk, int32_t batch, int32_t S,
+                             int32_t nb_max, int32_t bs, const int32_t* ctx_len,
+                             const int32_t* q_start, int32_t topk, const PrefillPlan& pl,
+                             char* ws, int32_t* ids, cudaStream_t st) {
+    auto kern = lci::index_prefill_tc_kernel<KT>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [kern] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        lci::pre::kSmemBytes);
+    });
+    if (attr_err != cudaSuccess)
+        return fail(LCI_ERR_CUDA, "index_select: %s", cudaGetErrorString(attr_err));
+    dim3 grid((unsigned)pl.n_split, (unsigned)pl.m_tiles, (unsigned)batch);
+    kern<<<grid, lci::pre::kThreads, lci::pre::kSmemBytes, st>>>(
+        tq, tk, S, nb_max, bs, ctx_len, q_start, topk, pl.ksteps, pl.m_tiles, pl.n_split,
+        reinterpret_cast<uint32_t*>(ws + pl.off_key), reinterpret_cast<int32_t*>(ws + pl.off_id),
+        reinterpret_cast<unsigned int*>(ws + pl.off_counters), ids);
+    return check_launch("index_select");
+}
+
+lci_status launch_index_prefill(const void* q_c, const void* k_c, int32_t batch, int32_t S,
+                                int32_t K, int32_t bs, int32_t nb_max, const int32_t* ctx_len,
+                                const int32_t* q_start, int32_t topk, int32_t* ids, void* ws,
+                                const PrefillPlan& pl, cudaStream_t st) {
+    CUtensorMap tq, tk;
+    lci_status s = encode_rows_map(&tq, q_c, (long long)batch * S, K, lci::pre::kBM);
+    if (s != LCI_OK) return s;
+    s = encode_rows_map(&tk, k_c, (long long)batch * nb_max, K, lci::pre::kBN);
+    if (s != LCI_OK) return s;
+    char* w = static_cast<char*>(ws);
+    if (pl.kt == 16)
+        return launch_prefill_kt<16>(tq, tk, batch, S, nb_max, bs, ctx_len, q_start, topk, pl, w, ids, st);
+    if (pl.kt == 32)
+        return launch_prefill_kt<32>(tq, tk, batch, S, nb_max, bs, ctx_len, q_start, topk, pl, w, ids, st);
+    return launch_prefill_kt<64>(tq, tk, batch, S, nb_max, bs, ctx_len, q_start, topk, pl, w, ids, st);
+}
+
 bool decode_kernel_fits(const lci_block_table* t, int32_t H_q, const void* k_pool,
                         const void* v_pool) {
     const int G = H_q / t->num_kv_heads;
@@ -383,7 +473,9 @@ lci_status lci_index_select_workspace_size(int32_t batch, int32_t S, int32_t H_i
     lci_status st = check_index_args(batch, S, H_i, d_c, nb_max, topk, LCI_BF16);
     if (st != LCI_OK && st != LCI_ERR_UNSUPPORTED) return st;
     (void)phase;
-    *bytes = plan_index(batch, S, H_i * d_c, nb_max, 2).bytes;
+    const size_t g = plan_index(batch, S, H_i * d_c, nb_max, 2).bytes;
+    const size_t t = plan_prefill(batch, S, H_i * d_c, nb_max, topk).bytes;
+    *bytes = g > t ? g : t;  // enough for whichever schedule the call picks
     return ok();
 }
 
@@ -408,7 +500,13 @@ lci_status lci_index_select(const void* q_c, const void* k_c, lci_dtype dtype, i
         return fail(LCI_ERR_WORKSPACE, "index_select: workspace needs %zu bytes, 256-byte aligned "
                     "(got %zu at %p)", pl.bytes, workspace_bytes, workspace);
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    (void)resolve_phase(phase, S);
+    if (prefill_path(dtype, phase, S, K, topk, q_c, k_c)) {
+        const PrefillPlan pp = plan_prefill(batch, S, K, nb_max, topk);
+        if (workspace_bytes < pp.bytes)
+            return fail(LCI_ERR_WORKSPACE, "index_select: workspace needs %zu bytes", pp.bytes);
+        return launch_index_prefill(q_c, k_c, batch, S, K, block_size, nb_max, d_ctx_len, d_q_start,
+                                    topk, d_ids, workspace, pp, cs);
+    }
     if (dtype == LCI_F32)
         return launch_index_gemv<float>(q_c, k_c, batch, S, K, block_size, nb_max, d_ctx_len,
                                         d_q_start, topk, d_ids, workspace, pl, cs);
