@@ -31,12 +31,18 @@ namespace lci {
 namespace pre {
 constexpr int kBM = 128, kBN = 256, kBK = 64;
 constexpr int kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kChunk = 16;               // TMEM columns per epilogue load
 constexpr int kABytes = kBM * kBK * 2;   // 16 KiB
 constexpr int kBBytes = kBN * kBK * 2;   // 32 KiB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kTmemCols = 2 * kBN;       // two accumulators
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int kMaxEpi = 256;             // epilogue threads (8 warps)
+constexpr int kCandBytes = kChunk * kMaxEpi * 8;  // per epilogue thread: one chunk of (key, id)
+constexpr int kSmemBytes = kStages * kStageBytes + kCandBytes + 1024 /*align*/ + 256 /*barriers*/;
+// epilogue warps: 8 (two per TMEM lane quarter, each half of every tile's
+// columns) when the per-row list is short, 4 for KT = 64 (register budget)
+template <int KT> struct Epi { static constexpr int kWarps = KT <= 32 ? 8 : 4; };
+template <int KT> struct Cfg { static constexpr int kThreads = 64 + 32 * Epi<KT>::kWarps; };
 // instruction descriptor: D fp32, A/B bf16, both K-major, N = 256, M = 128
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
                             ((uint32_t)(kBM >> 4) << 24);
@@ -71,25 +77,33 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// 32 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
-    uint32_t r[32];
+// Asynchronous 16-column TMEM load: tmem_ld16_issue starts it, tmem_ld16_wait
+// completes it. The wait names the destination registers as read-write
+// operands, so the compiler cannot use them before the data has landed.
+__device__ __forceinline__ void tmem_ld16_issue(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15}, [%16];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
           "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+          "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_ld16_wait(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
 }
 
-// Sorted (key desc) running top-KT list held in registers. A new element with
-// a key equal to an entry comes later in block order, so it ranks behind it.
+// Running top-KT of one row, sorted by key descending, in registers. Entries
+// start as (key 0, id -1), below every real key. A new element with a key equal
+// to an entry comes later in block order, so it ranks behind it: it enters
+// only when its key is strictly above the last entry. The insertion is a
+// shift network: every position updates from its own and its predecessor's
+// old values, so the KT updates are independent of one another.
 template <int KT>
 struct RowTopK {
     uint32_t key[KT];
@@ -97,12 +111,14 @@ struct RowTopK {
     __device__ __forceinline__ void init() {
 #pragma unroll
         for (int i = 0; i < KT; ++i) {
-            key[i] = 0u;  // below every real key
+            key[i] = 0u;
             id[i] = -1;
         }
+        thr_f = -INFINITY;
     }
+    float thr_f;  // score of the last entry once the list is full
     __device__ __forceinline__ uint32_t threshold() const { return key[KT - 1]; }
-    // Insert (k, j) when k > threshold(): shift the smaller entries down.
+    __device__ __forceinline__ bool full() const { return id[KT - 1] >= 0; }
     __device__ __forceinline__ void insert(uint32_t k, int32_t j) {
 #pragma unroll
         for (int i = KT - 1; i > 0; --i) {
@@ -115,21 +131,29 @@ struct RowTopK {
             key[0] = k;
             id[0] = j;
         }
+        // back from key to score: the inverse of score_key
+        const uint32_t w = key[KT - 1];
+        thr_f = __uint_as_float((w & 0x80000000u) ? (w & 0x7fffffffu) : ~w);
     }
 };
 
 template <int KT>
-__global__ void __launch_bounds__(pre::kThreads, 1) index_prefill_tc_kernel(
+__global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, int S,
     int nb_max, int bs, const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ q_start,
     int topk, int ksteps, int m_tiles, int n_split, uint32_t* __restrict__ part_key,
     int32_t* __restrict__ part_id, unsigned int* __restrict__ counters,
     int32_t* __restrict__ ids) {
     using namespace pre;
+    constexpr int kThreads = Cfg<KT>::kThreads;
+    constexpr int kEW = Epi<KT>::kWarps;           // epilogue warps
+    constexpr int kHalves = kEW / 4;               // warps per TMEM lane quarter
+    constexpr int kChunksPerHalf = kBN / kChunk / kHalves;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+    uint32_t* cand = reinterpret_cast<uint32_t*>(smem + kStages * kStageBytes);  // [32][kBM] keys, then ids
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes + kCandBytes);
     uint64_t* empty_bar = full_bar + kStages;
     uint64_t* tfull_bar = empty_bar + kStages;
     uint64_t* tempty_bar = tfull_bar + 2;
@@ -157,7 +181,7 @@ __global__ void __launch_bounds__(pre::kThreads, 1) index_prefill_tc_kernel(
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tfull_bar[i], 1);
-            mbar_init(&tempty_bar[i], 4);  // one arrive per epilogue warp
+            mbar_init(&tempty_bar[i], kEW);  // one arrive per epilogue warp
         }
         fence_mbar_init();
     }
@@ -218,12 +242,17 @@ __global__ void __launch_bounds__(pre::kThreads, 1) index_prefill_tc_kernel(
             }
         }
     } else {
-        // ---------------- epilogue: one query row per thread ----------------
-        const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+        // ---------------- epilogue: one query row per thread and half ----------------
+        const int ew = warp - 2;                // 0 .. kEW-1
+        const int quarter = warp & 3;           // TMEM lanes 32*quarter .. +31
+        const int half = ew >> 2;               // which chunks of every tile
         const int r = quarter * 32 + lane;
         const int s = row0 + r;
         const long long p = (long long)q_start[b] + s;
         const int vis = s < S ? visible_blocks(p, ctx, bs, nb_max) : 0;
+        const int et = ew * 32 + lane;          // epilogue thread index
+        uint32_t* ckey = cand + et;             // [q * kMaxEpi + et]
+        int32_t* cid = reinterpret_cast<int32_t*>(cand) + kChunk * kMaxEpi + et;
         RowTopK<KT> top;
         top.init();
         for (int t = 0; t < my_tiles; ++t) {
@@ -232,38 +261,124 @@ __global__ void __launch_bounds__(pre::kThreads, 1) index_prefill_tc_kernel(
             tc_fence_after();
             const int n0 = (t_lo + t) * kBN;
             if (ok) {
+                const uint32_t lane_base =
+                    tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kBN);
+                uint32_t raw[kChunk], nxt[kChunk];
+                __syncwarp();
+                tmem_ld16_issue(lane_base + (uint32_t)(half * kChunk), raw);
+                tmem_ld16_wait(raw);
 #pragma unroll 1
-                for (int c = 0; c < kBN / 32; ++c) {
-                    float v[32];
-                    tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kBN + c * 32), v);
-                    const int jb = n0 + c * 32;
-                    if (jb >= vis) continue;
+                for (int c = 0; c < kChunksPerHalf; ++c) {
+                    const int col = (c * kHalves + half) * kChunk;  // halves interleave chunks
+                    // start the next chunk's load while this one is filtered
+                    __syncwarp();  // reconverge before the warp-collective TMEM load
+                    if (c + 1 < kChunksPerHalf)
+                        tmem_ld16_issue(lane_base + (uint32_t)(((c + 1) * kHalves + half) * kChunk), nxt);
+                    const int jb = n0 + col;
+                    if (jb < vis) {
+                        // Fast filter on the raw fp32 scores: the chunk's maximum
+                        // against the weakest kept score (an exact order test, as
+                        // scores are finite and -0.0 == +0.0).
+                        float f[kChunk];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const uint32_t key = score_key(v[i]);
-                        if (jb + i < vis && key > top.threshold()) top.insert(key, jb + i);
+                        for (int i = 0; i < kChunk; ++i) f[i] = __uint_as_float(raw[i]);
+                        if (jb + kChunk > vis) {  // the chunk crosses this row's causal edge
+#pragma unroll
+                            for (int i = 0; i < kChunk; ++i) f[i] = jb + i < vis ? f[i] : -INFINITY;
+                        }
+                        float fmx = f[0];
+#pragma unroll
+                        for (int i = 1; i < kChunk; ++i) fmx = fmaxf(fmx, f[i]);
+                        if (!top.full() || fmx > top.thr_f) {
+                            // branch-free compaction of the values that may enter
+                            const bool all = !top.full();
+                            const float thr = top.thr_f;
+                            int nc = 0;
+#pragma unroll
+                            for (int i = 0; i < kChunk; ++i) {
+                                ckey[nc * kMaxEpi] = raw[i];
+                                cid[nc * kMaxEpi] = jb + i;
+                                nc += (jb + i < vis) && (all || f[i] > thr);
+                            }
+                            // one copy of the insertion network, for the few that passed
+                            for (int q = 0; q < nc; ++q) {
+                                const uint32_t k = score_key(__uint_as_float(ckey[q * kMaxEpi]));
+                                if (k > top.threshold()) top.insert(k, cid[q * kMaxEpi]);
+                            }
+                        }
+                    }
+                    __syncwarp();
+                    if (c + 1 < kChunksPerHalf) {
+                        tmem_ld16_wait(nxt);
+#pragma unroll
+                        for (int i = 0; i < kChunk; ++i) raw[i] = nxt[i];
                     }
                 }
+                __syncwarp();
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty_bar[buf]);
         }
-        // ---------------- output ----------------
-        if (n_split == 1) {
-            if (s < S) {
-                int32_t* orow = ids + ((size_t)b * S + s) * topk;
-#pragma unroll
-                for (int i = 0; i < KT; ++i)
-                    if (i < topk) orow[i] = top.id[i];
-            }
-        } else {
-            const size_t prow = (((size_t)b * m_tiles + mt) * kBM + r) * n_split + ns;
+        // ---------------- combine the halves, write in rank order ----------------
+        // (the stage memory is idle: every MMA and copy has completed)
+        uint32_t* xk = reinterpret_cast<uint32_t*>(smem);
+        int32_t* xi = reinterpret_cast<int32_t*>(smem) + kBM * KT;
+        if (kHalves == 2 && half == 1) {
 #pragma unroll
             for (int i = 0; i < KT; ++i) {
-                if (i < topk) {
-                    part_key[prow * topk + i] = top.key[i];
-                    part_id[prow * topk + i] = top.id[i];
+                xk[i * kBM + r] = top.key[i];
+                xi[i * kBM + r] = top.id[i];
+            }
+        }
+        named_barrier_sync(1, 32 * kEW);
+        if (half == 0) {
+            uint32_t okey[KT];
+            int32_t oid[KT];
+            if (kHalves == 2) {
+                // merge two sorted lists; on equal keys the lower id first
+                int ia = 0, ib = 0;
+#pragma unroll
+                for (int i = 0; i < KT; ++i) {
+                    uint32_t ka = 0u, kb = 0u;
+                    int32_t da = -1, db = -1;
+#pragma unroll
+                    for (int q = 0; q < KT; ++q) {
+                        ka = q == ia ? top.key[q] : ka;
+                        da = q == ia ? top.id[q] : da;
+                    }
+                    kb = xk[min(ib, KT - 1) * kBM + r];
+                    db = xi[min(ib, KT - 1) * kBM + r];
+                    if (ib >= KT) kb = 0u, db = -1;
+                    if (ia >= KT) ka = 0u, da = -1;
+                    const bool take_a = da >= 0 && (db < 0 || ka > kb || (ka == kb && da < db));
+                    okey[i] = take_a ? ka : kb;
+                    oid[i] = take_a ? da : db;
+                    ia += take_a;
+                    ib += !take_a;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < KT; ++i) {
+                    okey[i] = top.key[i];
+                    oid[i] = top.id[i];
+                }
+            }
+            if (n_split == 1) {
+                if (s < S) {
+                    int32_t* orow = ids + ((size_t)b * S + s) * topk;
+#pragma unroll
+                    for (int i = 0; i < KT; ++i)
+                        if (i < topk) orow[i] = oid[i];
+                }
+            } else {
+                const size_t prow = (((size_t)b * m_tiles + mt) * kBM + r) * n_split + ns;
+#pragma unroll
+                for (int i = 0; i < KT; ++i) {
+                    if (i < topk) {
+                        part_key[prow * topk + i] = okey[i];
+                        part_id[prow * topk + i] = oid[i];
+                    }
                 }
             }
         }
@@ -302,7 +417,7 @@ __global__ void __launch_bounds__(pre::kThreads, 1) index_prefill_tc_kernel(
         mi[e] = __ldcg(part_id + base + e);
     }
     __syncthreads();
-    if (warp < 2) return;
+    if (warp < 2 || warp >= 6) return;  // one thread per row merges
     const int r = (warp & 3) * 32 + lane;
     const int s = row0 + r;
     if (s >= S) return;

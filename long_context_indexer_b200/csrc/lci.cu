@@ -290,7 +290,7 @@ lci_status launch_prefill_kt(const CUtensorMap& tq, const CUtensorMap& tk, int32
     if (attr_err != cudaSuccess)
         return fail(LCI_ERR_CUDA, "index_select: %s", cudaGetErrorString(attr_err));
     dim3 grid((unsigned)pl.n_split, (unsigned)pl.m_tiles, (unsigned)batch);
-    kern<<<grid, lci::pre::kThreads, lci::pre::kSmemBytes, st>>>(
+    kern<<<grid, lci::pre::Cfg<KT>::kThreads, lci::pre::kSmemBytes, st>>>(
         tq, tk, S, nb_max, bs, ctx_len, q_start, topk, pl.ksteps, pl.m_tiles, pl.n_split,
         reinterpret_cast<uint32_t*>(ws + pl.off_key), reinterpret_cast<int32_t*>(ws + pl.off_id),
         reinterpret_cast<unsigned int*>(ws + pl.off_counters), ids);
