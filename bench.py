@@ -357,6 +357,25 @@ def oracle_throughput(cfg, min_seconds=10.0, max_rows=None, w=None):
 
 # ------------------------------------------------------------------ main
 
+def shard_seed_offset(rank: int) -> int:
+    """Each rank draws its own batch of sequences (weak scaling, no exchange)."""
+    return 1000 * rank
+
+
+def reduce_max_ms(values, device, world: int):
+    """Max over ranks of each timing (ms); identity on one rank."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(world: int, rows_per_rank: int, steps: int, total_ms: float) -> float:
+    """Whole-job tokens/s: every rank's query rows over the slowest rank's time."""
+    return world * rows_per_rank * steps / (total_ms / 1e3)
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -415,19 +434,16 @@ def main():
     global SAMPLER
     with ClockSampler(local) as clk:
         SAMPLER = clk
-        res = measure(cfg, args.steps, args.warmup, device, rank, seed_offset=1000 * rank)
+        res = measure(cfg, args.steps, args.warmup, device, rank,
+                      seed_offset=shard_seed_offset(rank))
         SAMPLER = None
     torch.cuda.synchronize()
     lci.get_device_status()
-    total_ms = torch.tensor([res["t_total_ms"], res["e2e_total_ms"]], device=device,
-                            dtype=torch.float64)
     if world > 1:
         dist.barrier()
-        dist.all_reduce(total_ms, op=dist.ReduceOp.MAX)
-    t_total, e_total = total_ms.tolist()
-    tokens = world * cfg.B * cfg.S * args.steps
-    value = tokens / (t_total / 1e3)
-    e2e_value = tokens / (e_total / 1e3)
+    t_total, e_total = reduce_max_ms([res["t_total_ms"], res["e2e_total_ms"]], device, world)
+    value = job_throughput(world, cfg.B * cfg.S, args.steps, t_total)
+    e2e_value = job_throughput(world, cfg.B * cfg.S, args.steps, e_total)
 
     alg = res["alg"]
     kernels = {
