@@ -149,6 +149,8 @@ class Pipeline:
         na = lci.sparse_attn_workspace_size(cfg.B, cfg.S, cfg.H_q, cfg.topk, self.bt)
         self.ws_i = torch.zeros(max(ni, 256), dtype=torch.uint8, device=device)
         self.ws_a = torch.zeros(max(na, 256), dtype=torch.uint8, device=device)
+        nd = lci.sparse_decode_workspace_size(cfg.B, cfg.S, cfg.H_i, cfg.d_c, cfg.NB, cfg.topk)
+        self.ws_d = torch.zeros(max(nd, 256), dtype=torch.uint8, device=device)
         self.launches_per_step = (1 if cfg.compress else 0) + 2
 
     def clone(self):
@@ -162,6 +164,7 @@ class Pipeline:
         other.out = torch.empty_like(self.out)
         other.ws_i = torch.zeros_like(self.ws_i)
         other.ws_a = torch.zeros_like(self.ws_a)
+        other.ws_d = torch.zeros_like(self.ws_d)
         other.launches_per_step = self.launches_per_step
         return other
 
@@ -203,8 +206,16 @@ class Pipeline:
                              d["q_start"], out=self.out, ws=self.ws_a)
 
     def step(self):
-        self.index()
-        self.attn()
+        c = self.cfg
+        if c.S == 1 and not c.compress:
+            # one decode step in one call: rows are attended as they are selected
+            d = self.d
+            self.lci.sparse_decode(d["q_c"], self.k_c, d["ctx_len"], d["q_start"], c.topk, d["q"],
+                                   d["k_pool"], d["v_pool"], self.bt, ids=self.ids, out=self.out,
+                                   ws=self.ws_d)
+        else:
+            self.index()
+            self.attn()
 
     # Algorithmic work, from the shapes and the produced ids (outside timing):
     # every byte that must cross HBM at least once (unique k_c and KV blocks,

@@ -225,6 +225,36 @@ LCI_API lci_status lci_index_select_noalloc(const void* q_c, const void* k_c, lc
                                             void* stream);
 
 /*
+ * Workspace bytes lci_sparse_decode needs for these sizes.
+ */
+LCI_API lci_status lci_sparse_decode_workspace_size(int32_t batch, int32_t S, int32_t H_i,
+                                                    int32_t d_c, int32_t nb_max, int32_t topk,
+                                                    size_t* bytes);
+
+/*
+ * One decode step in one call: lci_index_select (one-row-at-a-time schedule)
+ * followed by lci_sparse_attn, with identical results, block ids included.
+ * [GPU-stack] "Separate Paths for Prefill and Decode" asks that decode overlap
+ * index selection with the cache reads; here the indexer publishes each query
+ * row as soon as its block ids are final, and the attention kernel, launched
+ * behind it (programmatic dependent launch), starts on a row as soon as that
+ * row is published, while later rows are still being scored.
+ * Arguments are those of the two calls; k_c's nb_max must equal the table's
+ * max_blocks and all floating inputs share one dtype. The workspace holds the
+ * indexer's scratch and per-row publication flags: zero-fill it before its
+ * first call and again before using it with other sizes; every call leaves it
+ * ready for the next. Calls sharing a workspace must not overlap in time.
+ */
+LCI_API lci_status lci_sparse_decode(const void* q_c, const void* k_c, lci_dtype dtype,
+                                     int32_t batch, int32_t S, int32_t H_i, int32_t d_c,
+                                     int32_t nb_max, const int32_t* d_ctx_len,
+                                     const int32_t* d_q_start, int32_t topk, const void* q,
+                                     int32_t H_q, const void* k_pool, const void* v_pool,
+                                     const lci_block_table* table, float scale, int32_t* d_ids,
+                                     void* out, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the sticky device status
  * word of the current device: LCI_OK, or LCI_ERR_DEVICE_BOUNDS when a device
  * bounds check fired since the last call.

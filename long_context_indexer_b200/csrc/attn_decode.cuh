@@ -60,7 +60,8 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
     const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ table, int nb_max,
     int num_pages, int H_kv, int bs, int S, int H_q, const int32_t* __restrict__ ids, int topk,
     const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ q_start, float scale_log2,
-    __nv_bfloat16* __restrict__ out, int nsplit) {
+    __nv_bfloat16* __restrict__ out, int nsplit, unsigned int* __restrict__ ready,
+    unsigned int* __restrict__ consumed) {
     using namespace dec;
     namespace cg = cooperative_groups;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -122,8 +123,29 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
         const int nlines = min(nb_max, 8192) / 32;  // 128-byte lines of the row
         for (int l = lane; l < nlines; l += 32) prefetch_l2(trow + l * 32);
     }
-    // Block ids come from the previous kernel on the stream.
-    pdl_wait();
+    // Block ids come from the previous kernel on the stream: either wait for
+    // that whole grid (programmatic dependent launch), or, when it publishes
+    // rows one by one, only for this row's ready flag (bounded wait).
+    if (ready == nullptr) {
+        pdl_wait();
+    } else {
+        if (tid == 0) {
+            const unsigned long long t0 = global_ns();
+            while (ld_acquire_gpu(ready + row) == 0u) {
+                if (global_ns() - t0 > kWaitLimitNs) {
+                    raise_status(kStatusTimeout);
+                    break;
+                }
+            }
+            // the last of the row's CTAs to pass resets the flag for the next call
+            const unsigned n = atomicAdd(consumed + row, 1u);
+            if (n == (unsigned)(H_kv * nsplit - 1)) {
+                consumed[row] = 0u;
+                ready[row] = 0u;
+            }
+        }
+        __syncthreads();
+    }
 
     float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
     float o[2][8][4];
@@ -145,7 +167,7 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
             int t0 = -1, y = 0;
             if (u < u1) {
                 const int i = u / tiles_per_block, sub = u - i * tiles_per_block;
-                const int j = row_ids[i];
+                const int j = __ldcg(row_ids + i);
                 if (j >= 0 && j < nb_max) {
                     const int page = table[(size_t)b * nb_max + j];
                     if (page < 0 || page >= num_pages) {

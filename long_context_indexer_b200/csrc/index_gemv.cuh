@@ -1,7 +1,7 @@
 // index_gemv.cuh -- block scoring fused with the causal-masked top-k, one query
 // row at a time (the decode schedule; also the generic path for any S).
 //
-// Grid (rows, chunks). Each CTA scores one chunk of the row's causal-visible
+// Grid rows x chunks (1-D, chunk fastest). Each CTA scores one chunk of the row's causal-visible
 // blocks: k_c rows stream from HBM with 16-byte loads, every warp dots them
 // against the query row staged in shared memory and reduces with shuffles. The
 // fp32 scores go to the workspace (L2-resident, 4 bytes per 2 KiB block key).
@@ -41,7 +41,7 @@ __global__ void __launch_bounds__(NT) index_gemv_select_kernel(
     const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ q_start, int topk,
     int chunk_blocks, int nchunks, float* __restrict__ scores,
     uint32_t* __restrict__ chunk_max, unsigned int* __restrict__ counters,
-    int32_t* __restrict__ ids) {
+    int32_t* __restrict__ ids, unsigned int* __restrict__ ready) {
     // Dynamic shared memory: [k_c chunk: chunk_blocks * K * sizeof(T)]
     // [query row: K floats, only when KV == 0]; the last CTA of a row reuses it
     // for the select's scratch.
@@ -55,7 +55,9 @@ __global__ void __launch_bounds__(NT) index_gemv_select_kernel(
     // Let the attention kernel that follows on the stream start its prologue;
     // it waits for this grid's results before reading the block ids.
     pdl_trigger();
-    const int row = blockIdx.x, chunk = blockIdx.y;
+    // chunk fastest: a row's CTAs are dispatched together, so rows complete (and
+    // are selected) one after another instead of all at the end
+    const int row = blockIdx.x / nchunks, chunk = blockIdx.x - row * nchunks;
     const int b = row / S, s = row - b * S;
     const long long p = (long long)__ldg(&q_start[b]) + s;
     const int vis = visible_blocks(p, __ldg(&ctx_len[b]), bs, nb_max);
@@ -135,6 +137,13 @@ __global__ void __launch_bounds__(NT) index_gemv_select_kernel(
     SelectSmem& sel = *reinterpret_cast<SelectSmem*>(dyn_smem);
     cta_topk_select<NT>(row_scores, chunk_max + (size_t)row * nchunks, vis, chunk_blocks, topk,
                         ids + (size_t)row * topk, sel);
+    if (ready != nullptr) {  // publish the row to a consumer running concurrently
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            st_release_gpu(ready + row, 1u);
+        }
+    }
 }
 
 }  // namespace lci

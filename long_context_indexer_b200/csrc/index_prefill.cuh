@@ -31,18 +31,19 @@ namespace lci {
 namespace pre {
 constexpr int kBM = 128, kBN = 256, kBK = 64;
 constexpr int kStages = 4;
-constexpr int kChunk = 16;               // TMEM columns per epilogue load
+constexpr int kChunk = 8;                // TMEM columns per epilogue load
 constexpr int kABytes = kBM * kBK * 2;   // 16 KiB
 constexpr int kBBytes = kBN * kBK * 2;   // 32 KiB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kTmemCols = 2 * kBN;       // two accumulators
-constexpr int kMaxEpi = 256;             // epilogue threads (8 warps)
+constexpr int kMaxEpi = 512;             // epilogue threads (16 warps)
 constexpr int kCandBytes = kChunk * kMaxEpi * 8;  // per epilogue thread: one chunk of (key, id)
 constexpr int kSmemBytes = kStages * kStageBytes + kCandBytes + 1024 /*align*/ + 256 /*barriers*/;
-// epilogue warps: 8 (two per TMEM lane quarter, each half of every tile's
-// columns) when the per-row list is short, 4 for KT = 64 (register budget)
-template <int KT> struct Epi { static constexpr int kWarps = KT <= 32 ? 8 : 4; };
-template <int KT> struct Cfg { static constexpr int kThreads = 64 + 32 * Epi<KT>::kWarps; };
+// Epilogue warps: kParts per TMEM lane quarter, each taking every kParts-th
+// chunk of every tile with its own list. More parts hide more latency; the
+// register budget (65536 / threads) bounds them by the list length KT.
+template <int KT> struct Epi { static constexpr int kParts = KT <= 32 ? 2 : 1; };
+template <int KT> struct Cfg { static constexpr int kThreads = 64 + 128 * Epi<KT>::kParts; };
 // instruction descriptor: D fp32, A/B bf16, both K-major, N = 256, M = 128
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
                             ((uint32_t)(kBM >> 4) << 24);
@@ -77,23 +78,15 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// Asynchronous 16-column TMEM load: tmem_ld16_issue starts it, tmem_ld16_wait
-// completes it. The wait names the destination registers as read-write
-// operands, so the compiler cannot use them before the data has landed.
-__device__ __forceinline__ void tmem_ld16_issue(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-        "%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_ld16_wait(uint32_t (&r)[16]) {
+// 8 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;"
                  : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
-                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
-                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                   "+r"(r[6]), "+r"(r[7])
                  :
                  : "memory");
 }
@@ -146,9 +139,9 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
     int32_t* __restrict__ ids) {
     using namespace pre;
     constexpr int kThreads = Cfg<KT>::kThreads;
-    constexpr int kEW = Epi<KT>::kWarps;           // epilogue warps
-    constexpr int kHalves = kEW / 4;               // warps per TMEM lane quarter
-    constexpr int kChunksPerHalf = kBN / kChunk / kHalves;
+    constexpr int kParts = Epi<KT>::kParts;        // epilogue warps per TMEM lane quarter
+    constexpr int kEW = 4 * kParts;                // epilogue warps
+    constexpr int kChunksPerPart = kBN / kChunk / kParts;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -242,10 +235,10 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
             }
         }
     } else {
-        // ---------------- epilogue: one query row per thread and half ----------------
+        // ---------------- epilogue: kParts threads per query row ----------------
         const int ew = warp - 2;                // 0 .. kEW-1
         const int quarter = warp & 3;           // TMEM lanes 32*quarter .. +31
-        const int half = ew >> 2;               // which chunks of every tile
+        const int part = ew >> 2;               // which chunks of every tile
         const int r = quarter * 32 + lane;
         const int s = row0 + r;
         const long long p = (long long)q_start[b] + s;
@@ -263,17 +256,12 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
             if (ok) {
                 const uint32_t lane_base =
                     tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kBN);
-                uint32_t raw[kChunk], nxt[kChunk];
-                __syncwarp();
-                tmem_ld16_issue(lane_base + (uint32_t)(half * kChunk), raw);
-                tmem_ld16_wait(raw);
 #pragma unroll 1
-                for (int c = 0; c < kChunksPerHalf; ++c) {
-                    const int col = (c * kHalves + half) * kChunk;  // halves interleave chunks
-                    // start the next chunk's load while this one is filtered
+                for (int c = 0; c < kChunksPerPart; ++c) {
+                    const int col = (c * kParts + part) * kChunk;  // parts interleave chunks
+                    uint32_t raw[kChunk];
                     __syncwarp();  // reconverge before the warp-collective TMEM load
-                    if (c + 1 < kChunksPerHalf)
-                        tmem_ld16_issue(lane_base + (uint32_t)(((c + 1) * kHalves + half) * kChunk), nxt);
+                    tmem_ld8(lane_base + (uint32_t)col, raw);
                     const int jb = n0 + col;
                     if (jb < vis) {
                         // Fast filter on the raw fp32 scores: the chunk's maximum
@@ -281,11 +269,8 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
                         // scores are finite and -0.0 == +0.0).
                         float f[kChunk];
 #pragma unroll
-                        for (int i = 0; i < kChunk; ++i) f[i] = __uint_as_float(raw[i]);
-                        if (jb + kChunk > vis) {  // the chunk crosses this row's causal edge
-#pragma unroll
-                            for (int i = 0; i < kChunk; ++i) f[i] = jb + i < vis ? f[i] : -INFINITY;
-                        }
+                        for (int i = 0; i < kChunk; ++i)
+                            f[i] = jb + i < vis ? __uint_as_float(raw[i]) : -INFINITY;
                         float fmx = f[0];
 #pragma unroll
                         for (int i = 1; i < kChunk; ++i) fmx = fmaxf(fmx, f[i]);
@@ -307,12 +292,6 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
                             }
                         }
                     }
-                    __syncwarp();
-                    if (c + 1 < kChunksPerHalf) {
-                        tmem_ld16_wait(nxt);
-#pragma unroll
-                        for (int i = 0; i < kChunk; ++i) raw[i] = nxt[i];
-                    }
                 }
                 __syncwarp();
             }
@@ -320,65 +299,44 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty_bar[buf]);
         }
-        // ---------------- combine the halves, write in rank order ----------------
+        // ---------------- merge the parts, write in rank order ----------------
         // (the stage memory is idle: every MMA and copy has completed)
-        uint32_t* xk = reinterpret_cast<uint32_t*>(smem);
-        int32_t* xi = reinterpret_cast<int32_t*>(smem) + kBM * KT;
-        if (kHalves == 2 && half == 1) {
+        uint32_t* xk = reinterpret_cast<uint32_t*>(smem);                  // [part][i][row]
+        int32_t* xi = reinterpret_cast<int32_t*>(smem) + kParts * KT * kBM;
 #pragma unroll
-            for (int i = 0; i < KT; ++i) {
-                xk[i * kBM + r] = top.key[i];
-                xi[i * kBM + r] = top.id[i];
-            }
+        for (int i = 0; i < KT; ++i) {
+            xk[(part * KT + i) * kBM + r] = top.key[i];
+            xi[(part * KT + i) * kBM + r] = top.id[i];
         }
         named_barrier_sync(1, 32 * kEW);
-        if (half == 0) {
-            uint32_t okey[KT];
-            int32_t oid[KT];
-            if (kHalves == 2) {
-                // merge two sorted lists; on equal keys the lower id first
-                int ia = 0, ib = 0;
+        if (part == 0) {
+            int head[kParts];
 #pragma unroll
-                for (int i = 0; i < KT; ++i) {
-                    uint32_t ka = 0u, kb = 0u;
-                    int32_t da = -1, db = -1;
+            for (int q = 0; q < kParts; ++q) head[q] = 0;
+            const size_t prow = (((size_t)b * m_tiles + mt) * kBM + r) * n_split + ns;
+            int32_t* orow = ids + ((size_t)b * S + s) * topk;
+            for (int i = 0; i < topk; ++i) {
+                // the best head: key desc, then id asc; empty entries (id -1) last
+                int best = 0;
+                uint32_t bk = 0u;
+                int32_t bi = -1;
 #pragma unroll
-                    for (int q = 0; q < KT; ++q) {
-                        ka = q == ia ? top.key[q] : ka;
-                        da = q == ia ? top.id[q] : da;
-                    }
-                    kb = xk[min(ib, KT - 1) * kBM + r];
-                    db = xi[min(ib, KT - 1) * kBM + r];
-                    if (ib >= KT) kb = 0u, db = -1;
-                    if (ia >= KT) ka = 0u, da = -1;
-                    const bool take_a = da >= 0 && (db < 0 || ka > kb || (ka == kb && da < db));
-                    okey[i] = take_a ? ka : kb;
-                    oid[i] = take_a ? da : db;
-                    ia += take_a;
-                    ib += !take_a;
+                for (int q = 0; q < kParts; ++q) {
+                    const int h = min(head[q], KT - 1);
+                    const uint32_t kq = head[q] < KT ? xk[(q * KT + h) * kBM + r] : 0u;
+                    const int32_t iq = head[q] < KT ? xi[(q * KT + h) * kBM + r] : -1;
+                    const bool better = iq >= 0 && (bi < 0 || kq > bk || (kq == bk && iq < bi));
+                    best = better ? q : best;
+                    bk = better ? kq : bk;
+                    bi = better ? iq : bi;
                 }
-            } else {
 #pragma unroll
-                for (int i = 0; i < KT; ++i) {
-                    okey[i] = top.key[i];
-                    oid[i] = top.id[i];
-                }
-            }
-            if (n_split == 1) {
-                if (s < S) {
-                    int32_t* orow = ids + ((size_t)b * S + s) * topk;
-#pragma unroll
-                    for (int i = 0; i < KT; ++i)
-                        if (i < topk) orow[i] = oid[i];
-                }
-            } else {
-                const size_t prow = (((size_t)b * m_tiles + mt) * kBM + r) * n_split + ns;
-#pragma unroll
-                for (int i = 0; i < KT; ++i) {
-                    if (i < topk) {
-                        part_key[prow * topk + i] = okey[i];
-                        part_id[prow * topk + i] = oid[i];
-                    }
+                for (int q = 0; q < kParts; ++q) head[q] += (q == best && bi >= 0);
+                if (n_split == 1) {
+                    if (s < S) orow[i] = bi;
+                } else {
+                    part_key[prow * topk + i] = bk;
+                    part_id[prow * topk + i] = bi;
                 }
             }
         }

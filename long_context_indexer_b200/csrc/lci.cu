@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -125,7 +126,7 @@ template <typename T>
 lci_status launch_index_gemv(const void* q_c, const void* k_c, int32_t batch, int32_t S, int32_t K,
                              int32_t bs, int32_t nb_max, const int32_t* ctx_len,
                              const int32_t* q_start, int32_t topk, int32_t* ids, void* ws,
-                             const IndexPlan& pl, cudaStream_t st) {
+                             const IndexPlan& pl, cudaStream_t st, unsigned int* ready = nullptr) {
     constexpr int KV = 2048 / (16 * 32);
     auto kern = pl.qreg ? lci::index_gemv_select_kernel<T, kIndexThreads, KV>
                         : lci::index_gemv_select_kernel<T, kIndexThreads, 0>;
@@ -146,12 +147,13 @@ lci_status launch_index_gemv(const void* q_c, const void* k_c, int32_t batch, in
     if (pl.smem > (size_t)kIndexMaxSmem)
         return fail(LCI_ERR_UNSUPPORTED, "index_select: needs %zu bytes of shared memory", pl.smem);
     char* w = static_cast<char*>(ws);
-    dim3 grid((unsigned)(batch * S), (unsigned)pl.nchunks);
-    kern<<<grid, kIndexThreads, pl.smem, st>>>(
+    const long long nblk = (long long)batch * S * pl.nchunks;
+    if (nblk >= (1ll << 31)) return fail(LCI_ERR_UNSUPPORTED, "index_select: grid too large");
+    kern<<<(unsigned)nblk, kIndexThreads, pl.smem, st>>>(
         static_cast<const T*>(q_c), static_cast<const T*>(k_c), S, K, nb_max, bs, ctx_len, q_start,
         topk, pl.chunk_blocks, pl.nchunks, reinterpret_cast<float*>(w + pl.off_scores),
         reinterpret_cast<uint32_t*>(w + pl.off_chunk_max),
-        reinterpret_cast<unsigned int*>(w + pl.off_counters), ids);
+        reinterpret_cast<unsigned int*>(w + pl.off_counters), ids, ready);
     return check_launch("index_select");
 }
 
@@ -258,7 +260,7 @@ bool prefill_path(lci_dtype dtype, lci_phase phase, int32_t S, int32_t K, int32_
     const lci_phase ph = resolve_phase(phase, S);
     const bool wants = phase == LCI_PHASE_PREFILL || (ph == LCI_PHASE_PREFILL && S >= 32);
     return wants && dtype == LCI_BF16 && K % lci::pre::kBK == 0 && topk <= 64 && aligned16(q_c) &&
-           aligned16(k_c);
+           aligned16(k_c);  // (null pointers count as aligned: size queries pass them)
 }
 
 lci_status encode_rows_map(CUtensorMap* map, const void* base, long long rows, int K, int box_rows) {
@@ -332,7 +334,8 @@ int decode_splits(long long pairs, int units) {
 lci_status launch_attn_decode(const void* q, int32_t batch, int32_t S, int32_t H_q,
                               const void* k_pool, const void* v_pool, const lci_block_table* t,
                               const int32_t* ids, int32_t topk, const int32_t* ctx_len,
-                              const int32_t* q_start, float scale, void* out, cudaStream_t st) {
+                              const int32_t* q_start, float scale, void* out, cudaStream_t st,
+                              unsigned int* ready = nullptr, unsigned int* consumed = nullptr) {
     const long long rows = (long long)t->num_pages * t->num_kv_heads * t->block_size;
     CUtensorMap tm_k, tm_v;
     lci_status s = encode_pool_map(&tm_k, k_pool, rows);
@@ -374,7 +377,7 @@ lci_status launch_attn_decode(const void* q, int32_t batch, int32_t S, int32_t H
     cudaError_t e = cudaLaunchKernelEx(
         &cfg, lci::sparse_attn_decode_kernel, tm_k, tm_v, static_cast<const __nv_bfloat16*>(q),
         t->d_table, t->max_blocks, t->num_pages, t->num_kv_heads, t->block_size, S, H_q, ids, topk,
-        ctx_len, q_start, scale_log2, static_cast<__nv_bfloat16*>(out), nsplit);
+        ctx_len, q_start, scale_log2, static_cast<__nv_bfloat16*>(out), nsplit, ready, consumed);
     if (e != cudaSuccess) return fail(LCI_ERR_CUDA, "sparse_attn: %s", cudaGetErrorString(e));
     return check_launch("sparse_attn");
 }
@@ -473,9 +476,11 @@ lci_status lci_index_select_workspace_size(int32_t batch, int32_t S, int32_t H_i
     lci_status st = check_index_args(batch, S, H_i, d_c, nb_max, topk, LCI_BF16);
     if (st != LCI_OK && st != LCI_ERR_UNSUPPORTED) return st;
     (void)phase;
-    const size_t g = plan_index(batch, S, H_i * d_c, nb_max, 2).bytes;
-    const size_t t = plan_prefill(batch, S, H_i * d_c, nb_max, topk).bytes;
-    *bytes = g > t ? g : t;  // enough for whichever schedule the call picks
+    // the schedule a bf16 call with these sizes takes (fp32 always runs row-wise)
+    const int K = H_i * d_c;
+    const bool tc = prefill_path(LCI_BF16, phase, S, K, topk, nullptr, nullptr);
+    const size_t g = plan_index(batch, S, K, nb_max, 2).bytes;
+    *bytes = tc ? std::max(g, plan_prefill(batch, S, K, nb_max, topk).bytes) : g;
     return ok();
 }
 
@@ -622,6 +627,90 @@ extern "C" lci_status lci_index_select_noalloc(const void* q_c, const void* k_c,
 }
 
 extern "C" {
+
+// ---- fused decode step ----
+
+struct DecodePlan {
+    IndexPlan ix;
+    size_t off_ready, off_consumed, bytes;
+};
+
+DecodePlan plan_decode(int32_t batch, int32_t S, int32_t K, int32_t nb_max) {
+    DecodePlan d{};
+    d.ix = plan_index(batch, S, K, nb_max, 2);
+    const size_t rows = (size_t)batch * S;
+    d.off_ready = align_up(d.ix.bytes);
+    d.off_consumed = d.off_ready + align_up(rows * sizeof(unsigned int));
+    d.bytes = d.off_consumed + align_up(rows * sizeof(unsigned int));
+    return d;
+}
+
+lci_status lci_sparse_decode_workspace_size(int32_t batch, int32_t S, int32_t H_i, int32_t d_c,
+                                            int32_t nb_max, int32_t topk, size_t* bytes) {
+    if (!bytes) return fail(LCI_ERR_INVALID_ARG, "sparse_decode_workspace_size: null output");
+    lci_status st = check_index_args(batch, S, H_i, d_c, nb_max, topk, LCI_BF16);
+    if (st != LCI_OK && st != LCI_ERR_UNSUPPORTED) return st;
+    *bytes = plan_decode(batch, S, H_i * d_c, nb_max).bytes;
+    return ok();
+}
+
+lci_status lci_sparse_decode(const void* q_c, const void* k_c, lci_dtype dtype, int32_t batch,
+                             int32_t S, int32_t H_i, int32_t d_c, int32_t nb_max,
+                             const int32_t* d_ctx_len, const int32_t* d_q_start, int32_t topk,
+                             const void* q, int32_t H_q, const void* k_pool, const void* v_pool,
+                             const lci_block_table* table, float scale, int32_t* d_ids, void* out,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+    if (!q_c || !k_c || !d_ctx_len || !d_q_start || !d_ids || !q || !k_pool || !v_pool || !out)
+        return fail(LCI_ERR_INVALID_ARG, "sparse_decode: null pointer argument");
+    lci_status st = check_index_args(batch, S, H_i, d_c, nb_max, topk, dtype);
+    if (st != LCI_OK) return st;
+    st = check_attn_args(batch, S, H_q, table, topk);
+    if (st != LCI_OK) return st;
+    if (table->max_blocks != nb_max)
+        return fail(LCI_ERR_INVALID_ARG, "sparse_decode: nb_max %d differs from the table's %d",
+                    nb_max, table->max_blocks);
+    if (dtype != table->dtype)
+        return fail(LCI_ERR_INVALID_ARG, "sparse_decode: q_c/k_c and the pools differ in dtype");
+    if (!aligned16(q_c) || !aligned16(k_c))
+        return fail(LCI_ERR_INVALID_ARG, "sparse_decode: q_c and k_c must be 16-byte aligned");
+    const int K = H_i * d_c;
+    const DecodePlan pl = plan_decode(batch, S, K, nb_max);
+    if (!workspace || workspace_bytes < pl.bytes ||
+        (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+        return fail(LCI_ERR_WORKSPACE, "sparse_decode: workspace needs %zu bytes, 256-byte aligned "
+                    "(got %zu at %p)", pl.bytes, workspace_bytes, workspace);
+    if (!(scale > 0.f)) scale = 1.0f / std::sqrt((float)table->head_dim);
+    if (!std::isfinite(scale)) return fail(LCI_ERR_INVALID_ARG, "sparse_decode: non-finite scale");
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    char* w = static_cast<char*>(workspace);
+    if (dtype == LCI_BF16 && decode_kernel_fits(table, H_q, k_pool, v_pool)) {
+        // rows are published one by one and attended as soon as they are ready
+        unsigned int* ready = reinterpret_cast<unsigned int*>(w + pl.off_ready);
+        unsigned int* consumed = reinterpret_cast<unsigned int*>(w + pl.off_consumed);
+        st = launch_index_gemv<__nv_bfloat16>(q_c, k_c, batch, S, K, table->block_size, nb_max,
+                                              d_ctx_len, d_q_start, topk, d_ids, workspace, pl.ix,
+                                              cs, ready);
+        if (st != LCI_OK) return st;
+        return launch_attn_decode(q, batch, S, H_q, k_pool, v_pool, table, d_ids, topk, d_ctx_len,
+                                  d_q_start, scale, out, cs, ready, consumed);
+    }
+    // other shapes: the two calls in sequence
+    st = dtype == LCI_F32
+             ? launch_index_gemv<float>(q_c, k_c, batch, S, K, table->block_size, nb_max, d_ctx_len,
+                                        d_q_start, topk, d_ids, workspace, pl.ix, cs)
+             : launch_index_gemv<__nv_bfloat16>(q_c, k_c, batch, S, K, table->block_size, nb_max,
+                                                d_ctx_len, d_q_start, topk, d_ids, workspace, pl.ix,
+                                                cs);
+    if (st != LCI_OK) return st;
+    if (table->dtype == LCI_F32)
+        return launch_attn_simt<float>(q, batch, S, H_q, k_pool, v_pool, table, d_ids, topk,
+                                       d_ctx_len, d_q_start, scale, out, cs);
+    if (decode_kernel_fits(table, H_q, k_pool, v_pool))
+        return launch_attn_decode(q, batch, S, H_q, k_pool, v_pool, table, d_ids, topk, d_ctx_len,
+                                  d_q_start, scale, out, cs);
+    return launch_attn_simt<__nv_bfloat16>(q, batch, S, H_q, k_pool, v_pool, table, d_ids, topk,
+                                           d_ctx_len, d_q_start, scale, out, cs);
+}
 
 lci_status lci_get_device_status(void* stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

@@ -47,6 +47,10 @@ SIGNATURES = {
     "lci_sparse_attn": (_st, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _f32,
                               _st, _vp, _vp, _sz, _vp]),
     "lci_get_device_status": (_st, [_vp]),
+    "lci_sparse_decode_workspace_size": (_st, [_i32, _i32, _i32, _i32, _i32, _i32,
+                                               ctypes.POINTER(_sz)]),
+    "lci_sparse_decode": (_st, [_vp, _vp, _st, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp,
+                                _i32, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _sz, _vp]),
     "lci_index_select_noalloc": (_st, [_vp, _vp, _st, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp,
                                        _i32, _st, _vp, _vp]),
 }
@@ -289,6 +293,48 @@ def sparse_attn(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, tab
         _dev(out, "out", q.dtype, 4), _dev(ws, "workspace"), ws.numel() * ws.element_size(),
         _stream(stream)), "lci_sparse_attn")
     return out
+
+
+def sparse_decode_workspace_size(B, S, H_i, d_c, nb_max, topk) -> int:
+    n = ctypes.c_size_t()
+    _check(load_library().lci_sparse_decode_workspace_size(B, S, H_i, d_c, nb_max, topk,
+                                                           ctypes.byref(n)),
+           "lci_sparse_decode_workspace_size")
+    return n.value
+
+
+def sparse_decode(q_c: torch.Tensor, k_c: torch.Tensor, ctx_len: torch.Tensor,
+                  q_start: torch.Tensor, topk: int, q: torch.Tensor, k_pool: torch.Tensor,
+                  v_pool: torch.Tensor, table: BlockTable, scale: float = 0.0,
+                  ids: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                  ws: Optional[torch.Tensor] = None, stream=None):
+    """index_select + sparse_attn in one call (rows attended as they are selected).
+
+    Returns (ids [B, S, topk] int32, out [B, S, H_q, hd])."""
+    B, S, H_i, d_c = q_c.shape
+    nb_max = k_c.shape[1]
+    H_q = q.shape[2]
+    if tuple(q.shape[:2]) != (B, S):
+        raise ValueError("lci: q must be [B, S, H_q, hd] with q_c's B and S")
+    if tuple(k_pool.shape) != (table.num_pages, table.num_kv_heads, table.block_size,
+                               table.head_dim) or v_pool.shape != k_pool.shape:
+        raise ValueError("lci: pools do not match the block table")
+    if ids is None:
+        ids = torch.empty((B, S, topk), dtype=torch.int32, device=q_c.device)
+    if out is None:
+        out = torch.empty_like(q)
+    need = sparse_decode_workspace_size(B, S, H_i, d_c, nb_max, topk)
+    if ws is None:
+        ws = workspace(q_c.device, need, f"sparse_decode:{B}x{S}x{nb_max}:{H_i * d_c}")
+    _check(load_library().lci_sparse_decode(
+        _dev(q_c, "q_c", None, 4), _dev(k_c, "k_c", q_c.dtype, 4), _dtype_code(q_c), B, S, H_i,
+        d_c, nb_max, _dev(ctx_len, "ctx_len", torch.int32, 1),
+        _dev(q_start, "q_start", torch.int32, 1), topk, _dev(q, "q", q_c.dtype, 4), H_q,
+        _dev(k_pool, "k_pool", q_c.dtype), _dev(v_pool, "v_pool", q_c.dtype), table.handle,
+        float(scale), _dev(ids, "ids", torch.int32, 3), _dev(out, "out", q_c.dtype, 4),
+        _dev(ws, "workspace"), ws.numel() * ws.element_size(), _stream(stream)),
+        "lci_sparse_decode")
+    return ids, out
 
 
 def get_device_status(stream=None) -> None:

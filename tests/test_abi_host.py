@@ -68,6 +68,9 @@ def test_index_select_host_checks(lib):
     need = binding.index_select_workspace_size(2, 1, 8, 128, 512, 32)
     assert need > 0
     assert _index_select(lib, ws=FAKE, ws_bytes=need - 1) == WORKSPACE
+    # a prefill-shaped call (tensor-core schedule) asks for its own, larger workspace
+    need_p = binding.index_select_workspace_size(2, 512, 8, 128, 512, 32, "prefill")
+    assert _index_select(lib, S=512, phase=1, ws=FAKE, ws_bytes=need_p - 1) == WORKSPACE
     assert _index_select(lib, ws=ctypes.c_void_p(0x7F0000000010), ws_bytes=need) == WORKSPACE
     assert b"workspace" in lib.lci_last_error()
 

@@ -233,3 +233,25 @@ def test_unwritten_cache_slots_never_reach_the_output(S, q0):
     ref_ids, ref_out = oracle_rows(cfg, w)
     assert torch.equal(ids.cpu().reshape(-1, cfg.topk), ref_ids)
     assert_out_close(out.reshape(-1, cfg.H_q, cfg.hd), ref_out, torch.bfloat16, "nan-tail")
+
+
+@pytest.mark.parametrize("name", ["decode", "small", "small_f32", "1m_decode"])
+def test_fused_decode_step_matches_two_calls_and_oracle(name):
+    """lci_sparse_decode (rows attended as soon as they are selected) gives the
+    block ids and outputs of index_select + sparse_attn, call after call."""
+    cfg = {"decode": CONFIGS["decode"], "1m_decode": CONFIGS["1m_decode"], "small": SMALL,
+           "small_f32": SMALL.replace(dtype="f32")}[name]
+    w = generate(cfg)
+    d = upload(w)
+    _, ids2, out2 = run_gpu(cfg, d)
+    bt = lci.create_block_table(d["block_table"], d["k_pool"])
+    for _ in range(3):  # the per-row flags must reset between calls
+        ids, out = lci.sparse_decode(d["q_c"], d["k_c"], d["ctx_len"], d["q_start"], cfg.topk,
+                                     d["q"], d["k_pool"], d["v_pool"], bt)
+        torch.cuda.synchronize()
+        lci.get_device_status()
+        assert torch.equal(ids, ids2)
+        assert torch.equal(out, out2)
+    ref_ids, ref_out = oracle_rows(cfg, w)
+    assert torch.equal(ids.cpu().reshape(-1, cfg.topk), ref_ids)
+    assert_out_close(out.reshape(-1, cfg.H_q, cfg.hd), ref_out, cfg.torch_dtype, name)
