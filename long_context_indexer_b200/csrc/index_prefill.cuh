@@ -91,6 +91,28 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
                  : "memory");
 }
 
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                   "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                   "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                   "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
 // Running top-KT of one row, sorted by key descending, in registers. Entries
 // start as (key 0, id -1), below every real key. A new element with a key equal
 // to an entry comes later in block order, so it ranks behind it: it enters
@@ -141,7 +163,8 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
     constexpr int kThreads = Cfg<KT>::kThreads;
     constexpr int kParts = Epi<KT>::kParts;        // epilogue warps per TMEM lane quarter
     constexpr int kEW = 4 * kParts;                // epilogue warps
-    constexpr int kChunksPerPart = kBN / kChunk / kParts;
+    constexpr int kGroup = 32;                    // TMEM columns per load
+    constexpr int kGroupsPerPart = kBN / kGroup / kParts;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -244,10 +267,29 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
         const long long p = (long long)q_start[b] + s;
         const int vis = s < S ? visible_blocks(p, ctx, bs, nb_max) : 0;
         const int et = ew * 32 + lane;          // epilogue thread index
-        uint32_t* ckey = cand + et;             // [q * kMaxEpi + et]
-        int32_t* cid = reinterpret_cast<int32_t*>(cand) + kChunk * kMaxEpi + et;
+        // Candidates that beat the threshold are appended, branch-free, to this
+        // thread's buffer (entry q at cbuf[q * kEpiThreads]); the insertion
+        // network runs only when some lane's buffer is about to fill. A warp
+        // then pays for the network once per buffered candidate of its busiest
+        // lane, instead of once per chunk in which any of its 32 rows passed.
+        constexpr int kEpiThreads = 32 * kEW;
+        constexpr int kBuf = kCandBytes / (8 * kEpiThreads);
+        static_assert(kBuf >= 2 * kChunk, "candidate buffer too small");
+        uint2* cbuf = reinterpret_cast<uint2*>(cand) + et;
+        int nc = 0;
         RowTopK<KT> top;
         top.init();
+        auto flush = [&]() {
+            const int m = __reduce_max_sync(0xffffffffu, nc);
+            for (int q = 0; q < m; ++q) {
+                if (q < nc) {
+                    const uint2 e = cbuf[q * kEpiThreads];
+                    const uint32_t k = score_key(__uint_as_float(e.x));
+                    if (k > top.threshold()) top.insert(k, (int32_t)e.y);
+                }
+            }
+            nc = 0;
+        };
         for (int t = 0; t < my_tiles; ++t) {
             const int buf = t & 1;
             const bool ok = mbar_wait(&tfull_bar[buf], (t >> 1) & 1);
@@ -257,40 +299,28 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
                 const uint32_t lane_base =
                     tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kBN);
 #pragma unroll 1
-                for (int c = 0; c < kChunksPerPart; ++c) {
-                    const int col = (c * kParts + part) * kChunk;  // parts interleave chunks
-                    uint32_t raw[kChunk];
+                for (int c = 0; c < kGroupsPerPart; ++c) {
+                    const int col = (c * kParts + part) * kGroup;  // parts interleave groups
+                    uint32_t raw[kGroup];
                     __syncwarp();  // reconverge before the warp-collective TMEM load
-                    tmem_ld8(lane_base + (uint32_t)col, raw);
-                    const int jb = n0 + col;
-                    if (jb < vis) {
-                        // Fast filter on the raw fp32 scores: the chunk's maximum
-                        // against the weakest kept score (an exact order test, as
-                        // scores are finite and -0.0 == +0.0).
-                        float f[kChunk];
+                    tmem_ld32(lane_base + (uint32_t)col, raw);
 #pragma unroll
-                        for (int i = 0; i < kChunk; ++i)
-                            f[i] = jb + i < vis ? __uint_as_float(raw[i]) : -INFINITY;
-                        float fmx = f[0];
-#pragma unroll
-                        for (int i = 1; i < kChunk; ++i) fmx = fmaxf(fmx, f[i]);
-                        if (!top.full() || fmx > top.thr_f) {
-                            // branch-free compaction of the values that may enter
-                            const bool all = !top.full();
-                            const float thr = top.thr_f;
-                            int nc = 0;
+                    for (int sc = 0; sc < kGroup / kChunk; ++sc) {
+                        const int jb = n0 + col + sc * kChunk;
+                        if (jb < vis) {
+                            // exact order test on the raw fp32 scores (finite, and
+                            // -0.0 == +0.0); equal scores come later in block order
+                            // and so never enter a full list
+                            const float thr = top.full() ? top.thr_f : -INFINITY;
 #pragma unroll
                             for (int i = 0; i < kChunk; ++i) {
-                                ckey[nc * kMaxEpi] = raw[i];
-                                cid[nc * kMaxEpi] = jb + i;
-                                nc += (jb + i < vis) && (all || f[i] > thr);
-                            }
-                            // one copy of the insertion network, for the few that passed
-                            for (int q = 0; q < nc; ++q) {
-                                const uint32_t k = score_key(__uint_as_float(ckey[q * kMaxEpi]));
-                                if (k > top.threshold()) top.insert(k, cid[q * kMaxEpi]);
+                                const uint32_t v = raw[sc * kChunk + i];
+                                cbuf[nc * kEpiThreads] = make_uint2(v, (uint32_t)(jb + i));
+                                nc += (jb + i < vis) && __uint_as_float(v) > thr;
                             }
                         }
+                        __syncwarp();
+                        if (__any_sync(0xffffffffu, nc > kBuf - kChunk)) flush();
                     }
                 }
                 __syncwarp();
@@ -299,6 +329,7 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty_bar[buf]);
         }
+        flush();
         // ---------------- merge the parts, write in rank order ----------------
         // (the stage memory is idle: every MMA and copy has completed)
         uint32_t* xk = reinterpret_cast<uint32_t*>(smem);                  // [part][i][row]
