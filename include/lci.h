@@ -144,12 +144,13 @@ LCI_API lci_status lci_index_select_workspace_size(int32_t batch, int32_t S, int
  *   d_ctx_len  [batch] int32, d_q_start [batch] int32, device
  *   d_ids      [batch][S][topk] int32, device (output)
  *   workspace  >= lci_index_select_workspace_size bytes, 256-byte aligned.
- *              It holds arrival counters whose position depends on the sizes
- *              (batch, S, nb_max). Zero-fill a workspace before its first call;
- *              every call leaves its counters at zero again, so later calls
- *              with the same sizes need no clearing. Zero it again before using
- *              it with other sizes. Calls that share a workspace must not
- *              overlap in time.
+ *              It holds arrival counters and per-row selection bounds whose
+ *              position depends on the sizes (batch, S, nb_max). Zero-fill a
+ *              workspace before its first call; every successful call leaves
+ *              them at zero again, so later calls with the same sizes need no
+ *              clearing. Zero it again before using it with other sizes, and
+ *              after a call that failed on the device. Calls that share a
+ *              workspace must not overlap in time.
  * Scores are accumulated in fp32. Limits: 1 <= topk <= 256,
  * nb_max <= 16384, H_i*d_c <= 8192 and a multiple of 8 (bf16) or 4 (f32).
  */

@@ -17,6 +17,12 @@
 //               ([GPU-stack] "Operatorizing Index Selection": scoring, top-k
 //               and masking fused in one pass).
 //
+// Every list (a row's part inside one CTA) publishes its k-th best key to a
+// per-row bound in the workspace (atomicMax) and filters against the best bound
+// any list of the row has published: a list's k-th best is a lower bound on the
+// row's final k-th best, so a score below the bound cannot be selected. The
+// split lists of one row then filter almost as sharply as a single list would.
+//
 // n-tiles beyond the last visible block of the m-tile are skipped. When an
 // m-tile's n-tiles are split over several CTAs, each writes its per-row
 // candidates (key, id) to the workspace and the last CTA to arrive (atomic
@@ -36,8 +42,7 @@ constexpr int kABytes = kBM * kBK * 2;   // 16 KiB
 constexpr int kBBytes = kBN * kBK * 2;   // 32 KiB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kTmemCols = 2 * kBN;       // two accumulators
-constexpr int kMaxEpi = 512;             // epilogue threads (16 warps)
-constexpr int kCandBytes = kChunk * kMaxEpi * 8;  // per epilogue thread: one chunk of (key, id)
+constexpr int kCandBytes = 32 * 1024;            // per-thread candidate buffers (score, id)
 constexpr int kSmemBytes = kStages * kStageBytes + kCandBytes + 1024 /*align*/ + 256 /*barriers*/;
 // Epilogue warps: kParts per TMEM lane quarter, each taking every kParts-th
 // chunk of every tile with its own list. More parts hide more latency; the
@@ -135,22 +140,35 @@ struct RowTopK {
     __device__ __forceinline__ uint32_t threshold() const { return key[KT - 1]; }
     __device__ __forceinline__ bool full() const { return id[KT - 1] >= 0; }
     __device__ __forceinline__ void insert(uint32_t k, int32_t j) {
+        // c[i]: the new key beats entry i. Keys move with unsigned min/max
+        // (the list is sorted), ids follow the same decisions.
+        bool c[KT];
+#pragma unroll
+        for (int i = 0; i < KT; ++i) c[i] = k > key[i];
 #pragma unroll
         for (int i = KT - 1; i > 0; --i) {
-            const bool take_prev = k > key[i - 1];
-            const bool here = !take_prev && k > key[i];
-            key[i] = take_prev ? key[i - 1] : (here ? k : key[i]);
-            id[i] = take_prev ? id[i - 1] : (here ? j : id[i]);
+            id[i] = c[i - 1] ? id[i - 1] : (c[i] ? j : id[i]);
+            key[i] = min(key[i - 1], max(k, key[i]));
         }
-        if (k > key[0]) {
-            key[0] = k;
-            id[0] = j;
-        }
+        id[0] = c[0] ? j : id[0];
+        key[0] = max(k, key[0]);
         // back from key to score: the inverse of score_key
         const uint32_t w = key[KT - 1];
         thr_f = __uint_as_float((w & 0x80000000u) ? (w & 0x7fffffffu) : ~w);
     }
 };
+
+// The score of a nonzero key (the inverse of score_key).
+__device__ __forceinline__ float key_score(uint32_t w) {
+    return __uint_as_float((w & 0x80000000u) ? (w & 0x7fffffffu) : ~w);
+}
+// The largest float below a finite x: "s > below(x)" is "s >= x" for finite s
+// (with -0.0 == +0.0).
+__device__ __forceinline__ float float_below(float x) {
+    if (x == 0.f) return __uint_as_float(0x80000001u);
+    const uint32_t u = __float_as_uint(x);
+    return __uint_as_float(x > 0.f ? u - 1u : u + 1u);
+}
 
 template <int KT>
 __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_kernel(
@@ -158,7 +176,7 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
     int nb_max, int bs, const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ q_start,
     int topk, int ksteps, int m_tiles, int n_split, uint32_t* __restrict__ part_key,
     int32_t* __restrict__ part_id, unsigned int* __restrict__ counters,
-    int32_t* __restrict__ ids) {
+    unsigned int* __restrict__ row_bound, int32_t* __restrict__ ids) {
     using namespace pre;
     constexpr int kThreads = Cfg<KT>::kThreads;
     constexpr int kParts = Epi<KT>::kParts;        // epilogue warps per TMEM lane quarter
@@ -267,7 +285,7 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
         const long long p = (long long)q_start[b] + s;
         const int vis = s < S ? visible_blocks(p, ctx, bs, nb_max) : 0;
         const int et = ew * 32 + lane;          // epilogue thread index
-        // Candidates that beat the threshold are appended, branch-free, to this
+        // Candidates that beat the threshold are appended to this
         // thread's buffer (entry q at cbuf[q * kEpiThreads]); the insertion
         // network runs only when some lane's buffer is about to fill. A warp
         // then pays for the network once per buffered candidate of its busiest
@@ -279,6 +297,11 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
         int nc = 0;
         RowTopK<KT> top;
         top.init();
+        // the row's shared bound: gk is the best key seen (own or published),
+        // gthr the float filter it implies (-inf while there is none)
+        unsigned int* bound = s < S ? row_bound + (size_t)b * S + s : nullptr;
+        uint32_t gk = 0u;
+        float gthr = -INFINITY;
         auto flush = [&]() {
             const int m = __reduce_max_sync(0xffffffffu, nc);
             for (int q = 0; q < m; ++q) {
@@ -289,6 +312,11 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
                 }
             }
             nc = 0;
+            if (top.full() && top.threshold() > gk && bound != nullptr) {
+                gk = top.threshold();
+                gthr = float_below(key_score(gk));
+                atomicMax(bound, gk);
+            }
         };
         for (int t = 0; t < my_tiles; ++t) {
             const int buf = t & 1;
@@ -301,6 +329,8 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
 #pragma unroll 1
                 for (int c = 0; c < kGroupsPerPart; ++c) {
                     const int col = (c * kParts + part) * kGroup;  // parts interleave groups
+                    // the row's bound as published so far, used from the next group on
+                    const uint32_t gk_next = bound != nullptr ? ld_relaxed_gpu(bound) : 0u;
                     uint32_t raw[kGroup];
                     __syncwarp();  // reconverge before the warp-collective TMEM load
                     tmem_ld32(lane_base + (uint32_t)col, raw);
@@ -311,16 +341,25 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
                             // exact order test on the raw fp32 scores (finite, and
                             // -0.0 == +0.0); equal scores come later in block order
                             // and so never enter a full list
-                            const float thr = top.full() ? top.thr_f : -INFINITY;
+                            const float thr = fmaxf(top.full() ? top.thr_f : -INFINITY, gthr);
 #pragma unroll
                             for (int i = 0; i < kChunk; ++i) {
+                                // a store only for a passing score: shared-memory
+                                // bandwidth is shared with the TMA writes and the
+                                // MMA operand reads
                                 const uint32_t v = raw[sc * kChunk + i];
-                                cbuf[nc * kEpiThreads] = make_uint2(v, (uint32_t)(jb + i));
-                                nc += (jb + i < vis) && __uint_as_float(v) > thr;
+                                if ((jb + i < vis) && __uint_as_float(v) > thr) {
+                                    cbuf[nc * kEpiThreads] = make_uint2(v, (uint32_t)(jb + i));
+                                    ++nc;
+                                }
                             }
                         }
                         __syncwarp();
                         if (__any_sync(0xffffffffu, nc > kBuf - kChunk)) flush();
+                    }
+                    if (gk_next > gk) {
+                        gk = gk_next;
+                        gthr = float_below(key_score(gk));
                     }
                 }
                 __syncwarp();
@@ -340,6 +379,9 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
             xi[(part * KT + i) * kBM + r] = top.id[i];
         }
         named_barrier_sync(1, 32 * kEW);
+        // every list of the row is final: with one CTA per row range the bound
+        // is reset here, otherwise by the CTA that merges the splits
+        if (n_split == 1 && part == 0 && bound != nullptr) *bound = 0u;
         if (part == 0) {
             int head[kParts];
 #pragma unroll
@@ -416,6 +458,7 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
     int head[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) head[q] = 0;
+    row_bound[(size_t)b * S + s] = 0u;  // every CTA of the m-tile has finished with it
     int32_t* orow = ids + ((size_t)b * S + s) * topk;
     for (int i = 0; i < topk; ++i) {
         int best = -1;

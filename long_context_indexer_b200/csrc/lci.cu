@@ -230,7 +230,7 @@ lci_status encode_pool_map(CUtensorMap* map, const void* pool, long long rows) {
 // Tensor-core schedule for many queries per sequence (index_prefill.cuh).
 struct PrefillPlan {
     int m_tiles, n_split, kt, ksteps;
-    size_t off_counters, off_key, off_id, bytes;
+    size_t off_counters, off_key, off_id, off_bound, bytes;
 };
 
 PrefillPlan plan_prefill(int32_t batch, int32_t S, int32_t K, int32_t nb_max, int32_t topk) {
@@ -240,18 +240,21 @@ PrefillPlan plan_prefill(int32_t batch, int32_t S, int32_t K, int32_t nb_max, in
     pl.kt = topk <= 16 ? 16 : (topk <= 32 ? 32 : 64);
     const int n_tiles = (nb_max + lci::pre::kBN - 1) / lci::pre::kBN;
     // about one CTA per SM; the merge copies n_split * topk candidates per row
-    // of a 128-row tile into the 192 KiB of stage memory
+    // of a 128-row tile into the stage memory
     long long split = 148 / ((long long)batch * pl.m_tiles);
     split = split < 1 ? 1 : split;
     split = split > 8 ? 8 : split;
     split = split > n_tiles ? n_tiles : split;
-    while (split > 1 && (long long)lci::pre::kBM * split * topk * 8 > 4 * lci::pre::kStageBytes) --split;
+    while (split > 1 &&
+           (long long)lci::pre::kBM * split * topk * 8 > (long long)lci::pre::kStages * lci::pre::kStageBytes)
+        --split;
     pl.n_split = (int)split;
     const long long cand = (long long)batch * pl.m_tiles * lci::pre::kBM * pl.n_split * topk;
     pl.off_counters = 0;
     pl.off_key = align_up((size_t)batch * pl.m_tiles * sizeof(unsigned int));
     pl.off_id = pl.off_key + align_up((size_t)cand * sizeof(uint32_t));
-    pl.bytes = pl.off_id + align_up((size_t)cand * sizeof(int32_t));
+    pl.off_bound = pl.off_id + align_up((size_t)cand * sizeof(int32_t));
+    pl.bytes = pl.off_bound + align_up((size_t)batch * S * sizeof(unsigned int));
     return pl;
 }
 
@@ -295,7 +298,8 @@ lci_status launch_prefill_kt(const CUtensorMap& tq, const CUtensorMap& tk, int32
     kern<<<grid, lci::pre::Cfg<KT>::kThreads, lci::pre::kSmemBytes, st>>>(
         tq, tk, S, nb_max, bs, ctx_len, q_start, topk, pl.ksteps, pl.m_tiles, pl.n_split,
         reinterpret_cast<uint32_t*>(ws + pl.off_key), reinterpret_cast<int32_t*>(ws + pl.off_id),
-        reinterpret_cast<unsigned int*>(ws + pl.off_counters), ids);
+        reinterpret_cast<unsigned int*>(ws + pl.off_counters),
+        reinterpret_cast<unsigned int*>(ws + pl.off_bound), ids);
     return check_launch("index_select");
 }
 
