@@ -36,7 +36,10 @@ namespace lci {
 namespace dec {
 constexpr int kHD = 128;           // head dim
 constexpr int kTile = 64;          // tokens per unit
-constexpr int kStages = 3;         // shared-memory ring depth
+// shared-memory ring depth: 3 stages let two CTAs share an SM; 6 stages fill
+// one SM when the grid has about one CTA per SM
+constexpr int kStagesShallow = 3;
+constexpr int kStagesDeep = 6;
 constexpr int kConsumers = 4;      // consumer warps, 16 tokens each
 constexpr int kThreads = (kConsumers + 1) * 32;
 constexpr int kBox = 64 * 64 * 2;  // one 64x64 bf16 box = 8 KiB
@@ -44,7 +47,7 @@ constexpr int kStageBytes = 4 * kBox;  // K: 2 boxes, V: 2 boxes
 constexpr int kMaxSplit = 8;
 constexpr int kRows = 16;          // query heads per MMA (padded)
 // shared memory: stages, then barriers and metadata
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256;
+constexpr int smem_bytes(int stages) { return stages * kStageBytes + 1024 /*align*/ + 256; }
 }  // namespace dec
 
 __device__ __forceinline__ int tok_perm(int x) { return x ^ ((x & 1) << 2); }
@@ -55,6 +58,7 @@ __device__ __forceinline__ uint32_t tile_off(int r, int c) {
     return (uint32_t)((c >> 3) * dec::kBox + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
+template <int kStages>
 __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ table, int nb_max,

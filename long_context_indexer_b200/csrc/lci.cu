@@ -328,11 +328,32 @@ bool decode_kernel_fits(const lci_block_table* t, int32_t H_q, const void* k_poo
            G <= lci::dec::kRows && aligned16(k_pool) && aligned16(v_pool) && rows < (1ll << 31);
 }
 
-int decode_splits(long long pairs, int units) {
+struct DecodeShape {
+    int nsplit;  // CTAs (one cluster) per (row, KV head) pair
+    bool deep;   // one CTA per SM with the deep ring
+};
+
+DecodeShape decode_shape(long long pairs, int units) {
+    // When the pairs fill the SMs with clusters of 2-4 CTAs, give each SM one
+    // CTA with a deep ring; otherwise two shallow CTAs per SM and up to 8 splits.
+    const long long per_sm = 148 / pairs;
+    if (per_sm >= 2 && per_sm <= 4 && units >= 2 * per_sm) return {(int)per_sm, true};
     long long want = (2 * 148 + pairs - 1) / pairs;
     if (want > lci::dec::kMaxSplit) want = lci::dec::kMaxSplit;
     if (want > units) want = units;
-    return want < 1 ? 1 : (int)want;
+    return {want < 1 ? 1 : (int)want, false};
+}
+
+template <int ST>
+cudaError_t decode_kernel_attr() {
+    static std::once_flag once;
+    static cudaError_t err = cudaSuccess;
+    std::call_once(once, [] {
+        err = cudaFuncSetAttribute(lci::sparse_attn_decode_kernel<ST>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   lci::dec::smem_bytes(ST));
+    });
+    return err;
 }
 
 lci_status launch_attn_decode(const void* q, int32_t batch, int32_t S, int32_t H_q,
@@ -346,22 +367,19 @@ lci_status launch_attn_decode(const void* q, int32_t batch, int32_t S, int32_t H
     if (s != LCI_OK) return s;
     s = encode_pool_map(&tm_v, v_pool, rows);
     if (s != LCI_OK) return s;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(lci::sparse_attn_decode_kernel,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        lci::dec::kSmemBytes);
-    });
-    if (attr_err != cudaSuccess)
-        return fail(LCI_ERR_CUDA, "sparse_attn: %s", cudaGetErrorString(attr_err));
     const long long pairs = (long long)batch * S * t->num_kv_heads;
     const int units = topk * (t->block_size / 64);
-    const int nsplit = decode_splits(pairs, units);
+    const DecodeShape shape = decode_shape(pairs, units);
+    const int nsplit = shape.nsplit;
+    const int stages = shape.deep ? lci::dec::kStagesDeep : lci::dec::kStagesShallow;
+    const cudaError_t attr_err =
+        shape.deep ? decode_kernel_attr<lci::dec::kStagesDeep>() : decode_kernel_attr<lci::dec::kStagesShallow>();
+    if (attr_err != cudaSuccess)
+        return fail(LCI_ERR_CUDA, "sparse_attn: %s", cudaGetErrorString(attr_err));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)pairs, (unsigned)nsplit, 1);
     cfg.blockDim = dim3(lci::dec::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = lci::dec::kSmemBytes;
+    cfg.dynamicSmemBytes = lci::dec::smem_bytes(stages);
     cfg.stream = st;
     cudaLaunchAttribute attrs[2];
     int na = 0;
@@ -378,8 +396,10 @@ lci_status launch_attn_decode(const void* q, int32_t batch, int32_t S, int32_t H
     cfg.attrs = attrs;
     cfg.numAttrs = na;
     const float scale_log2 = scale * 1.4426950408889634f;
+    auto kern = shape.deep ? lci::sparse_attn_decode_kernel<lci::dec::kStagesDeep>
+                           : lci::sparse_attn_decode_kernel<lci::dec::kStagesShallow>;
     cudaError_t e = cudaLaunchKernelEx(
-        &cfg, lci::sparse_attn_decode_kernel, tm_k, tm_v, static_cast<const __nv_bfloat16*>(q),
+        &cfg, kern, tm_k, tm_v, static_cast<const __nv_bfloat16*>(q),
         t->d_table, t->max_blocks, t->num_pages, t->num_kv_heads, t->block_size, S, H_q, ids, topk,
         ctx_len, q_start, scale_log2, static_cast<__nv_bfloat16*>(out), nsplit, ready, consumed);
     if (e != cudaSuccess) return fail(LCI_ERR_CUDA, "sparse_attn: %s", cudaGetErrorString(e));
