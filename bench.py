@@ -70,9 +70,9 @@ def peaks():
 # sources the capture ran. Once those sources change the figure no longer
 # describes the kernel and the bench reports traffic as null.
 PROFILED_TRAFFIC = {
-    ("decode", "index_select"): (33683200, "1ed4df7aace2fb2e"),
-    ("decode", "sparse_attn"): (33802752, "1ed4df7aace2fb2e"),
-    ("1m_chunk", "index_select"): (25203456, "1ed4df7aace2fb2e"),
+    ("decode", "index_select"): (33683200, "c6c94016afb2eca9"),
+    ("decode", "sparse_attn"): (33798400, "c6c94016afb2eca9"),
+    ("1m_chunk", "index_select"): (25226496, "c6c94016afb2eca9"),
 }
 
 
