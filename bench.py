@@ -24,6 +24,7 @@ import datetime
 import glob
 import hashlib
 import json
+import re
 import math
 import os
 import statistics
@@ -70,22 +71,30 @@ def peaks():
 # sources the capture ran. Once those sources change the figure no longer
 # describes the kernel and the bench reports traffic as null.
 PROFILED_TRAFFIC = {
-    ("decode", "index_select"): (33683200, "c6c94016afb2eca9"),
-    ("decode", "sparse_attn"): (33798400, "c6c94016afb2eca9"),
-    ("1m_chunk", "index_select"): (25226496, "c6c94016afb2eca9"),
+    ("decode", "index_select"): (33683200, "c2e06c74883d2e86"),
+    ("decode", "sparse_attn"): (33798400, "c2e06c74883d2e86"),
+    ("1m_chunk", "index_select"): (25226496, "c2e06c74883d2e86"),
 }
 
 
+def _code_only(text: str) -> str:
+    """C/CUDA source with comments removed and whitespace collapsed."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def sources_digest() -> str:
-    """sha256 (first 16 hex digits) over the CUDA sources and the C header."""
+    """sha256 (first 16 hex digits) over the code of the CUDA sources and the C
+    header, comments and whitespace excluded."""
     files = sorted(glob.glob(os.path.join(ROOT, "long_context_indexer_b200", "csrc", "*.cu")) +
                    glob.glob(os.path.join(ROOT, "long_context_indexer_b200", "csrc", "*.cuh")) +
                    [os.path.join(ROOT, "include", "lci.h")])
     h = hashlib.sha256()
     for f in files:
         h.update(os.path.basename(f).encode())
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        with open(f, encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

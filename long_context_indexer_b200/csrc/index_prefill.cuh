@@ -10,18 +10,22 @@
 //   warp 1      one thread issues tcgen05.mma (M=128, N=256, K=16, bf16 ->
 //               fp32) into one of two TMEM accumulators (2 x 256 columns) and
 //               commits stage releases / accumulator-ready signals;
-//   warps 2..5  epilogue: thread r owns query row r (TMEM lane r). It reads
-//               its 256 scores with tcgen05.ld, drops blocks that are not
-//               causal-visible, and keeps a running exact top-k in registers
-//               behind a threshold test. Scores never reach global memory
-//               ([GPU-stack] "Operatorizing Index Selection": scoring, top-k
-//               and masking fused in one pass).
+//   warps 2..   epilogue (4 warps, or 8 for k <= 32): a thread owns one query
+//               row (TMEM lane) and, with two warps per lane quarter, every
+//               other 32-column group of each tile. It reads 32 scores per
+//               tcgen05.ld, drops blocks that are not causal-visible, appends
+//               the scores above its threshold to a shared-memory buffer, and
+//               inserts the buffer into a running exact top-k in registers
+//               when some lane's buffer nears full. Scores never reach global
+//               memory ([GPU-stack] "Operatorizing Index Selection": scoring,
+//               top-k and masking fused in one pass).
 //
 // Every list (a row's part inside one CTA) publishes its k-th best key to a
 // per-row bound in the workspace (atomicMax) and filters against the best bound
 // any list of the row has published: a list's k-th best is a lower bound on the
-// row's final k-th best, so a score below the bound cannot be selected. The
-// split lists of one row then filter almost as sharply as a single list would.
+// row's final k-th best, so a score below the bound cannot be selected. As the
+// lists of a row grow at the same time, the bound runs only a little ahead of
+// each list's own threshold.
 //
 // n-tiles beyond the last visible block of the m-tile are skipped. When an
 // m-tile's n-tiles are split over several CTAs, each writes its per-row
@@ -37,7 +41,7 @@ namespace lci {
 namespace pre {
 constexpr int kBM = 128, kBN = 256, kBK = 64;
 constexpr int kStages = 4;
-constexpr int kChunk = 8;                // TMEM columns per epilogue load
+constexpr int kChunk = 8;                // columns between checks of the candidate buffers
 constexpr int kABytes = kBM * kBK * 2;   // 16 KiB
 constexpr int kBBytes = kBN * kBK * 2;   // 32 KiB
 constexpr int kStageBytes = kABytes + kBBytes;
@@ -45,8 +49,9 @@ constexpr int kTmemCols = 2 * kBN;       // two accumulators
 constexpr int kCandBytes = 32 * 1024;            // per-thread candidate buffers (score, id)
 constexpr int kSmemBytes = kStages * kStageBytes + kCandBytes + 1024 /*align*/ + 256 /*barriers*/;
 // Epilogue warps: kParts per TMEM lane quarter, each taking every kParts-th
-// chunk of every tile with its own list. More parts hide more latency; the
-// register budget (65536 / threads) bounds them by the list length KT.
+// 32-column group of every tile with its own list. More parts hide more
+// latency; the register budget (65536 / threads) bounds them by the list
+// length KT.
 template <int KT> struct Epi { static constexpr int kParts = KT <= 32 ? 2 : 1; };
 template <int KT> struct Cfg { static constexpr int kThreads = 64 + 128 * Epi<KT>::kParts; };
 // instruction descriptor: D fp32, A/B bf16, both K-major, N = 256, M = 128
