@@ -255,3 +255,36 @@ def test_fused_decode_step_matches_two_calls_and_oracle(name):
     ref_ids, ref_out = oracle_rows(cfg, w)
     assert torch.equal(ids.cpu().reshape(-1, cfg.topk), ref_ids)
     assert_out_close(out.reshape(-1, cfg.H_q, cfg.hd), ref_out, cfg.torch_dtype, name)
+
+
+@pytest.mark.parametrize("topk", [48, 64])
+def test_prefill_tensor_core_long_lists_split_tiles(topk):
+    """The tensor-core indexer with lists longer than 32 (one epilogue warp per
+    TMEM lane quarter) and each row's n-tiles split over two CTAs whose lists
+    the last CTA merges."""
+    cfg = SMALL.replace(B=1, S=256, ctx=20000, q_start=20000 - 256, topk=topk)
+    assert cfg.NB > 256  # two 256-block n-tiles
+    w = generate(cfg)
+    _, ids, out = run_gpu(cfg, upload(w), phase="prefill")
+    ref_ids, ref_out = oracle_rows(cfg, w)
+    assert torch.equal(ids.cpu().reshape(-1, topk), ref_ids)
+    assert_out_close(out.reshape(-1, cfg.H_q, cfg.hd), ref_out, cfg.torch_dtype, "long lists")
+
+
+@pytest.mark.parametrize("B,H_kv", [(20, 2), (60, 1)])
+def test_decode_attention_deep_ring_uneven_splits(B, H_kv):
+    """Decode shapes whose (row, KV head) pairs fill the SMs with 3- or 2-CTA
+    clusters: the 6-stage ring, with units split unevenly over the cluster."""
+    cfg = CONFIGS["decode"].replace(name="deep", B=B, H_kv=H_kv, ctx=6000, q_start=5999,
+                                    topk=11, spare_pages=8)
+    w = generate(cfg)
+    d = upload(w)
+    _, ids, out = run_gpu(cfg, d)
+    ref_ids, ref_out = oracle_rows(cfg, w)
+    assert torch.equal(ids.cpu().reshape(-1, cfg.topk), ref_ids)
+    assert_out_close(out.reshape(-1, cfg.H_q, cfg.hd), ref_out, cfg.torch_dtype, "deep ring")
+    bt = lci.create_block_table(d["block_table"], d["k_pool"])
+    ids_f, out_f = lci.sparse_decode(d["q_c"], d["k_c"], d["ctx_len"], d["q_start"], cfg.topk,
+                                     d["q"], d["k_pool"], d["v_pool"], bt)
+    torch.cuda.synchronize()
+    assert torch.equal(ids_f, ids) and torch.equal(out_f, out)
