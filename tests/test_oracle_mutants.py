@@ -38,6 +38,25 @@ MUTANTS = [
     ("bf16 widened with the wrong shift", "<< 16;", "<< 15;"),
     ("block table row stride ignored", "int64_t page = block_table[b * nb_max + j];\n            for (int64_t u = 0; u < bs; ++u) {",
      "int64_t page = block_table[j];\n            for (int64_t u = 0; u < bs; ++u) {"),
+    ("visibility ignores the context length",
+     "    int64_t last = p < ctx - 1 ? p : ctx - 1;\n    if (last < 0) return 0;",
+     "    int64_t last = p;\n    if (last < 0) return 0;"),
+    ("attention ignores the context length",
+     "        int64_t last = p < ctx - 1 ? p : ctx - 1;\n        double* logit = (double*)malloc(sizeof(double) * (size_t)(topk * bs));",
+     "        int64_t last = p;\n        double* logit = (double*)malloc(sizeof(double) * (size_t)(topk * bs));"),
+    ("unused slots padded with block 0", "ids[r * topk + i] = i < k ? (int32_t)cand[i].id : -1;",
+     "ids[r * topk + i] = i < k ? (int32_t)cand[i].id : 0;"),
+    ("softmax normaliser dropped",
+     "            for (int64_t d = 0; d < hd; ++d) o[d] /= den;\n        }\n        free(logit); free(tok_page); free(tok_slot);",
+     "        }\n        free(logit); free(tok_page); free(tok_slot);"),
+    ("dense reference ignores the selection", "if (!selected) { logit[t] = -INFINITY; continue; }",
+     "if (0) { logit[t] = -INFINITY; continue; }"),
+    ("last visible block left out of the ranking", "qsort(cand, (size_t)vis, sizeof(scored_block), rank_cmp);",
+     "qsort(cand, (size_t)(vis > 0 ? vis - 1 : 0), sizeof(scored_block), rank_cmp);"),
+    ("attention reads the sequence's query, not the row's",
+     "dot += ld(q, dt, (row * H_q + h) * hd + d) *\n                           ld(k_pool, dt, pool_off(tok_page[t], g, tok_slot[t], d, H_kv, bs, hd));",
+     "dot += ld(q, dt, (b * H_q + h) * hd + d) *\n                           ld(k_pool, dt, pool_off(tok_page[t], g, tok_slot[t], d, H_kv, bs, hd));"),
+    ("token slot off by one", "tok_slot[n] = u;", "tok_slot[n] = u > 0 ? u - 1 : 0;"),
 ]
 
 

@@ -242,6 +242,25 @@ def test_sparse_attn_matches_sdpa_with_block_mask(H_q, H_kv):
         torch.testing.assert_close(got[r], ref, rtol=1e-12, atol=1e-12)
 
 
+def test_query_past_the_context_attends_only_cached_tokens():
+    # last = min(p, ctx - 1): a query positioned beyond the end of its cache
+    # attends to tokens up to ctx - 1 only, also inside a selected block whose
+    # later slots lie past the context.
+    q, k_pool, v_pool, table, _, _ = _attn_case(seed=17, S=3)
+    B, S, H_q, hd = q.shape
+    NB, bs, H_kv = table.shape[1], k_pool.shape[2], k_pool.shape[1]
+    ctx = torch.tensor([NB * bs - 3, 10], dtype=torch.int32)
+    q0 = torch.tensor([NB * bs + 5, 30], dtype=torch.int32)
+    ids = torch.arange(NB, dtype=torch.int32).repeat(B * S, 1)
+    scale = 0.3
+    got = oracle.sparse_attn(q, k_pool, v_pool, table, ids, ctx, q0, scale)
+    for r in range(B * S):
+        b, s = divmod(r, S)
+        mask = _block_mask(ids[r].tolist(), bs, NB, int(ctx[b]) - 1)
+        ref = _sdpa_row(q[b, s], k_pool, v_pool, table, b, mask, scale, H_kv)
+        torch.testing.assert_close(got[r], ref, rtol=1e-12, atol=1e-12)
+
+
 def test_sparse_attn_equals_dense_masked():
     q, k_pool, v_pool, table, ctx, q0 = _attn_case(seed=13, S=5)
     B, S = q.shape[:2]
