@@ -408,6 +408,27 @@ def measure(cfg, steps, warmup, device, rank=0, seed_offset=0, with_e2e=True):
     return res
 
 
+def config_entry(cfg, r, pk):
+    """Per-workload figures of one measure() result: times, rates, and each
+    kernel's rate as a fraction of the measured HBM and bf16 peaks."""
+    a = r["alg"]
+    rows = cfg.B * cfg.S
+    ti, ta = r["t_index_ms"] * 1e-3, r["t_attn_ms"] * 1e-3
+    e = {
+        "ms_step": r["t_step_ms"], "ms_index": r["t_index_ms"], "ms_attn": r["t_attn_ms"],
+        "tokens_per_s": rows / (r["t_step_ms"] * 1e-3),
+        "index_gbs": a["index_bytes"] / ti / 1e9,
+        "index_tflops": a["index_flops"] / ti / 1e12,
+        "attn_gbs": a["attn_bytes"] / ta / 1e9,
+        "attn_tflops": a["attn_flops"] / ta / 1e12,
+    }
+    e["index_frac_hbm"] = e["index_gbs"] / pk["hbm_gbs"]
+    e["index_frac_bf16"] = e["index_tflops"] / pk["bf16_tflops"]
+    e["attn_frac_hbm"] = e["attn_gbs"] / pk["hbm_gbs"]
+    e["attn_frac_bf16"] = e["attn_tflops"] / pk["bf16_tflops"]
+    return e
+
+
 # ------------------------------------------------------------------ CPU oracle
 
 def oracle_throughput(cfg, min_seconds=10.0, max_rows=None, w=None):
@@ -564,16 +585,7 @@ def main():
                 continue
             c = CONFIGS[name]
             r = measure(c, max(5, args.steps // 5), 3, device, with_e2e=False)
-            a = r["alg"]
-            rows = c.B * c.S
-            extra[name] = {
-                "ms_step": r["t_step_ms"], "ms_index": r["t_index_ms"], "ms_attn": r["t_attn_ms"],
-                "tokens_per_s": rows / (r["t_step_ms"] * 1e-3),
-                "index_gbs": a["index_bytes"] / (r["t_index_ms"] * 1e-3) / 1e9,
-                "index_tflops": a["index_flops"] / (r["t_index_ms"] * 1e-3) / 1e12,
-                "attn_gbs": a["attn_bytes"] / (r["t_attn_ms"] * 1e-3) / 1e9,
-                "attn_tflops": a["attn_flops"] / (r["t_attn_ms"] * 1e-3) / 1e12,
-            }
+            extra[name] = config_entry(c, r, pk)
             del r
             torch.cuda.empty_cache()
         line["other_configs"] = extra

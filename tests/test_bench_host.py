@@ -46,3 +46,15 @@ def test_profiled_traffic_is_reported_only_for_the_captured_sources(monkeypatch)
     monkeypatch.setattr(bench, "sources_digest", lambda: "0" * 16)
     assert bench.profiled_traffic(*key) is None
     assert bench.profiled_traffic("decode", "no_such_kernel") is None
+
+
+def test_config_entry_rates_and_fractions():
+    cfg = bench.CONFIGS["1m_chunk"]
+    r = {"t_step_ms": 0.5, "t_index_ms": 0.1, "t_attn_ms": 0.4,
+         "alg": {"index_bytes": 2e8, "index_flops": 6e10, "attn_bytes": 8e8, "attn_flops": 4e10}}
+    pk = {"hbm_gbs": 8000.0, "bf16_tflops": 2000.0}
+    e = bench.config_entry(cfg, r, pk)
+    assert abs(e["tokens_per_s"] - cfg.B * cfg.S / 5e-4) < 1e-6
+    assert abs(e["index_gbs"] - 2000.0) < 1e-9 and abs(e["index_frac_hbm"] - 0.25) < 1e-12
+    assert abs(e["index_tflops"] - 600.0) < 1e-9 and abs(e["index_frac_bf16"] - 0.3) < 1e-12
+    assert abs(e["attn_gbs"] - 2000.0) < 1e-9 and abs(e["attn_frac_bf16"] - 0.05) < 1e-12
