@@ -119,3 +119,55 @@ def test_binding_rejects_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
         binding._dev(torch.zeros(4), "x")
+
+
+def test_sparse_decode_host_checks(lib):
+    h = ctypes.c_void_p()
+    # bf16 table: 2 sequences x 8 blocks of 64 tokens, 1 KV head of dim 128, 20 pages
+    assert lib.lci_create_block_table(FAKE, 2, 8, 20, 64, 1, 128, 1, ctypes.byref(h)) == 0
+    try:
+        need = ctypes.c_size_t()
+        assert lib.lci_sparse_decode_workspace_size(2, 1, 8, 128, 8, 4, ctypes.byref(need)) == 0
+        assert need.value > 0
+        assert lib.lci_sparse_decode_workspace_size(2, 1, 8, 128, 8, 4, None) == INVALID
+
+        def dec(**kw):
+            a = dict(q_c=FAKE, k_c=FAKE, dtype=1, B=2, S=1, H_i=8, d_c=128, nb_max=8, ctx=FAKE,
+                     q0=FAKE, topk=4, q=FAKE, H_q=16, kp=FAKE, vp=FAKE, t=h, scale=0.0, ids=FAKE,
+                     out=FAKE, ws=FAKE, ws_bytes=need.value)
+            a.update(kw)
+            return lib.lci_sparse_decode(a["q_c"], a["k_c"], a["dtype"], a["B"], a["S"], a["H_i"],
+                                         a["d_c"], a["nb_max"], a["ctx"], a["q0"], a["topk"],
+                                         a["q"], a["H_q"], a["kp"], a["vp"], a["t"], a["scale"],
+                                         a["ids"], a["out"], a["ws"], a["ws_bytes"], None)
+        assert dec(q_c=None) == INVALID
+        assert dec(out=None) == INVALID
+        assert dec(t=None) == INVALID
+        assert dec(nb_max=7) == INVALID                 # differs from the table's 8 blocks
+        assert dec(dtype=0) == INVALID                  # fp32 indexer with a bf16 cache
+        assert dec(B=3) == INVALID                      # more sequences than the table
+        assert dec(q_c=ctypes.c_void_p(FAKE.value + 8)) == INVALID  # not 16-byte aligned
+        assert dec(ws=None) == WORKSPACE
+        assert dec(ws_bytes=need.value - 1) == WORKSPACE
+        assert dec(ws=ctypes.c_void_p(FAKE.value + 16)) == WORKSPACE  # not 256-byte aligned
+        assert dec(scale=float("inf")) == INVALID
+        assert dec(topk=0) == INVALID
+    finally:
+        assert lib.lci_destroy_block_table(h) == 0
+
+
+def test_index_select_noalloc_host_checks(lib):
+    def na(**kw):
+        a = dict(q_c=FAKE, k_c=FAKE, dtype=1, B=2, S=1, H_i=8, d_c=128, bs=64, nb_max=512,
+                 ctx=FAKE, q0=FAKE, topk=32, phase=0, ids=FAKE)
+        a.update(kw)
+        return lib.lci_index_select_noalloc(a["q_c"], a["k_c"], a["dtype"], a["B"], a["S"],
+                                            a["H_i"], a["d_c"], a["bs"], a["nb_max"], a["ctx"],
+                                            a["q0"], a["topk"], a["phase"], a["ids"], None)
+    assert na(k_c=None) == INVALID
+    assert na(bs=0) == INVALID
+    assert na(phase=9) == INVALID
+    assert na(k_c=ctypes.c_void_p(FAKE.value + 4)) == INVALID
+    # 256 rows x 16384 blocks of fp32 scores alone exceed the built-in scratch
+    assert na(B=256, nb_max=16384) == WORKSPACE
+    assert b"scratch" in lib.lci_last_error()
