@@ -71,9 +71,9 @@ def peaks():
 # sources the capture ran. Once those sources change the figure no longer
 # describes the kernel and the bench reports traffic as null.
 PROFILED_TRAFFIC = {
-    ("decode", "index_select"): (33683200, "c2e06c74883d2e86"),
-    ("decode", "sparse_attn"): (33798400, "c2e06c74883d2e86"),
-    ("1m_chunk", "index_select"): (25226496, "c2e06c74883d2e86"),
+    ("decode", "index_select"): (33683200, "29249c0d5d426974"),
+    ("decode", "sparse_attn"): (33798400, "29249c0d5d426974"),
+    ("1m_chunk", "index_select"): (25226496, "29249c0d5d426974"),
 }
 
 
