@@ -34,6 +34,11 @@
  * - Device-side checks (block ids outside [-1, nb_max), table entries outside
  *   [0, num_pages)) never trap: the offending item is skipped, a sticky device
  *   status word is set, and lci_get_device_status reports it.
+ * - Every device-side wait (a copy landing in shared memory, a row published
+ *   by a producer) is bounded by a wait limit (lci_set_wait_limit_ns, 2 s by
+ *   default). A wait that runs out skips its work, sets the sticky status word
+ *   and lets the kernel return; lci_get_device_status then reports
+ *   LCI_ERR_TIMEOUT. No kernel of the library can wait forever.
  * - Query position: p = d_q_start[b] + s for query s of sequence b. The last
  *   attendable token is last = min(p, d_ctx_len[b] - 1). Block j is causal-
  *   visible when j * block_size <= last (so vis = min(nb_max, last/bs + 1)).
@@ -61,7 +66,7 @@ typedef enum {
     LCI_ERR_WORKSPACE = 3,     /* workspace missing, misaligned or too small */
     LCI_ERR_CUDA = 4,          /* a CUDA runtime call failed (see lci_last_error) */
     LCI_ERR_DEVICE_BOUNDS = 5, /* a device-side bounds check fired (sticky word) */
-    LCI_ERR_TIMEOUT = 6        /* reserved: a bounded device wait gave up */
+    LCI_ERR_TIMEOUT = 6        /* a bounded device wait gave up (sticky word) */
 } lci_status;
 
 typedef enum { LCI_F32 = 0, LCI_BF16 = 1 } lci_dtype;
@@ -125,7 +130,9 @@ LCI_API lci_status lci_block_compress(const void* k_idx, lci_dtype dtype, int32_
                               void* stream);
 
 /*
- * Workspace bytes lci_index_select needs for these sizes (0 is possible).
+ * Workspace bytes lci_index_select needs for these sizes, for either dtype
+ * (0 is possible). With LCI_PHASE_DECODE it is the scratch of the
+ * one-row-at-a-time schedule alone, which lci_index_select_noalloc uses.
  */
 LCI_API lci_status lci_index_select_workspace_size(int32_t batch, int32_t S, int32_t H_i, int32_t d_c,
                                            int32_t nb_max, int32_t topk, lci_phase phase,
@@ -206,11 +213,15 @@ LCI_API lci_status lci_sparse_attn(const void* q, int32_t batch, int32_t S, int3
  * workspace; it always runs the one-row-at-a-time kernel (the decode schedule)
  * whatever the phase. Its scratch is one fixed array of
  * LCI_NOALLOC_SCRATCH_BYTES bytes inside the library, which every GPU that
- * loads the library holds until the process exits. Sizes whose scratch would
- * exceed it (about batch*S*(4*nb_max + 4) bytes plus alignment) return
+ * loads the library holds until the process exits. The scratch a call needs is
+ *   align256(4*rows) + align256(4*rows*nb_max) + align256(4*rows*nchunks)
+ * bytes (rows = batch*S; nchunks <= nb_max, the chunks a row is scored in),
+ * which is exactly what lci_index_select_workspace_size returns for the same
+ * sizes with LCI_PHASE_DECODE. Sizes whose scratch exceeds the array return
  * LCI_ERR_WORKSPACE before anything is launched.
- * The first call on each device looks up the array's device address (with that
- * device current); make that first call before any stream capture. Each call
+ * Every call looks up the array's device address for the current device (the
+ * first lookup on a device may load the library's device code: make the first
+ * call on each device before any stream capture). Each call
  * clears the array's arrival counters on `stream` before its kernel runs (the
  * array keeps the previous call's contents otherwise). All calls on a device
  * share the one array: calls that may overlap on the GPU (other streams, other
@@ -243,8 +254,11 @@ LCI_API lci_status lci_sparse_decode_workspace_size(int32_t batch, int32_t S, in
  * Arguments are those of the two calls; k_c's nb_max must equal the table's
  * max_blocks and all floating inputs share one dtype. The workspace holds the
  * indexer's scratch and per-row publication flags: zero-fill it before its
- * first call and again before using it with other sizes; every call leaves it
- * ready for the next. Calls sharing a workspace must not overlap in time.
+ * first call and again before using it with other sizes or after a call that
+ * failed on the device; every successful call leaves it ready for the next.
+ * The flags are cleared by each call itself before its attention kernel can
+ * start, so a flag left set by an earlier call is never taken for a new
+ * publication. Calls sharing a workspace must not overlap in time.
  */
 LCI_API lci_status lci_sparse_decode(const void* q_c, const void* k_c, lci_dtype dtype,
                                      int32_t batch, int32_t S, int32_t H_i, int32_t d_c,
@@ -256,9 +270,44 @@ LCI_API lci_status lci_sparse_decode(const void* q_c, const void* k_c, lci_dtype
                                      void* stream);
 
 /*
+ * A3 + A4 with the attention of each query row started as soon as a producer
+ * publishes that row ([Hetero] §IV: index retrieval and attention should be
+ * pipelined so that retrieval latency is hidden; [GPU-stack] "Separate Paths
+ * for Prefill and Decode": decode as a pipeline of index prefetching and
+ * incremental aggregation). This is the consumer half of lci_sparse_decode for
+ * callers that produce the block ids themselves, in a kernel running on
+ * another stream or earlier on this one.
+ *   d_ready  [batch][S] uint32, device. The producer writes row r of d_ids,
+ *            then sets d_ready[r] to a nonzero value with release semantics
+ *            (st.release.gpu, or a __threadfence() before a plain store). The
+ *            library only reads d_ready; the caller clears it between calls.
+ * Other arguments, layouts and results are those of lci_sparse_attn. A row
+ * whose flag stays zero for the wait limit (lci_set_wait_limit_ns) gets a
+ * zero output row, and lci_get_device_status reports LCI_ERR_TIMEOUT.
+ * Supported shape (else LCI_ERR_UNSUPPORTED): bf16 pools, head_dim 128,
+ * block_size a multiple of 64, at most 16 query heads per KV head.
+ */
+LCI_API lci_status lci_sparse_attn_pipelined(const void* q, int32_t batch, int32_t S, int32_t H_q,
+                                             const void* k_pool, const void* v_pool,
+                                             const lci_block_table* table, const int32_t* d_ids,
+                                             int32_t topk, const int32_t* d_ctx_len,
+                                             const int32_t* d_q_start, float scale,
+                                             const uint32_t* d_ready, void* out, void* stream);
+
+/*
+ * Limit, in nanoseconds of GPU global time, of every bounded device wait of
+ * the library on the current device (default 2 s; 1 ns .. 60 s, else
+ * LCI_ERR_INVALID_ARG). Takes effect for kernels launched after the call;
+ * not for use during stream capture.
+ */
+LCI_API lci_status lci_set_wait_limit_ns(uint64_t ns);
+LCI_API lci_status lci_get_wait_limit_ns(uint64_t* ns);
+
+/*
  * Synchronises `stream`, then returns and clears the sticky device status
- * word of the current device: LCI_OK, or LCI_ERR_DEVICE_BOUNDS when a device
- * bounds check fired since the last call.
+ * word of the current device: LCI_OK; LCI_ERR_TIMEOUT when a bounded device
+ * wait ran out since the last call; otherwise LCI_ERR_DEVICE_BOUNDS when a
+ * device bounds check fired. lci_last_error() lists every flag that was set.
  */
 LCI_API lci_status lci_get_device_status(void* stream);
 

@@ -5,11 +5,13 @@ thin ctypes binding and ``workloads`` the seeded synthetic input generator.
 Importing the package loads nothing; the library is loaded on first use.
 """
 from .lci import (BlockTable, LciError, block_compress, create_block_table, get_device_status,
-                  index_select, index_select_workspace_size, load_library, sparse_attn,
-                  sparse_attn_workspace_size, sparse_decode,
+                  get_wait_limit_ns, index_select, index_select_noalloc,
+                  index_select_workspace_size, load_library, set_wait_limit_ns, sparse_attn,
+                  sparse_attn_pipelined, sparse_attn_workspace_size, sparse_decode,
                   sparse_decode_workspace_size, version)
 
 __all__ = ["BlockTable", "LciError", "block_compress", "create_block_table", "get_device_status",
-           "index_select", "index_select_workspace_size", "load_library", "sparse_attn",
-           "sparse_attn_workspace_size", "sparse_decode", "sparse_decode_workspace_size",
-           "version"]
+           "get_wait_limit_ns", "index_select", "index_select_noalloc",
+           "index_select_workspace_size", "load_library", "set_wait_limit_ns", "sparse_attn",
+           "sparse_attn_pipelined", "sparse_attn_workspace_size", "sparse_decode",
+           "sparse_decode_workspace_size", "version"]

@@ -64,8 +64,7 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
     const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ table, int nb_max,
     int num_pages, int H_kv, int bs, int S, int H_q, const int32_t* __restrict__ ids, int topk,
     const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ q_start, float scale_log2,
-    __nv_bfloat16* __restrict__ out, int nsplit, unsigned int* __restrict__ ready,
-    unsigned int* __restrict__ consumed) {
+    __nv_bfloat16* __restrict__ out, int nsplit, const unsigned int* __restrict__ ready) {
     using namespace dec;
     namespace cg = cooperative_groups;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -127,29 +126,20 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
         const int nlines = min(nb_max, 8192) / 32;  // 128-byte lines of the row
         for (int l = lane; l < nlines; l += 32) prefetch_l2(trow + l * 32);
     }
-    // Block ids come from the previous kernel on the stream: either wait for
-    // that whole grid (programmatic dependent launch), or, when it publishes
-    // rows one by one, only for this row's ready flag (bounded wait).
+    // Block ids come from a producer: either the previous kernel on the stream
+    // (programmatic dependent launch: wait for that whole grid), or a producer
+    // that publishes rows one by one by a release store of a nonzero ready[row]
+    // after writing the row's ids (bounded wait on this row's flag only). The
+    // library's producer clears its flags itself before this grid can start. A
+    // row whose flag never comes is skipped (zero output, time-out status).
+    __shared__ int s_alive;
     if (ready == nullptr) {
         pdl_wait();
     } else {
-        if (tid == 0) {
-            const unsigned long long t0 = global_ns();
-            while (ld_acquire_gpu(ready + row) == 0u) {
-                if (global_ns() - t0 > kWaitLimitNs) {
-                    raise_status(kStatusTimeout);
-                    break;
-                }
-            }
-            // the last of the row's CTAs to pass resets the flag for the next call
-            const unsigned n = atomicAdd(consumed + row, 1u);
-            if (n == (unsigned)(H_kv * nsplit - 1)) {
-                consumed[row] = 0u;
-                ready[row] = 0u;
-            }
-        }
+        if (tid == 0) s_alive = wait_flag_set(ready + row) ? 1 : 0;
         __syncthreads();
     }
+    const bool alive = ready == nullptr || s_alive != 0;
 
     float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
     float o[2][8][4];
@@ -165,11 +155,11 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
         // Lanes resolve 32 units at a time (block id -> page -> TMA row), so the
         // dependent id and table loads overlap; lane 0 then issues the copies.
         const int32_t* row_ids = ids + (size_t)row * topk;
-        bool alive = true;
-        for (int base = u0; base < u1 && alive; base += 32) {
+        bool running = true;
+        for (int base = u0; base < u1 && running; base += 32) {
             const int u = base + lane;
             int t0 = -1, y = 0;
-            if (u < u1) {
+            if (u < u1 && alive) {
                 const int i = u / tiles_per_block, sub = u - i * tiles_per_block;
                 const int j = __ldcg(row_ids + i);
                 if (j >= 0 && j < nb_max) {
@@ -208,7 +198,7 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
                     }
                 }
                 if (!__shfl_sync(0xffffffffu, ok, 0)) {
-                    alive = false;
+                    running = false;
                     break;
                 }
             }

@@ -15,7 +15,12 @@ __device__ unsigned int g_device_status = 0u;
 enum : unsigned int {
     kStatusBadBlockId = 1u << 0,  // block id outside [-1, nb_max)
     kStatusBadPage = 1u << 1,     // table entry outside [0, num_pages)
+    kStatusTimeout = 1u << 2,     // a bounded device wait gave up
 };
+
+// Limit of every bounded device wait, in nanoseconds of global time. Set from
+// the host (lci_set_wait_limit_ns) between launches; 2 s unless changed.
+__device__ unsigned long long g_wait_limit_ns = 2000000000ull;
 
 __device__ __forceinline__ void raise_status(unsigned int bits) {
     atomicOr(&g_device_status, bits);

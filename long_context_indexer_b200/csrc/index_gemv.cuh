@@ -52,12 +52,24 @@ __global__ void __launch_bounds__(NT) index_gemv_select_kernel(
     constexpr int NW = NT / 32;
     constexpr int E = ElemsPer16B<T>::v;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    // Let the attention kernel that follows on the stream start its prologue;
-    // it waits for this grid's results before reading the block ids.
-    pdl_trigger();
     // chunk fastest: a row's CTAs are dispatched together, so rows complete (and
     // are selected) one after another instead of all at the end
     const int row = blockIdx.x / nchunks, chunk = blockIdx.x - row * nchunks;
+    // Publication flags (one per row) start every call cleared: the row's first
+    // CTA clears its flag before this CTA lets the dependent grid launch, so a
+    // flag left set by an earlier call (say one whose consumer gave up waiting)
+    // can never be taken for this call's publication. The row's publishing CTA
+    // arrives on the row counter after this CTA, so it stores after the clear.
+    if (ready != nullptr && chunk == 0) {
+        if (tid == 0) {
+            ready[row] = 0u;
+            __threadfence();
+        }
+        __syncthreads();
+    }
+    // Let the attention kernel that follows on the stream start its prologue;
+    // it waits for this grid's results (or its row's flag) before reading ids.
+    pdl_trigger();
     const int b = row / S, s = row - b * S;
     const long long p = (long long)__ldg(&q_start[b]) + s;
     const int vis = visible_blocks(p, __ldg(&ctx_len[b]), bs, nb_max);

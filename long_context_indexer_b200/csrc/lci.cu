@@ -55,6 +55,7 @@ lci_status check_launch(const char* what) {
 }
 
 constexpr size_t kAlign = 256;
+constexpr uint64_t kMaxWaitLimitNs = 60ull * 1000000000ull;  // 60 s
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool dtype_ok(lci_dtype d) { return d == LCI_F32 || d == LCI_BF16; }
@@ -81,21 +82,30 @@ struct IndexPlan {
     size_t smem;
 };
 
+// Blocks per chunk: at most 32 blocks and 32 KiB of block keys, halved while
+// the grid would not cover the 148 SMs about four times.
+int index_chunk(long long rows, int32_t K, int32_t nb_max, size_t esz) {
+    const size_t row_bytes = (size_t)K * esz;
+    int chunk = 32;
+    while (chunk > 1 && (size_t)chunk * row_bytes > 32768) chunk >>= 1;
+    while (chunk > 4 && rows * ((nb_max + chunk - 1) / chunk) < 4 * 148) chunk >>= 1;
+    return chunk;
+}
+
 IndexPlan plan_index(int32_t batch, int32_t S, int32_t K, int32_t nb_max, size_t esz) {
     IndexPlan pl{};
     const long long rows = (long long)batch * S;
     const size_t row_bytes = (size_t)K * esz;
-    // Chunks of at most 32 blocks and 32 KiB of block keys, halved while the
-    // grid would not cover the 148 SMs about four times.
-    int chunk = 32;
-    while (chunk > 1 && (size_t)chunk * row_bytes > 32768) chunk >>= 1;
-    while (chunk > 4 && rows * ((nb_max + chunk - 1) / chunk) < 4 * 148) chunk >>= 1;
+    const int chunk = index_chunk(rows, K, nb_max, esz);
     pl.chunk_blocks = chunk;
     pl.nchunks = (nb_max + chunk - 1) / chunk;
+    // The layout is sized for the smaller fp32 chunk, so that one workspace
+    // size serves both element types.
+    const int nchunks_alloc = (nb_max + index_chunk(rows, K, nb_max, 4) - 1) / index_chunk(rows, K, nb_max, 4);
     pl.off_counters = 0;
     pl.off_scores = align_up((size_t)rows * sizeof(unsigned int));
     pl.off_chunk_max = pl.off_scores + align_up((size_t)rows * nb_max * sizeof(float));
-    pl.bytes = pl.off_chunk_max + align_up((size_t)rows * pl.nchunks * sizeof(uint32_t));
+    pl.bytes = pl.off_chunk_max + align_up((size_t)rows * nchunks_alloc * sizeof(uint32_t));
     pl.qreg = row_bytes == 2048;
     const size_t stage = (size_t)chunk * row_bytes + (pl.qreg ? 0 : (size_t)K * sizeof(float));
     const size_t sel = sizeof(lci::SelectSmem);
@@ -360,7 +370,7 @@ lci_status launch_attn_decode(const void* q, int32_t batch, int32_t S, int32_t H
                               const void* k_pool, const void* v_pool, const lci_block_table* t,
                               const int32_t* ids, int32_t topk, const int32_t* ctx_len,
                               const int32_t* q_start, float scale, void* out, cudaStream_t st,
-                              unsigned int* ready = nullptr, unsigned int* consumed = nullptr) {
+                              const unsigned int* ready = nullptr, bool early_start = true) {
     const long long rows = (long long)t->num_pages * t->num_kv_heads * t->block_size;
     CUtensorMap tm_k, tm_v;
     lci_status s = encode_pool_map(&tm_k, k_pool, rows);
@@ -390,9 +400,11 @@ lci_status launch_attn_decode(const void* q, int32_t batch, int32_t S, int32_t H
         attrs[na].val.clusterDim.z = 1;
         ++na;
     }
-    attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attrs[na].val.programmaticStreamSerializationAllowed = 1;
-    ++na;
+    if (early_start) {  // may start under the previous kernel on the stream
+        attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attrs[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
     cfg.attrs = attrs;
     cfg.numAttrs = na;
     const float scale_log2 = scale * 1.4426950408889634f;
@@ -401,7 +413,7 @@ lci_status launch_attn_decode(const void* q, int32_t batch, int32_t S, int32_t H
     cudaError_t e = cudaLaunchKernelEx(
         &cfg, kern, tm_k, tm_v, static_cast<const __nv_bfloat16*>(q),
         t->d_table, t->max_blocks, t->num_pages, t->num_kv_heads, t->block_size, S, H_q, ids, topk,
-        ctx_len, q_start, scale_log2, static_cast<__nv_bfloat16*>(out), nsplit, ready, consumed);
+        ctx_len, q_start, scale_log2, static_cast<__nv_bfloat16*>(out), nsplit, ready);
     if (e != cudaSuccess) return fail(LCI_ERR_CUDA, "sparse_attn: %s", cudaGetErrorString(e));
     return check_launch("sparse_attn");
 }
@@ -503,7 +515,7 @@ lci_status lci_index_select_workspace_size(int32_t batch, int32_t S, int32_t H_i
     // the schedule a bf16 call with these sizes takes (fp32 always runs row-wise)
     const int K = H_i * d_c;
     const bool tc = prefill_path(LCI_BF16, phase, S, K, topk, nullptr, nullptr);
-    const size_t g = plan_index(batch, S, K, nb_max, 2).bytes;
+    const size_t g = plan_index(batch, S, K, nb_max, 2).bytes;  // same for both types
     *bytes = tc ? std::max(g, plan_prefill(batch, S, K, nb_max, topk).bytes) : g;
     return ok();
 }
@@ -587,29 +599,16 @@ lci_status lci_sparse_attn(const void* q, int32_t batch, int32_t S, int32_t H_q,
 // The scratch of lci_index_select_noalloc: one file-scope device array per GPU
 // that loads the library. Host code never passes its name to a kernel (on the
 // host it is only a stand-in symbol); the device address comes from
-// cudaGetSymbolAddress, once per device.
+// cudaGetSymbolAddress, looked up on every call with the caller's device
+// current (a host-side lookup once the module is loaded).
 static __device__ __align__(256) unsigned char g_noalloc_scratch[LCI_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-constexpr int kNoAllocMaxDevices = 64;
-std::once_flag g_noalloc_once[kNoAllocMaxDevices];
-void* g_noalloc_ptr[kNoAllocMaxDevices];
-cudaError_t g_noalloc_err[kNoAllocMaxDevices];
-
 lci_status noalloc_scratch(void** out) {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return fail(LCI_ERR_CUDA, "index_select_noalloc: %s", cudaGetErrorString(e));
-    if (dev < 0 || dev >= kNoAllocMaxDevices)
-        return fail(LCI_ERR_UNSUPPORTED, "index_select_noalloc: device %d above %d", dev,
-                    kNoAllocMaxDevices - 1);
-    std::call_once(g_noalloc_once[dev], [dev] {
-        g_noalloc_err[dev] = cudaGetSymbolAddress(&g_noalloc_ptr[dev], g_noalloc_scratch);
-    });
-    if (g_noalloc_err[dev] != cudaSuccess)
+    cudaError_t e = cudaGetSymbolAddress(out, g_noalloc_scratch);
+    if (e != cudaSuccess)
         return fail(LCI_ERR_CUDA, "index_select_noalloc: scratch address lookup failed: %s",
-                    cudaGetErrorString(g_noalloc_err[dev]));
-    *out = g_noalloc_ptr[dev];
+                    cudaGetErrorString(e));
     return LCI_OK;
 }
 }  // namespace
@@ -656,16 +655,15 @@ extern "C" {
 
 struct DecodePlan {
     IndexPlan ix;
-    size_t off_ready, off_consumed, bytes;
+    size_t off_ready, bytes;
 };
 
-DecodePlan plan_decode(int32_t batch, int32_t S, int32_t K, int32_t nb_max) {
+DecodePlan plan_decode(int32_t batch, int32_t S, int32_t K, int32_t nb_max, size_t esz) {
     DecodePlan d{};
-    d.ix = plan_index(batch, S, K, nb_max, 2);
+    d.ix = plan_index(batch, S, K, nb_max, esz);
     const size_t rows = (size_t)batch * S;
     d.off_ready = align_up(d.ix.bytes);
-    d.off_consumed = d.off_ready + align_up(rows * sizeof(unsigned int));
-    d.bytes = d.off_consumed + align_up(rows * sizeof(unsigned int));
+    d.bytes = d.off_ready + align_up(rows * sizeof(unsigned int));
     return d;
 }
 
@@ -674,7 +672,7 @@ lci_status lci_sparse_decode_workspace_size(int32_t batch, int32_t S, int32_t H_
     if (!bytes) return fail(LCI_ERR_INVALID_ARG, "sparse_decode_workspace_size: null output");
     lci_status st = check_index_args(batch, S, H_i, d_c, nb_max, topk, LCI_BF16);
     if (st != LCI_OK && st != LCI_ERR_UNSUPPORTED) return st;
-    *bytes = plan_decode(batch, S, H_i * d_c, nb_max).bytes;
+    *bytes = plan_decode(batch, S, H_i * d_c, nb_max, 2).bytes;  // same for both types
     return ok();
 }
 
@@ -698,7 +696,7 @@ lci_status lci_sparse_decode(const void* q_c, const void* k_c, lci_dtype dtype, 
     if (!aligned16(q_c) || !aligned16(k_c))
         return fail(LCI_ERR_INVALID_ARG, "sparse_decode: q_c and k_c must be 16-byte aligned");
     const int K = H_i * d_c;
-    const DecodePlan pl = plan_decode(batch, S, K, nb_max);
+    const DecodePlan pl = plan_decode(batch, S, K, nb_max, dtype_size(dtype));
     if (!workspace || workspace_bytes < pl.bytes ||
         (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
         return fail(LCI_ERR_WORKSPACE, "sparse_decode: workspace needs %zu bytes, 256-byte aligned "
@@ -710,13 +708,12 @@ lci_status lci_sparse_decode(const void* q_c, const void* k_c, lci_dtype dtype, 
     if (dtype == LCI_BF16 && decode_kernel_fits(table, H_q, k_pool, v_pool)) {
         // rows are published one by one and attended as soon as they are ready
         unsigned int* ready = reinterpret_cast<unsigned int*>(w + pl.off_ready);
-        unsigned int* consumed = reinterpret_cast<unsigned int*>(w + pl.off_consumed);
         st = launch_index_gemv<__nv_bfloat16>(q_c, k_c, batch, S, K, table->block_size, nb_max,
                                               d_ctx_len, d_q_start, topk, d_ids, workspace, pl.ix,
                                               cs, ready);
         if (st != LCI_OK) return st;
         return launch_attn_decode(q, batch, S, H_q, k_pool, v_pool, table, d_ids, topk, d_ctx_len,
-                                  d_q_start, scale, out, cs, ready, consumed);
+                                  d_q_start, scale, out, cs, ready, true);
     }
     // other shapes: the two calls in sequence
     st = dtype == LCI_F32
@@ -743,11 +740,52 @@ lci_status lci_get_device_status(void* stream) {
     e = cudaMemcpyFromSymbol(&v, lci::g_device_status, sizeof v);
     if (e == cudaSuccess) e = cudaMemcpyToSymbol(lci::g_device_status, &zero, sizeof zero);
     if (e != cudaSuccess) return fail(LCI_ERR_CUDA, "get_device_status: %s", cudaGetErrorString(e));
-    if (v != 0)
-        return fail(LCI_ERR_DEVICE_BOUNDS, "device bounds check fired (flags 0x%x:%s%s)", v,
-                    (v & lci::kStatusBadBlockId) ? " block id" : "",
-                    (v & lci::kStatusBadPage) ? " page" : "");
+    if (v == 0) return ok();
+    const lci_status code = (v & lci::kStatusTimeout) ? LCI_ERR_TIMEOUT : LCI_ERR_DEVICE_BOUNDS;
+    return fail(code, "device status flags 0x%x:%s%s%s", v,
+                (v & lci::kStatusBadBlockId) ? " block id out of range" : "",
+                (v & lci::kStatusBadPage) ? " page out of range" : "",
+                (v & lci::kStatusTimeout) ? " bounded wait timed out" : "");
+}
+
+lci_status lci_set_wait_limit_ns(uint64_t ns) {
+    if (ns == 0 || ns > kMaxWaitLimitNs)
+        return fail(LCI_ERR_INVALID_ARG, "set_wait_limit_ns: %llu outside [1, %llu]",
+                    (unsigned long long)ns, (unsigned long long)kMaxWaitLimitNs);
+    const unsigned long long v = ns;
+    cudaError_t e = cudaMemcpyToSymbol(lci::g_wait_limit_ns, &v, sizeof v);
+    if (e != cudaSuccess) return fail(LCI_ERR_CUDA, "set_wait_limit_ns: %s", cudaGetErrorString(e));
     return ok();
+}
+
+lci_status lci_get_wait_limit_ns(uint64_t* ns) {
+    if (!ns) return fail(LCI_ERR_INVALID_ARG, "get_wait_limit_ns: null output");
+    unsigned long long v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, lci::g_wait_limit_ns, sizeof v);
+    if (e != cudaSuccess) return fail(LCI_ERR_CUDA, "get_wait_limit_ns: %s", cudaGetErrorString(e));
+    *ns = v;
+    return ok();
+}
+
+lci_status lci_sparse_attn_pipelined(const void* q, int32_t batch, int32_t S, int32_t H_q,
+                                     const void* k_pool, const void* v_pool,
+                                     const lci_block_table* table, const int32_t* d_ids,
+                                     int32_t topk, const int32_t* d_ctx_len,
+                                     const int32_t* d_q_start, float scale,
+                                     const uint32_t* d_ready, void* out, void* stream) {
+    if (!q || !k_pool || !v_pool || !d_ids || !d_ctx_len || !d_q_start || !d_ready || !out)
+        return fail(LCI_ERR_INVALID_ARG, "sparse_attn_pipelined: null pointer argument");
+    lci_status st = check_attn_args(batch, S, H_q, table, topk);
+    if (st != LCI_OK) return st;
+    if (!decode_kernel_fits(table, H_q, k_pool, v_pool))
+        return fail(LCI_ERR_UNSUPPORTED, "sparse_attn_pipelined: needs bf16 pools, head_dim 128, "
+                    "block_size a multiple of 64, at most 16 query heads per KV head and "
+                    "16-byte aligned pools");
+    if (!(scale > 0.f)) scale = 1.0f / std::sqrt((float)table->head_dim);
+    if (!std::isfinite(scale)) return fail(LCI_ERR_INVALID_ARG, "sparse_attn_pipelined: non-finite scale");
+    return launch_attn_decode(q, batch, S, H_q, k_pool, v_pool, table, d_ids, topk, d_ctx_len,
+                              d_q_start, scale, out, static_cast<cudaStream_t>(stream),
+                              reinterpret_cast<const unsigned int*>(d_ready), false);
 }
 
 }  // extern "C"

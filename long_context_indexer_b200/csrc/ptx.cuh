@@ -1,7 +1,7 @@
 // ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers, TMA tensor
 // loads, bulk copies, programmatic dependent launch and bf16 mma.sync.
 //
-// Every wait on an mbarrier is bounded: it gives up after kWaitLimitNs of
+// Every wait on an mbarrier is bounded: it gives up after g_wait_limit_ns of
 // global time, raises kStatusTimeout in the device status word and returns
 // false, so a kernel can never hang the GPU.
 #pragma once
@@ -12,10 +12,6 @@
 #include "common.cuh"
 
 namespace lci {
-
-enum : unsigned int { kStatusTimeout = 1u << 2 };
-
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -65,12 +61,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait for phase `parity` of an mbarrier to complete, for at most kWaitLimitNs.
+// Wait for phase `parity` of an mbarrier to complete, for at most
+// g_wait_limit_ns.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
+    const unsigned long long limit = g_wait_limit_ns;
     while (!mbar_try_wait(bar, parity)) {
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (global_ns() - t0 > limit) {
             raise_status(kStatusTimeout);
             return false;
         }
@@ -126,6 +124,25 @@ __device__ __forceinline__ unsigned int ld_relaxed_gpu(const unsigned int* p) {
 }
 __device__ __forceinline__ void st_release_gpu(unsigned int* p, unsigned int v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Wait until *flag is nonzero (acquire), polling with a growing sleep so that
+// waiting CTAs do not flood L2, for at most g_wait_limit_ns. On time-out it
+// raises kStatusTimeout and returns false.
+__device__ __forceinline__ bool wait_flag_set(const unsigned int* flag) {
+    if (ld_acquire_gpu(flag) != 0u) return true;
+    const unsigned long long t0 = global_ns();
+    const unsigned long long limit = g_wait_limit_ns;
+    unsigned int sleep_ns = 32;
+    for (;;) {
+        __nanosleep(sleep_ns);
+        if (ld_acquire_gpu(flag) != 0u) return true;
+        if (global_ns() - t0 > limit) {
+            raise_status(kStatusTimeout);
+            return false;
+        }
+        sleep_ns = sleep_ns < 512 ? 2 * sleep_ns : 512;
+    }
 }
 
 // Barrier among `count` threads of the CTA (a multiple of 32), id 1..15.

@@ -53,6 +53,10 @@ SIGNATURES = {
                                 _i32, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _sz, _vp]),
     "lci_index_select_noalloc": (_st, [_vp, _vp, _st, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp,
                                        _i32, _st, _vp, _vp]),
+    "lci_sparse_attn_pipelined": (_st, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp,
+                                        _f32, _vp, _vp, _vp]),
+    "lci_set_wait_limit_ns": (_st, [ctypes.c_uint64]),
+    "lci_get_wait_limit_ns": (_st, [ctypes.POINTER(ctypes.c_uint64)]),
 }
 
 _lib = None
@@ -337,6 +341,42 @@ def sparse_decode(q_c: torch.Tensor, k_c: torch.Tensor, ctx_len: torch.Tensor,
     return ids, out
 
 
+def sparse_attn_pipelined(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                          table: BlockTable, ids: torch.Tensor, ctx_len: torch.Tensor,
+                          q_start: torch.Tensor, ready: torch.Tensor, scale: float = 0.0,
+                          out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """sparse_attn whose query rows each start once ready[row] (uint32 as int32,
+    [B, S]) is published nonzero by the caller's producer."""
+    B, S, H_q, hd = q.shape
+    topk = ids.shape[-1]
+    if tuple(ids.shape) != (B, S, topk) or tuple(ready.shape) != (B, S):
+        raise ValueError("lci: ids must be [B, S, topk] and ready [B, S]")
+    if tuple(k_pool.shape) != (table.num_pages, table.num_kv_heads, table.block_size,
+                               table.head_dim) or v_pool.shape != k_pool.shape:
+        raise ValueError("lci: pools do not match the block table")
+    if out is None:
+        out = torch.empty_like(q)
+    _check(load_library().lci_sparse_attn_pipelined(
+        _dev(q, "q", table.dtype, 4), B, S, H_q, _dev(k_pool, "k_pool", table.dtype),
+        _dev(v_pool, "v_pool", table.dtype), table.handle, _dev(ids, "ids", torch.int32, 3), topk,
+        _dev(ctx_len, "ctx_len", torch.int32, 1), _dev(q_start, "q_start", torch.int32, 1),
+        float(scale), _dev(ready, "ready", torch.int32, 2), _dev(out, "out", q.dtype, 4),
+        _stream(stream)), "lci_sparse_attn_pipelined")
+    return out
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Limit of every bounded device wait on the current device (nanoseconds)."""
+    _check(load_library().lci_set_wait_limit_ns(int(ns)), "lci_set_wait_limit_ns")
+
+
+def get_wait_limit_ns() -> int:
+    v = ctypes.c_uint64()
+    _check(load_library().lci_get_wait_limit_ns(ctypes.byref(v)), "lci_get_wait_limit_ns")
+    return v.value
+
+
 def get_device_status(stream=None) -> None:
-    """Synchronise the stream; raise LciError if a device bounds check fired."""
+    """Synchronise the stream; raise LciError (LCI_ERR_TIMEOUT or
+    LCI_ERR_DEVICE_BOUNDS) if a device wait ran out or a bounds check fired."""
     _check(load_library().lci_get_device_status(_stream(stream)), "lci_get_device_status")

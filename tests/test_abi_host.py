@@ -171,3 +171,40 @@ def test_index_select_noalloc_host_checks(lib):
     # 256 rows x 16384 blocks of fp32 scores alone exceed the built-in scratch
     assert na(B=256, nb_max=16384) == WORKSPACE
     assert b"scratch" in lib.lci_last_error()
+
+
+def test_wait_limit_and_pipelined_attention_host_checks(lib):
+    # limits outside [1 ns, 60 s] are rejected before any CUDA call
+    assert lib.lci_set_wait_limit_ns(0) == INVALID
+    assert lib.lci_set_wait_limit_ns(61 * 10**9) == INVALID
+    assert b"wait_limit" in lib.lci_last_error()
+    assert lib.lci_get_wait_limit_ns(None) == INVALID
+    h = ctypes.c_void_p()
+    assert lib.lci_create_block_table(FAKE, 2, 8, 20, 64, 1, 128, 1, ctypes.byref(h)) == 0
+    hf = ctypes.c_void_p()
+    assert lib.lci_create_block_table(FAKE, 2, 8, 20, 64, 1, 128, 0, ctypes.byref(hf)) == 0
+    try:
+        def pip(**kw):
+            a = dict(q=FAKE, B=2, S=1, H_q=16, kp=FAKE, vp=FAKE, t=h, ids=FAKE, topk=4, ctx=FAKE,
+                     q0=FAKE, scale=0.0, ready=FAKE, out=FAKE)
+            a.update(kw)
+            return lib.lci_sparse_attn_pipelined(a["q"], a["B"], a["S"], a["H_q"], a["kp"],
+                                                 a["vp"], a["t"], a["ids"], a["topk"], a["ctx"],
+                                                 a["q0"], a["scale"], a["ready"], a["out"], None)
+        assert pip(ready=None) == INVALID
+        assert pip(out=None) == INVALID
+        assert pip(t=None) == INVALID
+        assert pip(B=3) == INVALID
+        assert pip(H_q=32) == UNSUPPORTED                  # 32 query heads per KV head
+        assert pip(t=hf) == UNSUPPORTED                    # fp32 pools
+        assert pip(kp=ctypes.c_void_p(FAKE.value + 2)) == UNSUPPORTED  # misaligned pool
+        assert pip(scale=float("inf")) == INVALID
+    finally:
+        lib.lci_destroy_block_table(h)
+        lib.lci_destroy_block_table(hf)
+
+
+def test_device_status_names_timeouts():
+    assert binding.STATUS_NAMES[6] == "LCI_ERR_TIMEOUT"
+    text = open(HEADER).read()
+    assert "reserved" not in text.split("LCI_ERR_TIMEOUT = 6", 1)[1].split("\n", 1)[0]

@@ -8,6 +8,8 @@ scratch array, which keeps the previous call's contents. This file sorts last
 so that a run stopping at the first failure has already run every other test.
 """
 import ctypes
+import os
+import re
 
 import pytest
 import torch
@@ -17,7 +19,19 @@ from long_context_indexer_b200.workloads import CONFIGS, generate
 
 pytestmark = pytest.mark.gpu
 
-NOALLOC_BYTES = 8 << 20  # LCI_NOALLOC_SCRATCH_BYTES in include/lci.h
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "lci.h")
+
+
+def _scratch_limit():
+    """LCI_NOALLOC_SCRATCH_BYTES as the public header defines it."""
+    m = re.search(r"#define\s+LCI_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)",
+                  open(HEADER).read())
+    assert m, "LCI_NOALLOC_SCRATCH_BYTES not found in the header"
+    return int(m.group(1)) << int(m.group(2))
+
+
+NOALLOC_BYTES = _scratch_limit()
 
 
 def _inputs(cfg):
@@ -48,6 +62,39 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
         ref, got = _both(cfg)
         assert torch.equal(got, ref), cfg
         assert (got >= 0).any()
+
+
+def test_noalloc_binding_with_prefill_phase_matches_tensor_core_schedule():
+    """The Python wrapper, with phase='prefill' on a shape the tensor-core
+    schedule takes: the allocation-free call runs the row-wise kernel and must
+    still give the tensor-core schedule's block ids."""
+    cfg = CONFIGS["prefill"].replace(S=512, ctx=4096, q_start=4096 - 512, topk=32)
+    d = _inputs(cfg)
+    ref = lci.index_select(d["q_c"], d["k_c"], cfg.bs, d["ctx_len"], d["q_start"], cfg.topk,
+                           phase="prefill")
+    for _ in range(2):
+        got = lci.index_select_noalloc(d["q_c"], d["k_c"], cfg.bs, d["ctx_len"], d["q_start"],
+                                       cfg.topk, phase="prefill")
+        torch.cuda.synchronize()
+        lci.get_device_status()
+        assert torch.equal(got, ref)
+    with pytest.raises(TypeError):
+        lci.index_select_noalloc(d["q_c"], d["k_c"].float(), cfg.bs, d["ctx_len"], d["q_start"],
+                                 cfg.topk)
+
+
+def test_noalloc_accepts_every_size_within_its_scratch():
+    """The largest batch whose decode-schedule workspace fits the built-in
+    scratch is accepted; that workspace size bounds what the call needs."""
+    # narrow block keys (H_i*d_c = 8) keep the inputs small next to the scratch
+    cfg = CONFIGS["decode"].replace(H_i=1, d_c=8)
+    B = 1
+    while lci.index_select_workspace_size(B + 1, 1, cfg.H_i, cfg.d_c, cfg.NB, cfg.topk,
+                                          "decode") <= NOALLOC_BYTES:
+        B += 1
+    big = cfg.replace(B=B, spare_pages=0)
+    ref, got = _both(big)
+    assert torch.equal(got, ref)
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
