@@ -168,6 +168,59 @@ LCI_API lci_status lci_index_select(const void* q_c, const void* k_c, lci_dtype 
                             size_t workspace_bytes, void* stream);
 
 /*
+ * A0 online, over a paged pool ([GPU-stack] "Adapting Sparse Attention": the
+ * representation-generation stage; [GPU-stack] "Reorganizing KV Cache
+ * Layout": block-level caching shared between prefill and decode). The block
+ * keys live beside the KV pages, one per page, addressed through the same
+ * block table:
+ *   kc     [num_pages][H_i][d_c], dtype   (the key of the block held by a page)
+ *   kc_sum [num_pages][H_i*d_c] fp32      (running sum of the block's tokens)
+ * T new tokens of every sequence b, at positions d_start[b] .. d_start[b]+T-1,
+ * enter the cache with indexer keys k_idx [batch][T][H_i][d_c] (device,
+ * dtype). Every block they touch, at page table[b][block], gets
+ *   kc_sum[page] = (the block's earlier tokens' sum if it already held tokens
+ *                   before d_start[b], else 0) + the new tokens' sum
+ *   kc[page]     = kc_sum[page] / (tokens of the block now present)
+ * (fp32 sums, the quotient formed in fp64 and rounded once to dtype). T = 1
+ * is the decode step; a chunk of T tokens is prefill. After any sequence of
+ * calls that fills positions 0..n-1 in order, kc equals lci_block_compress of
+ * those n tokens (exactly, for inputs whose fp32 sums are exact, such as
+ * multiples of 1/16 of magnitude <= 2 in blocks of up to 2^17 tokens).
+ * A block index >= max_blocks or a page outside [0, num_pages) is skipped and
+ * sets the device status word. Calls for the same sequence must be in order.
+ */
+LCI_API lci_status lci_kc_update(const void* k_idx, lci_dtype dtype, int32_t batch, int32_t T,
+                                 int32_t H_i, int32_t d_c, const int32_t* d_start,
+                                 const lci_block_table* table, float* kc_sum, void* kc,
+                                 void* stream);
+
+/*
+ * Workspace bytes lci_index_select_paged needs for these sizes.
+ */
+LCI_API lci_status lci_index_select_paged_workspace_size(int32_t batch, int32_t S, int32_t H_i,
+                                                         int32_t d_c, int32_t topk,
+                                                         const lci_block_table* table,
+                                                         lci_dtype dtype, lci_phase phase,
+                                                         size_t* bytes);
+
+/*
+ * lci_index_select with the block keys read from the paged pool kc
+ * [num_pages][H_i][d_c] through the block table: block j of sequence b is
+ * scored with kc[table[b][j]] (nb_max and block_size are the table's). Same
+ * results as lci_index_select on the gathered dense keys. The decode schedule
+ * reads each block's key at its page directly; the tensor-core prefill
+ * schedule first gathers the keys of cached blocks into the workspace.
+ * Workspace: lci_index_select_paged_workspace_size bytes, 256-byte aligned,
+ * with lci_index_select's zero-fill rule.
+ */
+LCI_API lci_status lci_index_select_paged(const void* q_c, const void* kc, lci_dtype dtype,
+                                          int32_t batch, int32_t S, int32_t H_i, int32_t d_c,
+                                          const lci_block_table* table, const int32_t* d_ctx_len,
+                                          const int32_t* d_q_start, int32_t topk, lci_phase phase,
+                                          int32_t* d_ids, void* workspace, size_t workspace_bytes,
+                                          void* stream);
+
+/*
  * Workspace bytes lci_sparse_attn needs for these sizes (0 is possible).
  */
 LCI_API lci_status lci_sparse_attn_workspace_size(int32_t batch, int32_t S, int32_t H_q, int32_t topk,

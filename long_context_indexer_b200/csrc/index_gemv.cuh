@@ -41,7 +41,8 @@ __global__ void __launch_bounds__(NT) index_gemv_select_kernel(
     const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ q_start, int topk,
     int chunk_blocks, int nchunks, float* __restrict__ scores,
     uint32_t* __restrict__ chunk_max, unsigned int* __restrict__ counters,
-    int32_t* __restrict__ ids, unsigned int* __restrict__ ready) {
+    int32_t* __restrict__ ids, unsigned int* __restrict__ ready,
+    const int32_t* __restrict__ page_table, int num_pages) {
     // Dynamic shared memory: [k_c chunk: chunk_blocks * K * sizeof(T)]
     // [query row: K floats, only when KV == 0]; the last CTA of a row reuses it
     // for the select's scratch.
@@ -84,13 +85,27 @@ __global__ void __launch_bounds__(NT) index_gemv_select_kernel(
         if (tid == 0) {
             mbar_init(&bar, 1);
             fence_mbar_init();
-            // The chunk's block keys are one contiguous range of k_c.
             const uint32_t bytes = (uint32_t)((j1 - j0) * row_bytes);
-            const unsigned char* src =
-                reinterpret_cast<const unsigned char*>(k_c + ((size_t)b * nb_max + j0) * K);
             mbar_arrive_expect_tx(&bar, bytes);
-            for (uint32_t off = 0; off < bytes; off += 16384u)
-                bulk_load(tile + off, src + off, min(16384u, bytes - off), &bar);
+            if (page_table == nullptr) {
+                // The chunk's block keys are one contiguous range of k_c.
+                const unsigned char* src =
+                    reinterpret_cast<const unsigned char*>(k_c + ((size_t)b * nb_max + j0) * K);
+                for (uint32_t off = 0; off < bytes; off += 16384u)
+                    bulk_load(tile + off, src + off, min(16384u, bytes - off), &bar);
+            } else {
+                // Paged block keys: one row per block, at the block's page.
+                for (int j = j0; j < j1; ++j) {
+                    int page = page_table[(size_t)b * nb_max + j];
+                    if (page < 0 || page >= num_pages) {
+                        raise_status(kStatusBadPage);
+                        page = 0;  // keep the copy in bounds; the result is flagged
+                    }
+                    bulk_load(tile + (size_t)(j - j0) * row_bytes,
+                              reinterpret_cast<const unsigned char*>(k_c + (size_t)page * K),
+                              (uint32_t)row_bytes, &bar);
+                }
+            }
         }
         const T* qrow = q_c + (size_t)row * K;
         if constexpr (KV > 0) {

@@ -16,6 +16,7 @@
 
 #include "../../include/lci.h"
 #include "attn_decode.cuh"
+#include "attn_prefill.cuh"
 #include "attn_simt.cuh"
 #include "common.cuh"
 #include "compress.cuh"
@@ -136,7 +137,8 @@ template <typename T>
 lci_status launch_index_gemv(const void* q_c, const void* k_c, int32_t batch, int32_t S, int32_t K,
                              int32_t bs, int32_t nb_max, const int32_t* ctx_len,
                              const int32_t* q_start, int32_t topk, int32_t* ids, void* ws,
-                             const IndexPlan& pl, cudaStream_t st, unsigned int* ready = nullptr) {
+                             const IndexPlan& pl, cudaStream_t st, unsigned int* ready = nullptr,
+                             const int32_t* page_table = nullptr, int32_t num_pages = 0) {
     constexpr int KV = 2048 / (16 * 32);
     auto kern = pl.qreg ? lci::index_gemv_select_kernel<T, kIndexThreads, KV>
                         : lci::index_gemv_select_kernel<T, kIndexThreads, 0>;
@@ -163,7 +165,7 @@ lci_status launch_index_gemv(const void* q_c, const void* k_c, int32_t batch, in
         static_cast<const T*>(q_c), static_cast<const T*>(k_c), S, K, nb_max, bs, ctx_len, q_start,
         topk, pl.chunk_blocks, pl.nchunks, reinterpret_cast<float*>(w + pl.off_scores),
         reinterpret_cast<uint32_t*>(w + pl.off_chunk_max),
-        reinterpret_cast<unsigned int*>(w + pl.off_counters), ids, ready);
+        reinterpret_cast<unsigned int*>(w + pl.off_counters), ids, ready, page_table, num_pages);
     return check_launch("index_select");
 }
 
@@ -418,6 +420,50 @@ lci_status launch_attn_decode(const void* q, int32_t batch, int32_t S, int32_t H
     return check_launch("sparse_attn");
 }
 
+// The tensor-core prefill schedule (attn_prefill.cuh): the decode kernel's
+// shape limits, 4, 8 or 16 query heads per KV head (32, 16 or 8 queries per
+// 128-row tile), at most 16384 blocks per sequence and 1024 selected blocks per
+// tile.
+bool prefill_attn_fits(const lci_block_table* t, int32_t H_q, int32_t topk, const void* k_pool,
+                       const void* v_pool) {
+    if (!decode_kernel_fits(t, H_q, k_pool, v_pool)) return false;
+    const int G = H_q / t->num_kv_heads;
+    return (G == 4 || G == 8 || G == 16) && t->max_blocks <= 32 * lci::pfa::kMaxWords &&
+           (long long)(lci::pfa::kRows / G) * topk <= lci::pfa::kMaxUnion;
+}
+
+lci_status launch_attn_prefill(const void* q, int32_t batch, int32_t S, int32_t H_q,
+                               const void* k_pool, const void* v_pool, const lci_block_table* t,
+                               const int32_t* ids, int32_t topk, const int32_t* ctx_len,
+                               const int32_t* q_start, float scale, void* out, cudaStream_t st) {
+    const long long rows = (long long)t->num_pages * t->num_kv_heads * t->block_size;
+    CUtensorMap tm_k, tm_v;
+    lci_status s = encode_pool_map(&tm_k, k_pool, rows);
+    if (s != LCI_OK) return s;
+    s = encode_pool_map(&tm_v, v_pool, rows);
+    if (s != LCI_OK) return s;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(lci::sparse_attn_prefill_kernel,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        lci::pfa::kSmemBytes);
+    });
+    if (attr_err != cudaSuccess)
+        return fail(LCI_ERR_CUDA, "sparse_attn: %s", cudaGetErrorString(attr_err));
+    const int G = H_q / t->num_kv_heads;
+    const int QT = lci::pfa::kRows / G;
+    const int q_tiles = (S + QT - 1) / QT;
+    const long long tiles = (long long)batch * q_tiles * t->num_kv_heads;
+    if (tiles >= (1ll << 31)) return fail(LCI_ERR_UNSUPPORTED, "sparse_attn: grid too large");
+    const float scale_log2 = scale * 1.4426950408889634f;
+    lci::sparse_attn_prefill_kernel<<<(unsigned)tiles, lci::pfa::kThreads, lci::pfa::kSmemBytes, st>>>(
+        tm_k, tm_v, static_cast<const __nv_bfloat16*>(q), t->d_table, t->max_blocks, t->num_pages,
+        t->num_kv_heads, t->block_size, S, H_q, ids, topk, ctx_len, q_start, scale_log2,
+        static_cast<__nv_bfloat16*>(out), q_tiles);
+    return check_launch("sparse_attn");
+}
+
 __global__ void validate_table_kernel(const int32_t* __restrict__ table, long long n,
                                       int num_pages) {
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
@@ -555,6 +601,130 @@ lci_status lci_index_select(const void* q_c, const void* k_c, lci_dtype dtype, i
                                             d_q_start, topk, d_ids, workspace, pl, cs);
 }
 
+// ---- paged block keys (online producer, paged index selection) ----
+
+lci_status lci_kc_update(const void* k_idx, lci_dtype dtype, int32_t batch, int32_t T, int32_t H_i,
+                         int32_t d_c, const int32_t* d_start, const lci_block_table* table,
+                         float* kc_sum, void* kc, void* stream) {
+    if (!k_idx || !d_start || !table || !kc_sum || !kc)
+        return fail(LCI_ERR_INVALID_ARG, "kc_update: null pointer argument");
+    if (batch <= 0 || T <= 0 || H_i <= 0 || d_c <= 0)
+        return fail(LCI_ERR_INVALID_ARG, "kc_update: sizes must be positive");
+    if (!dtype_ok(dtype)) return fail(LCI_ERR_INVALID_ARG, "kc_update: unknown dtype");
+    if (batch > table->batch)
+        return fail(LCI_ERR_INVALID_ARG, "kc_update: batch %d exceeds the table's %d", batch,
+                    table->batch);
+    const long long HD = (long long)H_i * d_c;
+    const long long slots = ((long long)T + table->block_size - 1) / table->block_size + 1;
+    const long long total = (long long)batch * slots * HD;
+    const int threads = 256;
+    const long long want = (total + threads - 1) / threads;
+    const int blocks = (int)(want < 148 * 16 ? want : 148 * 16);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dtype == LCI_F32)
+        lci::kc_update_kernel<float><<<blocks, threads, 0, st>>>(
+            static_cast<const float*>(k_idx), batch, T, (int)HD, table->block_size, d_start,
+            table->d_table, table->max_blocks, table->num_pages, (int)slots, kc_sum,
+            static_cast<float*>(kc));
+    else
+        lci::kc_update_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(k_idx), batch, T, (int)HD, table->block_size, d_start,
+            table->d_table, table->max_blocks, table->num_pages, (int)slots, kc_sum,
+            static_cast<__nv_bfloat16*>(kc));
+    return check_launch("kc_update");
+}
+
+namespace {
+struct PagedPlan {
+    bool tc;             // tensor-core schedule over a dense gather of the keys
+    size_t off_dense;    // [batch][nb_max][K] gathered keys (tc only)
+    size_t off_rest;     // the schedule's own workspace
+    size_t bytes;
+    PrefillPlan pp;
+    IndexPlan ip;
+};
+
+PagedPlan plan_paged(lci_dtype dtype, int32_t batch, int32_t S, int32_t K, int32_t nb_max,
+                     int32_t topk, lci_phase phase, const void* q_c, const void* kc) {
+    PagedPlan pl{};
+    pl.tc = prefill_path(dtype, phase, S, K, topk, q_c, kc);
+    pl.ip = plan_index(batch, S, K, nb_max, dtype_size(dtype));
+    if (pl.tc) {
+        pl.pp = plan_prefill(batch, S, K, nb_max, topk);
+        pl.off_dense = 0;
+        pl.off_rest = align_up((size_t)batch * nb_max * K * dtype_size(dtype));
+        pl.bytes = pl.off_rest + pl.pp.bytes;
+    } else {
+        pl.off_rest = 0;
+        pl.bytes = pl.ip.bytes;
+    }
+    return pl;
+}
+}  // namespace
+
+lci_status lci_index_select_paged_workspace_size(int32_t batch, int32_t S, int32_t H_i,
+                                                 int32_t d_c, int32_t topk,
+                                                 const lci_block_table* table, lci_dtype dtype,
+                                                 lci_phase phase, size_t* bytes) {
+    if (!bytes || !table)
+        return fail(LCI_ERR_INVALID_ARG, "index_select_paged_workspace_size: null argument");
+    lci_status st = check_index_args(batch, S, H_i, d_c, table->max_blocks, topk, dtype);
+    if (st != LCI_OK) return st;
+    *bytes = plan_paged(dtype, batch, S, H_i * d_c, table->max_blocks, topk, phase, nullptr,
+                        nullptr).bytes;
+    return ok();
+}
+
+lci_status lci_index_select_paged(const void* q_c, const void* kc, lci_dtype dtype, int32_t batch,
+                                  int32_t S, int32_t H_i, int32_t d_c,
+                                  const lci_block_table* table, const int32_t* d_ctx_len,
+                                  const int32_t* d_q_start, int32_t topk, lci_phase phase,
+                                  int32_t* d_ids, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+    if (!q_c || !kc || !table || !d_ctx_len || !d_q_start || !d_ids)
+        return fail(LCI_ERR_INVALID_ARG, "index_select_paged: null pointer argument");
+    const int32_t nb_max = table->max_blocks;
+    lci_status st = check_index_args(batch, S, H_i, d_c, nb_max, topk, dtype);
+    if (st != LCI_OK) return st;
+    if (batch > table->batch)
+        return fail(LCI_ERR_INVALID_ARG, "index_select_paged: batch %d exceeds the table's %d",
+                    batch, table->batch);
+    if (phase != LCI_PHASE_AUTO && phase != LCI_PHASE_PREFILL && phase != LCI_PHASE_DECODE)
+        return fail(LCI_ERR_INVALID_ARG, "index_select_paged: unknown phase %d", (int)phase);
+    if (!aligned16(q_c) || !aligned16(kc))
+        return fail(LCI_ERR_INVALID_ARG, "index_select_paged: q_c and kc must be 16-byte aligned");
+    const int K = H_i * d_c;
+    const PagedPlan pl = plan_paged(dtype, batch, S, K, nb_max, topk, phase, q_c, kc);
+    if (!workspace || workspace_bytes < pl.bytes ||
+        (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+        return fail(LCI_ERR_WORKSPACE, "index_select_paged: workspace needs %zu bytes, 256-byte "
+                    "aligned (got %zu at %p)", pl.bytes, workspace_bytes, workspace);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    char* w = static_cast<char*>(workspace);
+    if (pl.tc) {
+        // gather the visible blocks' keys through the table, then the dense
+        // tensor-core schedule
+        const int vec = (int)(K * dtype_size(dtype) / 16);
+        const long long total = (long long)batch * nb_max * vec;
+        const long long want = (total + 255) / 256;
+        const int blocks = (int)(want < 148 * 16 ? want : 148 * 16);
+        lci::kc_gather_kernel<<<blocks, 256, 0, cs>>>(
+            static_cast<const uint4*>(kc), table->d_table, d_ctx_len, batch, nb_max,
+            table->block_size, table->num_pages, vec, reinterpret_cast<uint4*>(w + pl.off_dense));
+        st = check_launch("index_select_paged");
+        if (st != LCI_OK) return st;
+        return launch_index_prefill(q_c, w + pl.off_dense, batch, S, K, table->block_size, nb_max,
+                                    d_ctx_len, d_q_start, topk, d_ids, w + pl.off_rest, pl.pp, cs);
+    }
+    if (dtype == LCI_F32)
+        return launch_index_gemv<float>(q_c, kc, batch, S, K, table->block_size, nb_max, d_ctx_len,
+                                        d_q_start, topk, d_ids, w + pl.off_rest, pl.ip, cs, nullptr,
+                                        table->d_table, table->num_pages);
+    return launch_index_gemv<__nv_bfloat16>(q_c, kc, batch, S, K, table->block_size, nb_max,
+                                            d_ctx_len, d_q_start, topk, d_ids, w + pl.off_rest,
+                                            pl.ip, cs, nullptr, table->d_table, table->num_pages);
+}
+
 lci_status lci_sparse_attn_workspace_size(int32_t batch, int32_t S, int32_t H_q, int32_t topk,
                                           const lci_block_table* table, lci_phase phase,
                                           size_t* bytes) {
@@ -582,6 +752,11 @@ lci_status lci_sparse_attn(const void* q, int32_t batch, int32_t S, int32_t H_q,
     (void)workspace;
     (void)workspace_bytes;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    // many queries per sequence: the tensor-core tile schedule
+    const bool many = phase == LCI_PHASE_PREFILL || (phase == LCI_PHASE_AUTO && S >= 16);
+    if (many && prefill_attn_fits(table, H_q, topk, k_pool, v_pool))
+        return launch_attn_prefill(q, batch, S, H_q, k_pool, v_pool, table, d_ids, topk, d_ctx_len,
+                                   d_q_start, scale, out, cs);
     if (decode_kernel_fits(table, H_q, k_pool, v_pool))
         return launch_attn_decode(q, batch, S, H_q, k_pool, v_pool, table, d_ids, topk, d_ctx_len,
                                   d_q_start, scale, out, cs);

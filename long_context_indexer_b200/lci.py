@@ -56,6 +56,11 @@ SIGNATURES = {
     "lci_sparse_attn_pipelined": (_st, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp,
                                         _f32, _vp, _vp, _vp]),
     "lci_set_wait_limit_ns": (_st, [ctypes.c_uint64]),
+    "lci_kc_update": (_st, [_vp, _st, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
+    "lci_index_select_paged_workspace_size": (_st, [_i32, _i32, _i32, _i32, _i32, _vp, _st, _st,
+                                                    ctypes.POINTER(_sz)]),
+    "lci_index_select_paged": (_st, [_vp, _vp, _st, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _i32,
+                                     _st, _vp, _vp, _sz, _vp]),
     "lci_get_wait_limit_ns": (_st, [ctypes.POINTER(ctypes.c_uint64)]),
 }
 
@@ -339,6 +344,57 @@ def sparse_decode(q_c: torch.Tensor, k_c: torch.Tensor, ctx_len: torch.Tensor,
         _dev(ws, "workspace"), ws.numel() * ws.element_size(), _stream(stream)),
         "lci_sparse_decode")
     return ids, out
+
+
+class PagedKeys:
+    """Block keys stored per page of a paged KV cache (one key per page), with
+    the fp32 running sums the online producer extends."""
+
+    def __init__(self, num_pages: int, H_i: int, d_c: int, dtype: torch.dtype, device):
+        self.kc = torch.zeros((num_pages, H_i, d_c), dtype=dtype, device=device)
+        self.kc_sum = torch.zeros((num_pages, H_i * d_c), dtype=torch.float32, device=device)
+
+    def update(self, k_idx: torch.Tensor, start: torch.Tensor, table: BlockTable,
+               stream=None) -> None:
+        """Append k_idx [B, T, H_i, d_c] at positions start[b] .. start[b]+T-1."""
+        B, T, H_i, d_c = k_idx.shape
+        if k_idx.dtype != self.kc.dtype or tuple(self.kc.shape[1:]) != (H_i, d_c):
+            raise ValueError("lci: k_idx must match the paged keys' dtype and [H_i, d_c]")
+        if self.kc.shape[0] != table.num_pages:
+            raise ValueError("lci: paged keys and block table differ in page count")
+        _check(load_library().lci_kc_update(
+            _dev(k_idx, "k_idx", None, 4), _dtype_code(k_idx), B, T, H_i, d_c,
+            _dev(start, "start", torch.int32, 1), table.handle, _dev(self.kc_sum, "kc_sum"),
+            _dev(self.kc, "kc"), _stream(stream)), "lci_kc_update")
+
+
+def index_select_paged(q_c: torch.Tensor, keys: "PagedKeys", table: BlockTable,
+                       ctx_len: torch.Tensor, q_start: torch.Tensor, topk: int,
+                       phase: str = "auto", ids: Optional[torch.Tensor] = None,
+                       ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """index_select with block keys read from the paged pool through the table."""
+    B, S, H_i, d_c = q_c.shape
+    kc = keys.kc if isinstance(keys, PagedKeys) else keys
+    if kc.dtype != q_c.dtype or tuple(kc.shape[1:]) != (H_i, d_c):
+        raise ValueError("lci: paged keys must be [num_pages, H_i, d_c] with q_c's dtype")
+    if ids is None:
+        ids = torch.empty((B, S, topk), dtype=torch.int32, device=q_c.device)
+    lib = load_library()
+    n = ctypes.c_size_t()
+    _check(lib.lci_index_select_paged_workspace_size(B, S, H_i, d_c, topk, table.handle,
+                                                     _dtype_code(q_c), PHASES[phase],
+                                                     ctypes.byref(n)),
+           "lci_index_select_paged_workspace_size")
+    if ws is None:
+        ws = workspace(q_c.device, n.value,
+                       f"index_select_paged:{B}x{S}x{table.max_blocks}:{H_i * d_c}:{phase}")
+    _check(lib.lci_index_select_paged(
+        _dev(q_c, "q_c", None, 4), _dev(kc, "kc", q_c.dtype, 3), _dtype_code(q_c), B, S, H_i, d_c,
+        table.handle, _dev(ctx_len, "ctx_len", torch.int32, 1),
+        _dev(q_start, "q_start", torch.int32, 1), topk, PHASES[phase],
+        _dev(ids, "ids", torch.int32, 3), _dev(ws, "workspace"), ws.numel() * ws.element_size(),
+        _stream(stream)), "lci_index_select_paged")
+    return ids
 
 
 def sparse_attn_pipelined(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,

@@ -208,3 +208,44 @@ def test_device_status_names_timeouts():
     assert binding.STATUS_NAMES[6] == "LCI_ERR_TIMEOUT"
     text = open(HEADER).read()
     assert "reserved" not in text.split("LCI_ERR_TIMEOUT = 6", 1)[1].split("\n", 1)[0]
+
+
+def test_paged_key_entry_points_host_checks(lib):
+    h = ctypes.c_void_p()
+    # bf16 table: 2 sequences x 8 blocks of 64 tokens, 20 pages
+    assert lib.lci_create_block_table(FAKE, 2, 8, 20, 64, 1, 128, 1, ctypes.byref(h)) == 0
+    try:
+        upd = lambda **kw: lib.lci_kc_update(  # noqa: E731
+            kw.get("k", FAKE), kw.get("dtype", 1), kw.get("B", 2), kw.get("T", 1), 8, 128,
+            kw.get("start", FAKE), kw.get("t", h), kw.get("sum", FAKE), kw.get("kc", FAKE), None)
+        assert upd(k=None) == INVALID
+        assert upd(t=None) == INVALID
+        assert upd(sum=None) == INVALID
+        assert upd(T=0) == INVALID
+        assert upd(B=3) == INVALID          # more sequences than the table
+        assert upd(dtype=5) == INVALID
+        n = ctypes.c_size_t()
+        assert lib.lci_index_select_paged_workspace_size(2, 1, 8, 128, 32, h, 1, 0,
+                                                         ctypes.byref(n)) == 0
+        assert n.value > 0
+        assert lib.lci_index_select_paged_workspace_size(2, 1, 8, 128, 32, None, 1, 0,
+                                                         ctypes.byref(n)) == INVALID
+
+        def sel(**kw):
+            a = dict(q_c=FAKE, kc=FAKE, dtype=1, B=2, S=1, H_i=8, d_c=128, t=h, ctx=FAKE, q0=FAKE,
+                     topk=32, phase=0, ids=FAKE, ws=FAKE, ws_bytes=n.value)
+            a.update(kw)
+            return lib.lci_index_select_paged(a["q_c"], a["kc"], a["dtype"], a["B"], a["S"],
+                                              a["H_i"], a["d_c"], a["t"], a["ctx"], a["q0"],
+                                              a["topk"], a["phase"], a["ids"], a["ws"],
+                                              a["ws_bytes"], None)
+        assert sel(kc=None) == INVALID
+        assert sel(t=None) == INVALID
+        assert sel(B=3) == INVALID
+        assert sel(phase=7) == INVALID
+        assert sel(topk=300) == UNSUPPORTED
+        assert sel(kc=ctypes.c_void_p(FAKE.value + 8)) == INVALID
+        assert sel(ws=None) == WORKSPACE
+        assert sel(ws_bytes=n.value - 1) == WORKSPACE
+    finally:
+        lib.lci_destroy_block_table(h)

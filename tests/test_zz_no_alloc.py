@@ -78,7 +78,7 @@ def test_noalloc_binding_with_prefill_phase_matches_tensor_core_schedule():
         torch.cuda.synchronize()
         lci.get_device_status()
         assert torch.equal(got, ref)
-    with pytest.raises(TypeError):
+    with pytest.raises(ValueError):  # the wrapper checks dtypes before any call
         lci.index_select_noalloc(d["q_c"], d["k_c"].float(), cfg.bs, d["ctx_len"], d["q_start"],
                                  cfg.topk)
 
