@@ -255,6 +255,80 @@ LCI_API lci_status lci_sparse_attn(const void* q, int32_t batch, int32_t S, int3
                            void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Context parallelism: one long context split into block ranges over several
+ * GPUs ([AI-acc] §3: communication libraries for multi-card inference;
+ * [Hetero] §VII: communication overlap). Each rank holds the block keys and
+ * KV pages of its range [j_lo, j_hi) and runs the steps below; the caller
+ * exchanges the small per-query results between ranks (an all-gather).
+ *
+ * 1. lci_index_select on the rank's keys with positions shifted by -j_lo*bs
+ *    (q_start - j_lo*bs, ctx_len - j_lo*bs): the rank's local top-k.
+ *    lci_ids_shift(lo=0, hi=j_hi-j_lo, offset=+j_lo) makes the ids global and
+ *    lci_block_scores_at gives their scores.
+ * 2. After gathering every rank's (scores, ids), lci_topk_merge yields the
+ *    global top-k, identical on every rank and equal to the one-GPU result:
+ *    the global top-k lies in the union of the local ones.
+ * 3. lci_ids_shift(lo=j_lo, hi=j_hi, offset=-j_lo) keeps the selected blocks
+ *    the rank holds; lci_sparse_attn_partial attends over them and returns the
+ *    normalised output and its log-sum-exp.
+ * 4. After gathering every rank's (out, lse), lci_attn_merge combines them.
+ */
+
+/*
+ * scores[b][s][i] = sum_h sum_d q_c[b][s][h][d] * k_c[b][ids[b][s][i]][h][d]
+ * (fp32), -inf where the id is -1. Layouts as lci_index_select; d_scores
+ * [batch][S][topk] float, device (output). An id outside [-1, nb_max) is
+ * scored -inf and sets the device status word.
+ */
+LCI_API lci_status lci_block_scores_at(const void* q_c, const void* k_c, lci_dtype dtype,
+                                       int32_t batch, int32_t S, int32_t H_i, int32_t d_c,
+                                       int32_t nb_max, const int32_t* d_ids, int32_t topk,
+                                       float* d_scores, void* stream);
+
+/*
+ * d_out[i] = (lo <= d_ids[i] < hi) ? d_ids[i] + offset : -1 for i < n
+ * (device arrays of int32; in place is allowed).
+ */
+LCI_API lci_status lci_ids_shift(const int32_t* d_ids, int64_t n, int32_t lo, int32_t hi,
+                                 int32_t offset, int32_t* d_out, void* stream);
+
+/*
+ * Top-k of nlists ranked lists per row. d_scores, d_ids [nlists][rows][topk]
+ * (device): list r of a row holds block ids in rank order (score descending,
+ * id ascending), ended by -1. d_out [rows][topk] int32 (device): the best topk
+ * ids of the union by the same order, -1 padded. nlists <= 64.
+ */
+LCI_API lci_status lci_topk_merge(const float* d_scores, const int32_t* d_ids, int32_t nlists,
+                                  int64_t rows, int32_t topk, int32_t* d_out, void* stream);
+
+/*
+ * lci_sparse_attn that also returns, per query row and head, the log2 of the
+ * sum of 2^(scale*log2(e)*q.k) over the attended tokens (the log-sum-exp of
+ * the scaled logits in base 2): d_lse [batch][S][H_q] float (device), -inf
+ * where no token is attended (the output row is then zero). Supported shape:
+ * bf16 pools, head_dim 128, block_size a multiple of 64, at most 16 query
+ * heads per KV head (else LCI_ERR_UNSUPPORTED). Needs no workspace.
+ */
+LCI_API lci_status lci_sparse_attn_partial(const void* q, int32_t batch, int32_t S, int32_t H_q,
+                                           const void* k_pool, const void* v_pool,
+                                           const lci_block_table* table, const int32_t* d_ids,
+                                           int32_t topk, const int32_t* d_ctx_len,
+                                           const int32_t* d_q_start, float scale, lci_phase phase,
+                                           void* out, float* d_lse, void* stream);
+
+/*
+ * Exact combination of nlists partial attention results:
+ *   out[x][:] = sum_r w_r o[r][x][:] / sum_r w_r,  w_r = 2^(lse[r][x] - max_r lse[r][x])
+ * for every (row, head) x; zero where every lse is -inf.
+ *   d_o   [nlists][rows_heads][head_dim], dtype (device)
+ *   d_lse [nlists][rows_heads] float (device)
+ *   d_out [rows_heads][head_dim], dtype (device, output)
+ */
+LCI_API lci_status lci_attn_merge(const void* d_o, const float* d_lse, lci_dtype dtype,
+                                  int32_t nlists, int64_t rows_heads, int32_t head_dim,
+                                  void* d_out, void* stream);
+
+/*
  * lci_index_select without any device allocation. The reference pages have no
  * counterpart; this entry point exists for callers that are not allowed to
  * allocate device memory or to hold a workspace of their own: for example code

@@ -64,7 +64,8 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
     const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ table, int nb_max,
     int num_pages, int H_kv, int bs, int S, int H_q, const int32_t* __restrict__ ids, int topk,
     const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ q_start, float scale_log2,
-    __nv_bfloat16* __restrict__ out, int nsplit, const unsigned int* __restrict__ ready) {
+    __nv_bfloat16* __restrict__ out, int nsplit, const unsigned int* __restrict__ ready,
+    float* __restrict__ lse) {
     using namespace dec;
     namespace cg = cooperative_groups;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -356,6 +357,9 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
         }
         cm[tid] = M;
         cl[tid] = L;
+        // log2-sum-exp2 of the scaled logits, for combining partial results
+        if (lse != nullptr && nsplit == 1 && tid < G)
+            lse[(size_t)row * H_q + (size_t)g * G + tid] = L > 0.f ? M + log2f(L) : -INFINITY;
     }
     __syncthreads();
     __nv_bfloat16* orow = out + ((size_t)row * H_q + (size_t)g * G) * kHD;
@@ -397,6 +401,8 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
             if (c < nsplit) L += f * cluster.map_shared_rank(cl, c)[tid];
         }
         xl[tid] = L > 0.f ? 1.f / L : 0.f;
+        if (lse != nullptr && split == 0 && tid < G)
+            lse[(size_t)row * H_q + (size_t)g * G + tid] = L > 0.f ? M + log2f(L) : -INFINITY;
     }
     __syncthreads();
     const int chunk = (kElems + nsplit - 1) / nsplit;

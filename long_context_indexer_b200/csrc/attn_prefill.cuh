@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
     const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ table, int nb_max,
     int num_pages, int H_kv, int bs, int S, int H_q, const int32_t* __restrict__ ids, int topk,
     const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ q_start, float scale_log2,
-    __nv_bfloat16* __restrict__ out, int q_tiles) {
+    __nv_bfloat16* __restrict__ out, int q_tiles, float* __restrict__ lse) {
     using namespace pfa;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -507,6 +507,10 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
             tc_fence_after();
         }
         const float inv = l > 0.f ? 1.f / l : 0.f;
+        // log2-sum-exp2 of the scaled logits, for combining partial results
+        if (lse != nullptr && s < S)
+            lse[((size_t)b * S + s) * H_q + (size_t)g * G + (r - qi * G)] =
+                l > 0.f ? m_ref + log2f(l) : -INFINITY;
         __nv_bfloat16* orow = out + (((size_t)b * S + s) * H_q + (size_t)g * G + (r - qi * G)) * kHD;
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {

@@ -20,6 +20,7 @@
 #include "attn_simt.cuh"
 #include "common.cuh"
 #include "compress.cuh"
+#include "cp_merge.cuh"
 #include "index_gemv.cuh"
 #include "index_prefill.cuh"
 #include "topk_select.cuh"
@@ -372,7 +373,8 @@ lci_status launch_attn_decode(const void* q, int32_t batch, int32_t S, int32_t H
                               const void* k_pool, const void* v_pool, const lci_block_table* t,
                               const int32_t* ids, int32_t topk, const int32_t* ctx_len,
                               const int32_t* q_start, float scale, void* out, cudaStream_t st,
-                              const unsigned int* ready = nullptr, bool early_start = true) {
+                              const unsigned int* ready = nullptr, bool early_start = true,
+                              float* lse = nullptr) {
     const long long rows = (long long)t->num_pages * t->num_kv_heads * t->block_size;
     CUtensorMap tm_k, tm_v;
     lci_status s = encode_pool_map(&tm_k, k_pool, rows);
@@ -415,7 +417,7 @@ lci_status launch_attn_decode(const void* q, int32_t batch, int32_t S, int32_t H
     cudaError_t e = cudaLaunchKernelEx(
         &cfg, kern, tm_k, tm_v, static_cast<const __nv_bfloat16*>(q),
         t->d_table, t->max_blocks, t->num_pages, t->num_kv_heads, t->block_size, S, H_q, ids, topk,
-        ctx_len, q_start, scale_log2, static_cast<__nv_bfloat16*>(out), nsplit, ready);
+        ctx_len, q_start, scale_log2, static_cast<__nv_bfloat16*>(out), nsplit, ready, lse);
     if (e != cudaSuccess) return fail(LCI_ERR_CUDA, "sparse_attn: %s", cudaGetErrorString(e));
     return check_launch("sparse_attn");
 }
@@ -435,7 +437,8 @@ bool prefill_attn_fits(const lci_block_table* t, int32_t H_q, int32_t topk, cons
 lci_status launch_attn_prefill(const void* q, int32_t batch, int32_t S, int32_t H_q,
                                const void* k_pool, const void* v_pool, const lci_block_table* t,
                                const int32_t* ids, int32_t topk, const int32_t* ctx_len,
-                               const int32_t* q_start, float scale, void* out, cudaStream_t st) {
+                               const int32_t* q_start, float scale, void* out, cudaStream_t st,
+                               float* lse = nullptr) {
     const long long rows = (long long)t->num_pages * t->num_kv_heads * t->block_size;
     CUtensorMap tm_k, tm_v;
     lci_status s = encode_pool_map(&tm_k, k_pool, rows);
@@ -460,7 +463,7 @@ lci_status launch_attn_prefill(const void* q, int32_t batch, int32_t S, int32_t 
     lci::sparse_attn_prefill_kernel<<<(unsigned)tiles, lci::pfa::kThreads, lci::pfa::kSmemBytes, st>>>(
         tm_k, tm_v, static_cast<const __nv_bfloat16*>(q), t->d_table, t->max_blocks, t->num_pages,
         t->num_kv_heads, t->block_size, S, H_q, ids, topk, ctx_len, q_start, scale_log2,
-        static_cast<__nv_bfloat16*>(out), q_tiles);
+        static_cast<__nv_bfloat16*>(out), q_tiles, lse);
     return check_launch("sparse_attn");
 }
 
@@ -765,6 +768,108 @@ lci_status lci_sparse_attn(const void* q, int32_t batch, int32_t S, int32_t H_q,
                                        d_ctx_len, d_q_start, scale, out, cs);
     return launch_attn_simt<__nv_bfloat16>(q, batch, S, H_q, k_pool, v_pool, table, d_ids, topk,
                                            d_ctx_len, d_q_start, scale, out, cs);
+}
+
+// ---- context parallelism: partial results and their exact combination ----
+
+lci_status lci_sparse_attn_partial(const void* q, int32_t batch, int32_t S, int32_t H_q,
+                                   const void* k_pool, const void* v_pool,
+                                   const lci_block_table* table, const int32_t* d_ids,
+                                   int32_t topk, const int32_t* d_ctx_len,
+                                   const int32_t* d_q_start, float scale, lci_phase phase,
+                                   void* out, float* lse, void* stream) {
+    if (!q || !k_pool || !v_pool || !d_ids || !d_ctx_len || !d_q_start || !out || !lse)
+        return fail(LCI_ERR_INVALID_ARG, "sparse_attn_partial: null pointer argument");
+    lci_status st = check_attn_args(batch, S, H_q, table, topk);
+    if (st != LCI_OK) return st;
+    if (phase != LCI_PHASE_AUTO && phase != LCI_PHASE_PREFILL && phase != LCI_PHASE_DECODE)
+        return fail(LCI_ERR_INVALID_ARG, "sparse_attn_partial: unknown phase %d", (int)phase);
+    if (!decode_kernel_fits(table, H_q, k_pool, v_pool))
+        return fail(LCI_ERR_UNSUPPORTED, "sparse_attn_partial: needs bf16 pools, head_dim 128, "
+                    "block_size a multiple of 64, at most 16 query heads per KV head and "
+                    "16-byte aligned pools");
+    if (!(scale > 0.f)) scale = 1.0f / std::sqrt((float)table->head_dim);
+    if (!std::isfinite(scale)) return fail(LCI_ERR_INVALID_ARG, "sparse_attn_partial: non-finite scale");
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const bool many = phase == LCI_PHASE_PREFILL || (phase == LCI_PHASE_AUTO && S >= 16);
+    if (many && prefill_attn_fits(table, H_q, topk, k_pool, v_pool))
+        return launch_attn_prefill(q, batch, S, H_q, k_pool, v_pool, table, d_ids, topk, d_ctx_len,
+                                   d_q_start, scale, out, cs, lse);
+    return launch_attn_decode(q, batch, S, H_q, k_pool, v_pool, table, d_ids, topk, d_ctx_len,
+                              d_q_start, scale, out, cs, nullptr, true, lse);
+}
+
+lci_status lci_block_scores_at(const void* q_c, const void* k_c, lci_dtype dtype, int32_t batch,
+                               int32_t S, int32_t H_i, int32_t d_c, int32_t nb_max,
+                               const int32_t* d_ids, int32_t topk, float* d_scores, void* stream) {
+    if (!q_c || !k_c || !d_ids || !d_scores)
+        return fail(LCI_ERR_INVALID_ARG, "block_scores_at: null pointer argument");
+    lci_status st = check_index_args(batch, S, H_i, d_c, nb_max, topk, dtype);
+    if (st != LCI_OK) return st;
+    if (!aligned16(q_c) || !aligned16(k_c))
+        return fail(LCI_ERR_INVALID_ARG, "block_scores_at: q_c and k_c must be 16-byte aligned");
+    const long long pairs = (long long)batch * S * topk;
+    const long long want = (pairs + 7) / 8;  // 8 warps per CTA
+    const int blocks = (int)(want < 148 * 32 ? want : 148 * 32);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const int K = H_i * d_c;
+    if (dtype == LCI_F32)
+        lci::block_scores_at_kernel<float><<<blocks, 256, 0, cs>>>(
+            static_cast<const float*>(q_c), static_cast<const float*>(k_c), S, K, nb_max, d_ids,
+            topk, pairs, d_scores);
+    else
+        lci::block_scores_at_kernel<__nv_bfloat16><<<blocks, 256, 0, cs>>>(
+            static_cast<const __nv_bfloat16*>(q_c), static_cast<const __nv_bfloat16*>(k_c), S, K,
+            nb_max, d_ids, topk, pairs, d_scores);
+    return check_launch("block_scores_at");
+}
+
+lci_status lci_ids_shift(const int32_t* d_ids, int64_t n, int32_t lo, int32_t hi, int32_t offset,
+                         int32_t* d_out, void* stream) {
+    if (!d_ids || !d_out) return fail(LCI_ERR_INVALID_ARG, "ids_shift: null pointer argument");
+    if (n < 0) return fail(LCI_ERR_INVALID_ARG, "ids_shift: negative count");
+    if (n == 0) return ok();
+    const long long want = (n + 255) / 256;
+    const int blocks = (int)(want < 148 * 16 ? want : 148 * 16);
+    lci::ids_shift_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(d_ids, n, lo, hi,
+                                                                                 offset, d_out);
+    return check_launch("ids_shift");
+}
+
+lci_status lci_topk_merge(const float* d_scores, const int32_t* d_ids, int32_t nlists, int64_t rows,
+                          int32_t topk, int32_t* d_out, void* stream) {
+    if (!d_scores || !d_ids || !d_out)
+        return fail(LCI_ERR_INVALID_ARG, "topk_merge: null pointer argument");
+    if (nlists <= 0 || rows <= 0 || topk <= 0)
+        return fail(LCI_ERR_INVALID_ARG, "topk_merge: sizes must be positive");
+    if (nlists > lci::kMaxLists)
+        return fail(LCI_ERR_UNSUPPORTED, "topk_merge: %d lists above %d", nlists, lci::kMaxLists);
+    const long long blocks = (rows + 127) / 128;
+    if (blocks >= (1ll << 31)) return fail(LCI_ERR_UNSUPPORTED, "topk_merge: too many rows");
+    lci::topk_merge_kernel<<<(unsigned)blocks, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+        d_scores, d_ids, nlists, rows, topk, d_out);
+    return check_launch("topk_merge");
+}
+
+lci_status lci_attn_merge(const void* d_o, const float* d_lse, lci_dtype dtype, int32_t nlists,
+                          int64_t rows_heads, int32_t head_dim, void* d_out, void* stream) {
+    if (!d_o || !d_lse || !d_out) return fail(LCI_ERR_INVALID_ARG, "attn_merge: null pointer argument");
+    if (nlists <= 0 || rows_heads <= 0 || head_dim <= 0)
+        return fail(LCI_ERR_INVALID_ARG, "attn_merge: sizes must be positive");
+    if (!dtype_ok(dtype)) return fail(LCI_ERR_INVALID_ARG, "attn_merge: unknown dtype");
+    const long long total = rows_heads * head_dim;
+    const long long want = (total + 255) / 256;
+    const int blocks = (int)(want < 148 * 16 ? want : 148 * 16);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (dtype == LCI_F32)
+        lci::attn_merge_kernel<float><<<blocks, 256, 0, cs>>>(
+            static_cast<const float*>(d_o), d_lse, nlists, rows_heads, head_dim,
+            static_cast<float*>(d_out));
+    else
+        lci::attn_merge_kernel<__nv_bfloat16><<<blocks, 256, 0, cs>>>(
+            static_cast<const __nv_bfloat16*>(d_o), d_lse, nlists, rows_heads, head_dim,
+            static_cast<__nv_bfloat16*>(d_out));
+    return check_launch("attn_merge");
 }
 
 }  // extern "C"

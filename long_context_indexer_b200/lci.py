@@ -56,6 +56,13 @@ SIGNATURES = {
     "lci_sparse_attn_pipelined": (_st, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp,
                                         _f32, _vp, _vp, _vp]),
     "lci_set_wait_limit_ns": (_st, [ctypes.c_uint64]),
+    "lci_block_scores_at": (_st, [_vp, _vp, _st, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _vp,
+                                  _vp]),
+    "lci_ids_shift": (_st, [_vp, ctypes.c_int64, _i32, _i32, _i32, _vp, _vp]),
+    "lci_topk_merge": (_st, [_vp, _vp, _i32, ctypes.c_int64, _i32, _vp, _vp]),
+    "lci_sparse_attn_partial": (_st, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp,
+                                      _f32, _st, _vp, _vp, _vp]),
+    "lci_attn_merge": (_st, [_vp, _vp, _st, _i32, ctypes.c_int64, _i32, _vp, _vp]),
     "lci_kc_update": (_st, [_vp, _st, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "lci_index_select_paged_workspace_size": (_st, [_i32, _i32, _i32, _i32, _i32, _vp, _st, _st,
                                                     ctypes.POINTER(_sz)]),
@@ -395,6 +402,87 @@ def index_select_paged(q_c: torch.Tensor, keys: "PagedKeys", table: BlockTable,
         _dev(ids, "ids", torch.int32, 3), _dev(ws, "workspace"), ws.numel() * ws.element_size(),
         _stream(stream)), "lci_index_select_paged")
     return ids
+
+
+def block_scores_at(q_c: torch.Tensor, k_c: torch.Tensor, ids: torch.Tensor,
+                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """scores [B, S, topk] fp32 of the given block ids (-inf for -1)."""
+    B, S, H_i, d_c = q_c.shape
+    topk = ids.shape[-1]
+    if tuple(ids.shape) != (B, S, topk):
+        raise ValueError("lci: ids must be [B, S, topk]")
+    if out is None:
+        out = torch.empty((B, S, topk), dtype=torch.float32, device=q_c.device)
+    _check(load_library().lci_block_scores_at(
+        _dev(q_c, "q_c", None, 4), _dev(k_c, "k_c", q_c.dtype, 4), _dtype_code(q_c), B, S, H_i, d_c,
+        k_c.shape[1], _dev(ids, "ids", torch.int32, 3), topk, _dev(out, "scores", torch.float32, 3),
+        _stream(stream)), "lci_block_scores_at")
+    return out
+
+
+def ids_shift(ids: torch.Tensor, lo: int, hi: int, offset: int,
+              out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """(lo <= id < hi) ? id + offset : -1, elementwise."""
+    if out is None:
+        out = torch.empty_like(ids)
+    _check(load_library().lci_ids_shift(_dev(ids, "ids", torch.int32), ids.numel(), int(lo),
+                                        int(hi), int(offset), _dev(out, "out", torch.int32),
+                                        _stream(stream)), "lci_ids_shift")
+    return out
+
+
+def topk_merge(scores: torch.Tensor, ids: torch.Tensor, out: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    """Merge [L, ..., topk] ranked lists into the top-k [..., topk] of their union."""
+    L, topk = ids.shape[0], ids.shape[-1]
+    if scores.shape != ids.shape:
+        raise ValueError("lci: scores and ids must have the same shape")
+    rows = ids[0].numel() // topk
+    if out is None:
+        out = torch.empty(ids.shape[1:], dtype=torch.int32, device=ids.device)
+    _check(load_library().lci_topk_merge(_dev(scores, "scores", torch.float32),
+                                         _dev(ids, "ids", torch.int32), L, rows, topk,
+                                         _dev(out, "out", torch.int32), _stream(stream)),
+           "lci_topk_merge")
+    return out
+
+
+def sparse_attn_partial(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                        table: BlockTable, ids: torch.Tensor, ctx_len: torch.Tensor,
+                        q_start: torch.Tensor, scale: float = 0.0, phase: str = "auto",
+                        out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                        stream=None):
+    """sparse_attn plus the base-2 log-sum-exp [B, S, H_q] of each row's logits."""
+    B, S, H_q, hd = q.shape
+    topk = ids.shape[-1]
+    if tuple(ids.shape) != (B, S, topk):
+        raise ValueError("lci: ids must be [B, S, topk]")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, S, H_q), dtype=torch.float32, device=q.device)
+    _check(load_library().lci_sparse_attn_partial(
+        _dev(q, "q", table.dtype, 4), B, S, H_q, _dev(k_pool, "k_pool", table.dtype),
+        _dev(v_pool, "v_pool", table.dtype), table.handle, _dev(ids, "ids", torch.int32, 3), topk,
+        _dev(ctx_len, "ctx_len", torch.int32, 1), _dev(q_start, "q_start", torch.int32, 1),
+        float(scale), PHASES[phase], _dev(out, "out", q.dtype, 4),
+        _dev(lse, "lse", torch.float32, 3), _stream(stream)), "lci_sparse_attn_partial")
+    return out, lse
+
+
+def attn_merge(o: torch.Tensor, lse: torch.Tensor, out: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    """Combine partials o [L, ..., hd] with lse [L, ...] into out [..., hd]."""
+    L, hd = o.shape[0], o.shape[-1]
+    if tuple(lse.shape) != tuple(o.shape[:-1]):
+        raise ValueError("lci: lse must be o's shape without the last dim")
+    if out is None:
+        out = torch.empty(o.shape[1:], dtype=o.dtype, device=o.device)
+    _check(load_library().lci_attn_merge(_dev(o, "o", None), _dev(lse, "lse", torch.float32),
+                                         _dtype_code(o), L, lse[0].numel(), hd,
+                                         _dev(out, "out", o.dtype), _stream(stream)),
+           "lci_attn_merge")
+    return out
 
 
 def sparse_attn_pipelined(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,

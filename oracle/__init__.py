@@ -57,6 +57,9 @@ def _load():
         for f in (lib.orc_block_compress, lib.orc_block_scores, lib.orc_index_select,
                   lib.orc_sparse_attn, lib.orc_dense_masked):
             f.restype = ctypes.c_int
+        lib.orc_gated_state_scan.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, i64, i64, i64,
+                                             i64, i64, i64, vp]
+        lib.orc_gated_state_scan.restype = ctypes.c_int
         lib.orc_num_threads.restype = ctypes.c_int
         lib.orc_set_num_threads.argtypes = [ctypes.c_int]
         _lib = lib
@@ -188,3 +191,27 @@ def dense_masked(q, k_pool, v_pool, block_table, ids, ctx_len, q_start, scale, r
     """Full causal attention with non-selected positions masked to -inf. [nrows,H_q,hd] fp64."""
     return _attn(_load().orc_dense_masked, q, k_pool, v_pool, block_table, ids, ctx_len,
                  q_start, scale, rows)
+
+
+def gated_state_scan(q, k, v, gate, state, C):
+    """N4: chunked gated state scan. q, k [B,T,H,dk], v [B,T,H,dv], gate
+    [B,H,nchunks], state [B,H,dk,dv]. Returns (out [B,T,H,dv], final state)
+    in fp64; the input state is not modified."""
+    q, k, v = _cpu(q), _cpu(k), _cpu(v)
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("oracle: q, k and v must share a dtype")
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    if tuple(k.shape) != (B, T, H, dk) or tuple(v.shape[:3]) != (B, T, H):
+        raise ValueError("oracle: q, k, v shapes disagree")
+    nchunks = (T + C - 1) // C
+    gate = _cpu(gate).to(torch.float64).contiguous()
+    if tuple(gate.shape) != (B, H, nchunks):
+        raise ValueError("oracle: gate must be [B, H, nchunks]")
+    st = _cpu(state).to(torch.float64).clone().contiguous()
+    if tuple(st.shape) != (B, H, dk, dv):
+        raise ValueError("oracle: state must be [B, H, dk, dv]")
+    out = torch.empty((B, T, H, dv), dtype=torch.float64)
+    _check(_load().orc_gated_state_scan(_ptr(q), _ptr(k), _ptr(v), _dt(q), _ptr(gate), _ptr(st),
+                                        B, T, H, dk, dv, C, _ptr(out)), "gated_state_scan")
+    return out, st

@@ -24,6 +24,8 @@
  *                           id asc), padded with -1 (same page, section 4.1;
  *                           the score/top-k/mask combination of page 1's
  *                           section "Operatorizing Index Selection").
+ *   N4  gated state scan    the chunked gated state update and readout of the
+ *                           linear-attention family (orc_gated_state_scan below).
  *   A3+A4 sparse attention  exact softmax attention of each query head over the
  *                           tokens of the selected blocks only, gathered from a
  *                           paged KV pool through a block table (page 2 section
@@ -371,5 +373,53 @@ int orc_dense_masked(const void* q, const void* k_pool, const void* v_pool, int 
         }
         free(logit);
     }
+    return nomem ? ORC_NOMEM : ORC_OK;
+}
+
+/*
+ * N4. Chunked gated state scan ("Day-0 Adaptation for Trillion-Parameter MoE
+ * Models", section III, the gated incremental state update of the linear
+ * attention family: the sequence is scanned in chunks of C tokens and a state
+ * matrix is carried from chunk to chunk). For every sequence b and head h, with
+ * the state S [dk][dv] starting at state[b][h] and chunk c holding tokens
+ * [c*C, min(T, (c+1)*C)):
+ *     S        = gate[b][h][c] * S + sum_{t in chunk c} k_t^T v_t
+ *     out[t]   = q_t S                       for every t in chunk c
+ * (the readout uses the state after the chunk's own update). On return
+ * state[b][h] holds the final S.
+ *   q, k [B][T][H][dk]; v [B][T][H][dv] (type dt); gate [B][H][nchunks];
+ *   state [B][H][dk][dv] (in/out); out [B][T][H][dv].
+ */
+int orc_gated_state_scan(const void* q, const void* k, const void* v, int dt, const double* gate,
+                         double* state, int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
+                         int64_t C, double* out) {
+    if (!q || !k || !v || !gate || !state || !out || B < 0 || T < 0 || H <= 0 || dk <= 0 ||
+        dv <= 0 || C <= 0)
+        return ORC_BAD_ARG;
+    const int64_t nchunks = (T + C - 1) / C;
+    int nomem = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t h = 0; h < H; ++h) {
+            double* S = state + (b * H + h) * dk * dv;
+            for (int64_t c = 0; c < nchunks; ++c) {
+                const int64_t t0 = c * C, t1 = (c + 1) * C < T ? (c + 1) * C : T;
+                const double g = gate[(b * H + h) * nchunks + c];
+                for (int64_t i = 0; i < dk * dv; ++i) S[i] *= g;
+                for (int64_t t = t0; t < t1; ++t)
+                    for (int64_t i = 0; i < dk; ++i) {
+                        const double ki = ld(k, dt, ((b * T + t) * H + h) * dk + i);
+                        for (int64_t j = 0; j < dv; ++j)
+                            S[i * dv + j] += ki * ld(v, dt, ((b * T + t) * H + h) * dv + j);
+                    }
+                for (int64_t t = t0; t < t1; ++t)
+                    for (int64_t j = 0; j < dv; ++j) {
+                        double acc = 0.0;
+                        for (int64_t i = 0; i < dk; ++i)
+                            acc += ld(q, dt, ((b * T + t) * H + h) * dk + i) * S[i * dv + j];
+                        out[((b * T + t) * H + h) * dv + j] = acc;
+                    }
+            }
+        }
     return nomem ? ORC_NOMEM : ORC_OK;
 }

@@ -57,6 +57,19 @@ MUTANTS = [
      "dot += ld(q, dt, (row * H_q + h) * hd + d) *\n                           ld(k_pool, dt, pool_off(tok_page[t], g, tok_slot[t], d, H_kv, bs, hd));",
      "dot += ld(q, dt, (b * H_q + h) * hd + d) *\n                           ld(k_pool, dt, pool_off(tok_page[t], g, tok_slot[t], d, H_kv, bs, hd));"),
     ("token slot off by one", "tok_slot[n] = u;", "tok_slot[n] = u > 0 ? u - 1 : 0;"),
+    ("state scan reads out before the chunk's update",
+     "                for (int64_t t = t0; t < t1; ++t)\n                    for (int64_t i = 0; i < dk; ++i) {\n                        const double ki",
+     "                for (int64_t t = t1; t < t1; ++t)\n                    for (int64_t i = 0; i < dk; ++i) {\n                        const double ki"),
+    ("state scan gate dropped", "for (int64_t i = 0; i < dk * dv; ++i) S[i] *= g;",
+     "for (int64_t i = 0; i < dk * dv; ++i) S[i] *= 1.0;"),
+    ("state scan k and v swapped in the update",
+     "S[i * dv + j] += ki * ld(v, dt, ((b * T + t) * H + h) * dv + j);",
+     "S[i * dv + j] += ki * ld(v, dt, ((b * T + t) * H + h) * dv + (j + i) % dv);"),
+    ("state scan gate index off by one chunk", "const double g = gate[(b * H + h) * nchunks + c];",
+     "const double g = gate[(b * H + h) * nchunks + (c > 0 ? c - 1 : 0)];"),
+    ("state scan chunk end ignores T",
+     "const int64_t t0 = c * C, t1 = (c + 1) * C < T ? (c + 1) * C : T;",
+     "const int64_t t0 = c * C, t1 = (c + 1) * C < T ? (c + 1) * C : T - 1;"),
 ]
 
 

@@ -386,3 +386,94 @@ def test_oracle_rejects_out_of_range_ids():
         oracle.sparse_attn(q, k_pool, v_pool, table, torch.tensor([[6, -1, -1]]), ctx, q0, 0.5)
     with pytest.raises(ValueError):
         oracle.sparse_attn(q, k_pool, v_pool, table, torch.tensor([[-2, -1, -1]]), ctx, q0, 0.5)
+
+
+# ---------------------------------------------------------------- N4 gated state scan
+# ("Day-0 Adaptation for Trillion-Parameter MoE Models", section III: the state
+# is scaled by the chunk's gate, extended by k^T v over the chunk, and read out
+# by q for every token of the chunk.)
+
+def _scan_inputs(B, T, H, dk, dv, C, seed, gate_lo=0.5):
+    g = _gen(seed)
+    q = torch.randn((B, T, H, dk), generator=g, dtype=torch.float64)
+    k = torch.randn((B, T, H, dk), generator=g, dtype=torch.float64)
+    v = torch.randn((B, T, H, dv), generator=g, dtype=torch.float64)
+    nchunks = (T + C - 1) // C
+    gate = gate_lo + (1 - gate_lo) * torch.rand((B, H, nchunks), generator=g, dtype=torch.float64)
+    s0 = torch.randn((B, H, dk, dv), generator=g, dtype=torch.float64)
+    return q, k, v, gate, s0
+
+
+def test_state_scan_token_chunks_equal_the_gated_recurrence_closed_form():
+    """C = 1: o_t = prod_{r<=t} g_r q_t S0 + sum_{s<=t} prod_{s<r<=t} g_r (q_t.k_s) v_s."""
+    B, T, H, dk, dv = 2, 9, 3, 4, 5
+    q, k, v, gate, s0 = _scan_inputs(B, T, H, dk, dv, 1, 31)
+    out, st = oracle.gated_state_scan(q, k, v, gate, s0, 1)
+    qn, kn, vn, gn, sn = (x.numpy() for x in (q, k, v, gate, s0))
+    for b in range(B):
+        for h in range(H):
+            g = gn[b, h]
+            for t in range(T):
+                dec0 = np.prod(g[: t + 1])
+                expect = dec0 * qn[b, t, h] @ sn[b, h]
+                for s in range(t + 1):
+                    expect = expect + np.prod(g[s + 1: t + 1]) * (qn[b, t, h] @ kn[b, s, h]) * vn[b, s, h]
+                np.testing.assert_allclose(out[b, t, h].numpy(), expect, rtol=1e-12, atol=1e-12)
+
+
+def test_state_scan_ungated_is_chunk_masked_linear_attention():
+    """gate = 1, S0 = 0: out = ((Q K^T) masked to s < end of t's chunk) V, by
+    matmul, with a partial last chunk and dk != dv."""
+    B, T, H, dk, dv, C = 1, 11, 2, 6, 3, 4
+    q, k, v, _, _ = _scan_inputs(B, T, H, dk, dv, C, 32)
+    nchunks = (T + C - 1) // C
+    out, _ = oracle.gated_state_scan(q, k, v, torch.ones((B, H, nchunks), dtype=torch.float64),
+                                     torch.zeros((B, H, dk, dv), dtype=torch.float64), C)
+    t = np.arange(T)
+    end = (t // C + 1) * C
+    mask = (t[None, :] < end[:, None]).astype(np.float64)       # [t, s]
+    for h in range(H):
+        qh, kh, vh = q[0, :, h].numpy(), k[0, :, h].numpy(), v[0, :, h].numpy()
+        expect = ((qh @ kh.T) * mask) @ vh
+        np.testing.assert_allclose(out[0, :, h].numpy(), expect, rtol=1e-12, atol=1e-12)
+
+
+def test_state_scan_final_state_closed_form_and_input_untouched():
+    """S_final = prod_c g_c S0 + sum_s prod_{c > chunk(s)} g_c k_s^T v_s."""
+    B, T, H, dk, dv, C = 2, 13, 2, 4, 3, 5
+    q, k, v, gate, s0 = _scan_inputs(B, T, H, dk, dv, C, 33)
+    s0_copy = s0.clone()
+    _, st = oracle.gated_state_scan(q, k, v, gate, s0, C)
+    assert torch.equal(s0, s0_copy)
+    gn = gate.numpy()
+    for b in range(B):
+        for h in range(H):
+            expect = np.prod(gn[b, h]) * s0[b, h].numpy()
+            for s in range(T):
+                c = s // C
+                expect = expect + np.prod(gn[b, h, c + 1:]) * np.outer(k[b, s, h].numpy(),
+                                                                        v[b, s, h].numpy())
+            np.testing.assert_allclose(st[b, h].numpy(), expect, rtol=1e-12, atol=1e-12)
+
+
+def test_state_scan_zero_gate_forgets_earlier_chunks():
+    """gate = 0: every chunk reads out q_t (K_c^T V_c) of its own chunk only."""
+    B, T, H, dk, dv, C = 1, 8, 1, 3, 4, 4
+    q, k, v, _, s0 = _scan_inputs(B, T, H, dk, dv, C, 34)
+    out, st = oracle.gated_state_scan(q, k, v, torch.zeros((B, H, 2), dtype=torch.float64), s0, C)
+    for c in range(2):
+        kc, vc = k[0, c * C:(c + 1) * C, 0].numpy(), v[0, c * C:(c + 1) * C, 0].numpy()
+        expect = q[0, c * C:(c + 1) * C, 0].numpy() @ (kc.T @ vc)
+        np.testing.assert_allclose(out[0, c * C:(c + 1) * C, 0].numpy(), expect, rtol=1e-12,
+                                   atol=1e-12)
+    np.testing.assert_allclose(st[0, 0].numpy(), k[0, 4:, 0].numpy().T @ v[0, 4:, 0].numpy(),
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_state_scan_bf16_inputs_are_widened_exactly():
+    B, T, H, dk, dv, C = 1, 6, 2, 8, 8, 3
+    q, k, v, gate, s0 = _scan_inputs(B, T, H, dk, dv, C, 35)
+    qb, kb, vb = (x.to(torch.bfloat16) for x in (q, k, v))
+    o1, s1 = oracle.gated_state_scan(qb, kb, vb, gate, s0, C)
+    o2, s2 = oracle.gated_state_scan(qb.double(), kb.double(), vb.double(), gate, s0, C)
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
