@@ -431,6 +431,30 @@ LCI_API lci_status lci_set_wait_limit_ns(uint64_t ns);
 LCI_API lci_status lci_get_wait_limit_ns(uint64_t* ns);
 
 /*
+ * N4 -- chunked gated state scan of the linear-attention family ([Hetero]
+ * §II: gated incremental state updates maintained across strides; §III: the
+ * state scanned over the sequence in chunks, updated by the gate and k^T v,
+ * read out by q). For every sequence b and head h, with S [dk][dv] starting
+ * at state_in[b][h] and chunk c holding tokens [c*chunk, min(T, (c+1)*chunk)):
+ *   S      = gate[b][h][c] * S + sum_{t in chunk c} k[b][t][h]^T v[b][t][h]
+ *   out[b][t][h] = q[b][t][h] S            for every t in chunk c
+ * (the readout sees the chunk's own update); state_out[b][h] = the final S.
+ *   q, k   [batch][T][H][dk], v [batch][T][H][dv], dtype (device)
+ *   d_gate [batch][H][ceil(T/chunk)] float (device)
+ *   d_state_in, d_state_out [batch][H][dk][dv] float (device; may be the same
+ *          array: the update is then in place)
+ *   d_out  [batch][T][H][dv] float (device, output)
+ * The state stays in fp32 in TMEM; the readout multiplies q by the state split
+ * into two bf16 parts (hi + lo, relative error about 2^-17). Supported: bf16,
+ * dk = dv = 128, chunk = 128 (else LCI_ERR_UNSUPPORTED).
+ */
+LCI_API lci_status lci_gated_state_scan(const void* q, const void* k, const void* v,
+                                        lci_dtype dtype, const float* d_gate,
+                                        const float* d_state_in, float* d_state_out,
+                                        int32_t batch, int32_t T, int32_t H, int32_t dk,
+                                        int32_t dv, int32_t chunk, float* d_out, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the sticky device status
  * word of the current device: LCI_OK; LCI_ERR_TIMEOUT when a bounded device
  * wait ran out since the last call; otherwise LCI_ERR_DEVICE_BOUNDS when a

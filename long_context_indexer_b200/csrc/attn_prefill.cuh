@@ -23,7 +23,8 @@
 // of once per query.
 //
 // Warps: 0 TMA producer (K and V rings, 128-byte swizzle), 1 MMA issuer (one
-// thread), 2..5 softmax: thread = TMEM lane = MMA row. The softmax is online
+// thread), 2..9 softmax: two threads per MMA row (TMEM lane), each taking one
+// 64-token unit of a stage and 64 of the output dims. The softmax is online
 // with a lazy rescale: a row's reference maximum m moves only when a stage's
 // maximum exceeds it by more than 8 (log2 units), so P <= 2^8 and O is
 // rescaled in TMEM only then (after the previous P V has completed). The
@@ -50,7 +51,8 @@ constexpr int kTileBytes = 2 * kHalf;  // 128 rows x 128 dims bf16: 32 KiB
 constexpr int kKStages = 2, kVStages = 2;
 constexpr int kMaxWords = 512;         // block bitmap words: nb_max <= 16384
 constexpr int kMaxUnion = 1024;        // distinct blocks per tile (QT * topk)
-constexpr int kThreads = 192;
+constexpr int kSoftWarps = 8;            // two threads per MMA row
+constexpr int kThreads = 64 + 32 * kSoftWarps;
 constexpr int kColO = 0, kColS = 128, kColP = 384, kTmemCols = 512;
 constexpr float kLazy = 8.0f;          // rescale when the maximum grows past m + 8
 // shared memory layout (offsets from a 1024-byte aligned base)
@@ -60,7 +62,10 @@ constexpr int kOffV = kOffK + kKStages * kTileBytes;
 constexpr int kOffUnion = kOffV + kVStages * kTileBytes;
 constexpr int kUnionBytes = 2 * kMaxWords * 4 + 3 * kMaxUnion * 4;
 constexpr int kOffBar = kOffUnion + kUnionBytes;
-constexpr int kSmemBytes = kOffBar + 256 + 1024 /*alignment slack*/;
+// exchange between a row's two threads: [3][2][128] floats (two stage buffers
+// of row maxima, then the row sums) and [2][2][128] ints (wait outcomes)
+constexpr int kOffXchg = kOffBar + 256;
+constexpr int kSmemBytes = kOffXchg + 3 * 2 * 128 * 4 + 2 * 2 * 128 * 4 + 1024 /*alignment slack*/;
 // instruction descriptors: D fp32, A and B bf16, M = 128, N = 128;
 // S = Q K^T with both operands K-major, O += P V with V (B) MN-major
 constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(128 >> 3) << 17) |
@@ -174,7 +179,7 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sfull[i], 1);
-            mbar_init(&pfull[i], 4);
+            mbar_init(&pfull[i], kSoftWarps);
         }
         mbar_init(obar, 1);
         mbar_init(ofin, 1);
@@ -263,13 +268,13 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
 
     // ---------------- Q tile -> shared memory (swizzled, K-major) ----------------
     if (warp >= 2) {
-        const int r = (warp & 3) * 32 + lane;
+        const int r = (warp & 3) * 32 + lane, hf = (warp - 2) >> 2;
         const int qi = r / G, s = s0 + qi;
         const uint4* src = reinterpret_cast<const uint4*>(
             q + (((size_t)b * S + s) * H_q + (size_t)g * G + (r - qi * G)) * kHD);
         unsigned char* qs = smem + kOffQ;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
+        for (int c = 8 * hf; c < 8 * hf + 8; ++c) {
             const uint4 v = s < S ? src[c] : make_uint4(0, 0, 0, 0);
             *reinterpret_cast<uint4*>(qs + pfa_off(r, c)) = v;
         }
@@ -383,117 +388,149 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
             mbar_wait(drain, 0);
         }
     } else {
-        // ---------------- softmax and epilogue: one MMA row per thread ----------------
+        // ---------------- softmax and epilogue: two threads per MMA row ----------------
+        // Thread (r, hf) owns row r's tokens of unit slot hf (stage columns
+        // 64*hf .. 64*hf+63) and output dims 64*hf .. 64*hf+63. The two halves
+        // of a row agree on its maximum through shared memory and a named
+        // barrier of their two warps (ids 1..4, one per TMEM lane quarter).
         const int quarter = warp & 3;
+        const int hf = (warp - 2) >> 2;
         const int r = quarter * 32 + lane;
+        const int bar_id = 1 + quarter;
         const int qi = r / G, s = s0 + qi;
         const long long p = (long long)q_start[b] + s;
         const long long last = s < S ? (p < ctx - 1 ? p : ctx - 1) : -1;
         const uint32_t qbit = 1u << qi;
         const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
-        float m_ref = -INFINITY;  // reference maximum (log2 units)
-        float l = 0.f;
+        float* xchg = reinterpret_cast<float*>(smem + kOffXchg);  // [3][2][128]
+        int* xok = reinterpret_cast<int*>(xchg + 3 * 2 * 128);      // [2][2][128]
+        float m_ref = -INFINITY;  // reference maximum (log2 units), the same in both halves
+        float l = 0.f;            // this half's share of the row sum
         for (int i = 0; i < nstages; ++i) {
-            // the stage's two units: first token and whether this row takes it
-            int t0[2];
-            bool take[2], absent[2];
-            for (int c = 0; c < 2; ++c) {
-                const int u = 2 * i + c;
-                t0[c] = 0;
-                take[c] = false;
-                absent[c] = true;
-                if (u < nunits) {
-                    const int blk = u / upb, sub = u - blk * upb;
-                    if (upage[blk] >= 0) {
-                        absent[c] = false;
-                        t0[c] = ublk[blk] * bs + sub * 64;
-                        take[c] = (umask[blk] & qbit) != 0u && (long long)t0[c] <= last;
+            // this half's unit: its first token, whether the row takes it, and
+            // how many of its 64 tokens the row may see
+            const int u = 2 * i + hf;
+            int t0 = 0, nval = 0;
+            if (u < nunits) {
+                const int blk = u / upb, sub = u - blk * upb;
+                if (upage[blk] >= 0) {
+                    t0 = ublk[blk] * bs + sub * 64;
+                    if ((umask[blk] & qbit) != 0u && (long long)t0 <= last) {
+                        const long long nv = last - t0 + 1;
+                        nval = nv < 64 ? (int)nv : 64;
                     }
                 }
             }
             const bool waited = mbar_wait(&sfull[i & 1], (i >> 1) & 1);
-            if (!__all_sync(0xffffffffu, waited && !*s_abort)) {  // warp-uniform exit
+            const int my_ok = waited && !*s_abort;
+            tc_fence_after();
+            uint32_t sv[2][32];
+            float mx = -INFINITY;
+            const bool warp_any = __any_sync(0xffffffffu, nval > 0);
+            if (warp_any) {
+                tmem_ld32(lane_addr + kColS + (i & 1) * 128 + hf * 64, sv[0]);
+                tmem_ld32(lane_addr + kColS + (i & 1) * 128 + hf * 64 + 32, sv[1]);
+                if (nval == 64) {
+#pragma unroll
+                    for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sv[ch][e]));
+                } else {
+#pragma unroll
+                    for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const bool ok = ch * 32 + e < nval;
+                            sv[ch][e] = ok ? sv[ch][e] : __float_as_uint(-INFINITY);
+                            mx = fmaxf(mx, __uint_as_float(sv[ch][e]));
+                        }
+                }
+            }
+            // the row maximum of the stage (raw scores; the scale is positive),
+            // and whether both halves may go on: one decision for the pair of
+            // warps, so their named barriers always match
+            float* xm = xchg + (i & 1) * 256;
+            int* xo = xok + (i & 1) * 256;
+            xm[hf * 128 + r] = mx;
+            xo[hf * 128 + r] = my_ok;
+            named_barrier_sync(bar_id, 64);
+            if (!__all_sync(0xffffffffu, my_ok && xo[(hf ^ 1) * 128 + r])) {
                 *s_abort = 1;
                 break;
             }
-            tc_fence_after();
-            uint32_t sv[4][32];
-            float mx = -INFINITY;
-            const bool warp_any = __any_sync(0xffffffffu, take[0] || take[1]);
-            if (warp_any) {
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch)
-                    tmem_ld32(lane_addr + kColS + (i & 1) * 128 + ch * 32, sv[ch]);
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    const int c = ch >> 1;
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const long long t = (long long)t0[c] + (ch & 1) * 32 + e;
-                        const bool ok = take[c] && t <= last;
-                        const float x = __uint_as_float(sv[ch][e]) * scale_log2;
-                        sv[ch][e] = __float_as_uint(ok ? x : -INFINITY);
-                        mx = fmaxf(mx, ok ? x : -INFINITY);
-                    }
-                }
-            }
+            const float mrow = fmaxf(mx, xm[(hf ^ 1) * 128 + r]) * scale_log2;
             // lazy reference: move m only when the stage's maximum passes m + 8
             float corr = 1.f;
-            if (mx > m_ref + kLazy) {
-                corr = l > 0.f ? exp2f(m_ref - mx) : 1.f;
-                m_ref = mx;
+            if (mrow > m_ref + kLazy) {
+                corr = m_ref > -INFINITY ? fast_exp2(m_ref - mrow) : 1.f;
+                m_ref = mrow;
             }
             if (__any_sync(0xffffffffu, corr != 1.f)) {
-                // O holds earlier stages of this row: rescale it once the
-                // previous P V has landed
+                // O holds earlier stages of this row: rescale this half's
+                // columns once the previous P V has landed
                 if (!mbar_wait(obar, (i - 1) & 1)) *s_abort = 1;
                 tc_fence_after();
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
+                for (int ch = 0; ch < 2; ++ch) {
                     uint32_t ov[32];
-                    tmem_ld32(lane_addr + kColO + ch * 32, ov);
+                    tmem_ld32(lane_addr + kColO + hf * 64 + ch * 32, ov);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
-                    tmem_st32(lane_addr + kColO + ch * 32, ov);
+                    tmem_st32(lane_addr + kColO + hf * 64 + ch * 32, ov);
                 }
                 l *= corr;
             }
-            // P = exp2(x - m) as bf16 pairs into this stage's P buffer
-            float lsum = 0.f;
+            // P = 2^(s*c - m) as bf16 pairs into this stage's P buffer
+            const float neg_m = -m_ref;
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
+            for (int ch = 0; ch < 2; ++ch) {
                 uint32_t pk[16];
+                if (nval > 0) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    float a = 0.f, bb = 0.f;
-                    if (warp_any) {
-                        // masked entries hold -inf (m_ref may be -inf too)
-                        const float xa = __uint_as_float(sv[ch][2 * e]);
-                        const float xb = __uint_as_float(sv[ch][2 * e + 1]);
-                        a = xa == -INFINITY ? 0.f : exp2f(xa - m_ref);
-                        bb = xb == -INFINITY ? 0.f : exp2f(xb - m_ref);
+                    for (int e = 0; e < 16; ++e) {
+                        // masked entries hold -inf: 2^-inf = 0
+                        const float a = fast_exp2(fmaf(__uint_as_float(sv[ch][2 * e]), scale_log2, neg_m));
+                        const float bb = fast_exp2(fmaf(__uint_as_float(sv[ch][2 * e + 1]), scale_log2, neg_m));
+                        l += a + bb;
+                        pk[e] = pack_bf16x2(a, bb);
                     }
-                    lsum += a + bb;
-                    pk[e] = pack_bf16x2(a, bb);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = 0u;
                 }
-                tmem_st16(lane_addr + kColP + (i & 1) * 64 + ch * 16, pk);
+                tmem_st16(lane_addr + kColP + (i & 1) * 64 + hf * 32 + ch * 16, pk);
             }
-            l += lsum;
             tmem_wait_st();
-            // V rows of absent units and of tokens past the context length
-            // must be zero before the P V MMA reads them
-            const bool tail = absent[0] || absent[1] || (long long)t0[0] + 64 > ctx ||
-                              (long long)t0[1] + 64 > ctx;
-            if (tail) {
+            // V rows of an absent unit and of tokens past the context length
+            // must be zero before the P V MMA reads them (this thread: token row
+            // r of the stage, dims 64*hf .. 64*hf+63)
+            bool v_absent[2];
+            long long v_t0[2];
+            bool stage_tail = false;  // the same for every thread
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const int uv = 2 * i + c;
+                v_absent[c] = true;
+                v_t0[c] = 0;
+                if (uv < nunits) {
+                    const int blk = uv / upb, sub = uv - blk * upb;
+                    if (upage[blk] >= 0) {
+                        v_absent[c] = false;
+                        v_t0[c] = (long long)ublk[blk] * bs + sub * 64;
+                    }
+                }
+                stage_tail = stage_tail || v_absent[c] || v_t0[c] + 64 > ctx;
+            }
+            if (stage_tail) {
                 const int vs = i % kVStages;
                 if (!mbar_wait(&vfull[vs], (i / kVStages) & 1)) *s_abort = 1;
-                const int c = r >> 6;
-                const long long t = (long long)t0[c] + (r & 63);
-                if (absent[c] || t >= ctx) {
-                    unsigned char* vrow = smem + kOffV + vs * kTileBytes;
+                const bool mine_absent = (r >> 6) ? v_absent[1] : v_absent[0];
+                const long long mine_t0 = (r >> 6) ? v_t0[1] : v_t0[0];
+                if (mine_absent || mine_t0 + (r & 63) >= ctx) {
+                    unsigned char* vt = smem + kOffV + vs * kTileBytes;
 #pragma unroll
-                    for (int cc = 0; cc < 16; ++cc)
-                        *reinterpret_cast<uint4*>(vrow + pfa_off(r, cc)) = make_uint4(0, 0, 0, 0);
+                    for (int cc = 8 * hf; cc < 8 * hf + 8; ++cc)
+                        *reinterpret_cast<uint4*>(vt + pfa_off(r, cc)) = make_uint4(0, 0, 0, 0);
                 }
                 fence_proxy_async_smem();
             }
@@ -502,21 +539,25 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
             if (lane == 0) mbar_arrive(&pfull[i & 1]);
         }
         // ---------------- epilogue: O / l -> bf16 ----------------
+        float* xl = xchg + 2 * 256;
+        xl[hf * 128 + r] = l;
+        named_barrier_sync(bar_id, 64);
+        const float ltot = l + xl[(hf ^ 1) * 128 + r];
         if (nstages > 0 && !*s_abort) {
             if (!mbar_wait(ofin, 0)) *s_abort = 1;
             tc_fence_after();
         }
-        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
         // log2-sum-exp2 of the scaled logits, for combining partial results
-        if (lse != nullptr && s < S)
+        if (lse != nullptr && s < S && hf == 0)
             lse[((size_t)b * S + s) * H_q + (size_t)g * G + (r - qi * G)] =
-                l > 0.f ? m_ref + log2f(l) : -INFINITY;
+                ltot > 0.f ? m_ref + __log2f(ltot) : -INFINITY;
         __nv_bfloat16* orow = out + (((size_t)b * S + s) * H_q + (size_t)g * G + (r - qi * G)) * kHD;
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int ch = 0; ch < 2; ++ch) {
             uint32_t ov[32];
             if (nstages > 0) {
-                tmem_ld32(lane_addr + kColO + ch * 32, ov);
+                tmem_ld32(lane_addr + kColO + hf * 64 + ch * 32, ov);
             } else {
 #pragma unroll
                 for (int e = 0; e < 32; ++e) ov[e] = 0u;
@@ -527,7 +568,7 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
                 for (int e = 0; e < 16; ++e)
                     pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv,
                                         __uint_as_float(ov[2 * e + 1]) * inv);
-                uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+                uint4* dst = reinterpret_cast<uint4*>(orow + hf * 64 + ch * 32);
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
                     dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);

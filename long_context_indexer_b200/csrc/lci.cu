@@ -23,12 +23,19 @@
 #include "cp_merge.cuh"
 #include "index_gemv.cuh"
 #include "index_prefill.cuh"
+#include "state_scan.cuh"
 #include "topk_select.cuh"
 
 struct lci_block_table {
     const int32_t* d_table;
     int32_t batch, max_blocks, num_pages, block_size, num_kv_heads, head_dim;
     lci_dtype dtype;
+    // TMA descriptors of the last pool pair the table was used with: a decode
+    // loop calls with the same pools every step, so they are encoded once
+    std::mutex map_mu;
+    const void* map_k_pool = nullptr;
+    const void* map_v_pool = nullptr;
+    CUtensorMap map_k, map_v;
 };
 
 namespace {
@@ -240,6 +247,29 @@ lci_status encode_pool_map(CUtensorMap* map, const void* pool, long long rows) {
     return LCI_OK;
 }
 
+// The pools' tensor maps, from the table's cache when the pools are the ones
+// it last saw.
+lci_status pool_maps(const lci_block_table* t, const void* k_pool, const void* v_pool,
+                     CUtensorMap* tm_k, CUtensorMap* tm_v) {
+    lci_block_table* mt = const_cast<lci_block_table*>(t);
+    std::lock_guard<std::mutex> lock(mt->map_mu);
+    if (mt->map_k_pool != k_pool || mt->map_v_pool != v_pool) {
+        const long long rows = (long long)t->num_pages * t->num_kv_heads * t->block_size;
+        lci_status s = encode_pool_map(&mt->map_k, k_pool, rows);
+        if (s != LCI_OK) return s;
+        s = encode_pool_map(&mt->map_v, v_pool, rows);
+        if (s != LCI_OK) {
+            mt->map_k_pool = mt->map_v_pool = nullptr;
+            return s;
+        }
+        mt->map_k_pool = k_pool;
+        mt->map_v_pool = v_pool;
+    }
+    *tm_k = mt->map_k;
+    *tm_v = mt->map_v;
+    return LCI_OK;
+}
+
 // Tensor-core schedule for many queries per sequence (index_prefill.cuh).
 struct PrefillPlan {
     int m_tiles, n_split, kt, ksteps;
@@ -375,11 +405,8 @@ lci_status launch_attn_decode(const void* q, int32_t batch, int32_t S, int32_t H
                               const int32_t* q_start, float scale, void* out, cudaStream_t st,
                               const unsigned int* ready = nullptr, bool early_start = true,
                               float* lse = nullptr) {
-    const long long rows = (long long)t->num_pages * t->num_kv_heads * t->block_size;
     CUtensorMap tm_k, tm_v;
-    lci_status s = encode_pool_map(&tm_k, k_pool, rows);
-    if (s != LCI_OK) return s;
-    s = encode_pool_map(&tm_v, v_pool, rows);
+    lci_status s = pool_maps(t, k_pool, v_pool, &tm_k, &tm_v);
     if (s != LCI_OK) return s;
     const long long pairs = (long long)batch * S * t->num_kv_heads;
     const int units = topk * (t->block_size / 64);
@@ -434,16 +461,26 @@ bool prefill_attn_fits(const lci_block_table* t, int32_t H_q, int32_t topk, cons
            (long long)(lci::pfa::kRows / G) * topk <= lci::pfa::kMaxUnion;
 }
 
+// Which attention kernel a call runs: the tensor-core tile schedule when asked
+// for (LCI_PHASE_PREFILL) and it fits, or, under LCI_PHASE_AUTO, for many
+// queries per sequence whose selections are likely to share blocks (at most
+// four times as many blocks as a tile's queries select in all); otherwise the
+// one-row-at-a-time kernel, which gathers each query's blocks on its own.
+bool use_prefill_attn(const lci_block_table* t, int32_t S, int32_t H_q, int32_t topk,
+                      lci_phase phase, const void* k_pool, const void* v_pool) {
+    if (phase == LCI_PHASE_DECODE || !prefill_attn_fits(t, H_q, topk, k_pool, v_pool)) return false;
+    if (phase == LCI_PHASE_PREFILL) return true;
+    const int QT = lci::pfa::kRows / (H_q / t->num_kv_heads);
+    return S >= 16 && (long long)t->max_blocks <= 4ll * QT * topk;
+}
+
 lci_status launch_attn_prefill(const void* q, int32_t batch, int32_t S, int32_t H_q,
                                const void* k_pool, const void* v_pool, const lci_block_table* t,
                                const int32_t* ids, int32_t topk, const int32_t* ctx_len,
                                const int32_t* q_start, float scale, void* out, cudaStream_t st,
                                float* lse = nullptr) {
-    const long long rows = (long long)t->num_pages * t->num_kv_heads * t->block_size;
     CUtensorMap tm_k, tm_v;
-    lci_status s = encode_pool_map(&tm_k, k_pool, rows);
-    if (s != LCI_OK) return s;
-    s = encode_pool_map(&tm_v, v_pool, rows);
+    lci_status s = pool_maps(t, k_pool, v_pool, &tm_k, &tm_v);
     if (s != LCI_OK) return s;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
@@ -509,8 +546,14 @@ lci_status lci_create_block_table(const int32_t* d_table, int32_t batch, int32_t
     if (!dtype_ok(kv_dtype)) return fail(LCI_ERR_INVALID_ARG, "create_block_table: unknown dtype");
     lci_block_table* t = new (std::nothrow) lci_block_table;
     if (!t) return fail(LCI_ERR_INVALID_ARG, "create_block_table: host allocation failed");
-    *t = lci_block_table{d_table, batch, max_blocks, num_pages, block_size, num_kv_heads, head_dim,
-                         kv_dtype};
+    t->d_table = d_table;
+    t->batch = batch;
+    t->max_blocks = max_blocks;
+    t->num_pages = num_pages;
+    t->block_size = block_size;
+    t->num_kv_heads = num_kv_heads;
+    t->head_dim = head_dim;
+    t->dtype = kv_dtype;
     *out = t;
     return ok();
 }
@@ -755,9 +798,7 @@ lci_status lci_sparse_attn(const void* q, int32_t batch, int32_t S, int32_t H_q,
     (void)workspace;
     (void)workspace_bytes;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    // many queries per sequence: the tensor-core tile schedule
-    const bool many = phase == LCI_PHASE_PREFILL || (phase == LCI_PHASE_AUTO && S >= 16);
-    if (many && prefill_attn_fits(table, H_q, topk, k_pool, v_pool))
+    if (use_prefill_attn(table, S, H_q, topk, phase, k_pool, v_pool))
         return launch_attn_prefill(q, batch, S, H_q, k_pool, v_pool, table, d_ids, topk, d_ctx_len,
                                    d_q_start, scale, out, cs);
     if (decode_kernel_fits(table, H_q, k_pool, v_pool))
@@ -791,8 +832,7 @@ lci_status lci_sparse_attn_partial(const void* q, int32_t batch, int32_t S, int3
     if (!(scale > 0.f)) scale = 1.0f / std::sqrt((float)table->head_dim);
     if (!std::isfinite(scale)) return fail(LCI_ERR_INVALID_ARG, "sparse_attn_partial: non-finite scale");
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    const bool many = phase == LCI_PHASE_PREFILL || (phase == LCI_PHASE_AUTO && S >= 16);
-    if (many && prefill_attn_fits(table, H_q, topk, k_pool, v_pool))
+    if (use_prefill_attn(table, S, H_q, topk, phase, k_pool, v_pool))
         return launch_attn_prefill(q, batch, S, H_q, k_pool, v_pool, table, d_ids, topk, d_ctx_len,
                                    d_q_start, scale, out, cs, lse);
     return launch_attn_decode(q, batch, S, H_q, k_pool, v_pool, table, d_ids, topk, d_ctx_len,
@@ -873,6 +913,65 @@ lci_status lci_attn_merge(const void* d_o, const float* d_lse, lci_dtype dtype, 
 }
 
 }  // extern "C"
+
+// ---- chunked gated state scan ----
+
+namespace {
+// [B][T][H][128] bf16 as a 4-D tensor (d, h, t, b), read in 64 x 1 x 128 x 1
+// boxes with the 128-byte swizzle; tokens past T read as zero.
+lci_status encode_bthd_map(CUtensorMap* map, const void* base, int32_t B, int32_t T, int32_t H) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return fail(LCI_ERR_CUDA, "gated_state_scan: cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[4] = {128, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {256, (cuuint64_t)H * 256, (cuuint64_t)T * H * 256};
+    cuuint32_t box[4] = {64, 1, 128, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(LCI_ERR_CUDA, "gated_state_scan: tensor map encode failed (%d)", (int)r);
+    return LCI_OK;
+}
+}  // namespace
+
+extern "C" lci_status lci_gated_state_scan(const void* q, const void* k, const void* v,
+                                           lci_dtype dtype, const float* d_gate,
+                                           const float* d_state_in, float* d_state_out,
+                                           int32_t batch, int32_t T, int32_t H, int32_t dk,
+                                           int32_t dv, int32_t chunk, float* d_out, void* stream) {
+    if (!q || !k || !v || !d_gate || !d_state_in || !d_state_out || !d_out)
+        return fail(LCI_ERR_INVALID_ARG, "gated_state_scan: null pointer argument");
+    if (batch <= 0 || T <= 0 || H <= 0 || dk <= 0 || dv <= 0 || chunk <= 0)
+        return fail(LCI_ERR_INVALID_ARG, "gated_state_scan: sizes must be positive");
+    if (!dtype_ok(dtype)) return fail(LCI_ERR_INVALID_ARG, "gated_state_scan: unknown dtype");
+    if (dtype != LCI_BF16 || dk != lci::gss::kD || dv != lci::gss::kD || chunk != lci::gss::kC)
+        return fail(LCI_ERR_UNSUPPORTED, "gated_state_scan: supports bf16 q/k/v with dk = dv = %d "
+                    "and chunks of %d tokens", lci::gss::kD, lci::gss::kC);
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v))
+        return fail(LCI_ERR_INVALID_ARG, "gated_state_scan: q, k and v must be 16-byte aligned");
+    if ((long long)batch * H >= (1ll << 31))
+        return fail(LCI_ERR_UNSUPPORTED, "gated_state_scan: grid too large");
+    CUtensorMap tq, tk, tv;
+    lci_status s = encode_bthd_map(&tq, q, batch, T, H);
+    if (s == LCI_OK) s = encode_bthd_map(&tk, k, batch, T, H);
+    if (s == LCI_OK) s = encode_bthd_map(&tv, v, batch, T, H);
+    if (s != LCI_OK) return s;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(lci::gated_state_scan_kernel,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        lci::gss::kSmemBytes);
+    });
+    if (attr_err != cudaSuccess)
+        return fail(LCI_ERR_CUDA, "gated_state_scan: %s", cudaGetErrorString(attr_err));
+    const int nchunks = (T + chunk - 1) / chunk;
+    lci::gated_state_scan_kernel<<<(unsigned)(batch * H), lci::gss::kThreads, lci::gss::kSmemBytes,
+                                   static_cast<cudaStream_t>(stream)>>>(
+        tq, tk, tv, d_gate, d_state_in, d_state_out, T, H, nchunks, d_out);
+    return check_launch("gated_state_scan");
+}
 
 // ---- index selection without device allocation ----
 //

@@ -145,6 +145,13 @@ __device__ __forceinline__ bool wait_flag_set(const unsigned int* flag) {
     }
 }
 
+// 2^x by the hardware approximation (relative error about 2^-22; 2^-inf = 0).
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Barrier among `count` threads of the CTA (a multiple of 32), id 1..15.
 __device__ __forceinline__ void named_barrier_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

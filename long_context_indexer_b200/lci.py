@@ -56,6 +56,8 @@ SIGNATURES = {
     "lci_sparse_attn_pipelined": (_st, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp,
                                         _f32, _vp, _vp, _vp]),
     "lci_set_wait_limit_ns": (_st, [ctypes.c_uint64]),
+    "lci_gated_state_scan": (_st, [_vp, _vp, _vp, _st, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
+                                   _i32, _vp, _vp]),
     "lci_block_scores_at": (_st, [_vp, _vp, _st, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _vp,
                                   _vp]),
     "lci_ids_shift": (_st, [_vp, ctypes.c_int64, _i32, _i32, _i32, _vp, _vp]),
@@ -311,12 +313,19 @@ def sparse_attn(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, tab
     return out
 
 
+_decode_ws_sizes: Dict[Tuple[int, ...], int] = {}
+
+
 def sparse_decode_workspace_size(B, S, H_i, d_c, nb_max, topk) -> int:
-    n = ctypes.c_size_t()
-    _check(load_library().lci_sparse_decode_workspace_size(B, S, H_i, d_c, nb_max, topk,
-                                                           ctypes.byref(n)),
-           "lci_sparse_decode_workspace_size")
-    return n.value
+    key = (B, S, H_i, d_c, nb_max, topk)
+    n = _decode_ws_sizes.get(key)
+    if n is None:
+        c = ctypes.c_size_t()
+        _check(load_library().lci_sparse_decode_workspace_size(B, S, H_i, d_c, nb_max, topk,
+                                                               ctypes.byref(c)),
+               "lci_sparse_decode_workspace_size")
+        n = _decode_ws_sizes[key] = c.value
+    return n
 
 
 def sparse_decode(q_c: torch.Tensor, k_c: torch.Tensor, ctx_len: torch.Tensor,
@@ -483,6 +492,30 @@ def attn_merge(o: torch.Tensor, lse: torch.Tensor, out: Optional[torch.Tensor] =
                                          _dev(out, "out", o.dtype), _stream(stream)),
            "lci_attn_merge")
     return out
+
+
+def gated_state_scan(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tensor,
+                     state: torch.Tensor, chunk: int = 128, out: Optional[torch.Tensor] = None,
+                     state_out: Optional[torch.Tensor] = None, stream=None):
+    """N4: chunked gated state scan. q, k [B, T, H, dk], v [B, T, H, dv] (bf16),
+    gate [B, H, ceil(T/chunk)] and state [B, H, dk, dv] (fp32). Returns
+    (out [B, T, H, dv] fp32, final state); state_out=state updates in place."""
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    if tuple(k.shape) != (B, T, H, dk) or tuple(v.shape[:3]) != (B, T, H):
+        raise ValueError("lci: q, k, v shapes disagree")
+    if tuple(gate.shape) != (B, H, -(-T // chunk)) or tuple(state.shape) != (B, H, dk, dv):
+        raise ValueError("lci: gate must be [B, H, nchunks] and state [B, H, dk, dv]")
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=torch.float32, device=q.device)
+    if state_out is None:
+        state_out = torch.empty_like(state)
+    _check(load_library().lci_gated_state_scan(
+        _dev(q, "q", None, 4), _dev(k, "k", q.dtype, 4), _dev(v, "v", q.dtype, 4), _dtype_code(q),
+        _dev(gate, "gate", torch.float32, 3), _dev(state, "state", torch.float32, 4),
+        _dev(state_out, "state_out", torch.float32, 4), B, T, H, dk, dv, chunk,
+        _dev(out, "out", torch.float32, 4), _stream(stream)), "lci_gated_state_scan")
+    return out, state_out
 
 
 def sparse_attn_pipelined(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,

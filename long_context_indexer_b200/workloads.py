@@ -33,7 +33,8 @@ from typing import Dict, Optional
 
 import torch
 
-__all__ = ["Config", "CONFIGS", "generate", "grid_values"]
+__all__ = ["Config", "CONFIGS", "generate", "grid_values", "ScanConfig", "SCAN_CONFIGS",
+           "generate_scan"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -157,3 +158,51 @@ def generate(cfg: Config, seed: Optional[int] = None, with_kv: bool = True,
     out["q_start"] = torch.full((B,), cfg.q_start, dtype=torch.int32)
     return out
 
+
+
+# ---------------------------------------------------------------- state scan
+
+@dataclasses.dataclass(frozen=True)
+class ScanConfig:
+    """A chunked gated state scan workload: B sequences of T tokens, H heads,
+    dk = dv = d, chunks of C tokens."""
+    name: str
+    B: int
+    T: int
+    H: int
+    d: int
+    C: int
+    seed: int
+    gate_lo: float = 0.9     # gates uniform in [gate_lo, 1)
+
+    @property
+    def nchunks(self) -> int:
+        return (self.T + self.C - 1) // self.C
+
+    def replace(self, **kw) -> "ScanConfig":
+        return dataclasses.replace(self, **kw)
+
+
+# 9 sequences x 16 heads = 144 (sequence, head) scans of 16384 tokens: one per SM
+SCAN_CONFIGS: Dict[str, ScanConfig] = {
+    "scan": ScanConfig("scan", B=9, T=16384, H=16, d=128, C=128, seed=5),
+    "scan_small": ScanConfig("scan_small", B=2, T=300, H=3, d=128, C=128, seed=6),
+}
+
+
+def generate_scan(cfg: ScanConfig, seed: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """q, k, v ~ N(0, 1/d) in bf16 (unit-norm scale for the dot products), gates
+    uniform in [gate_lo, 1) (fp32), initial state ~ N(0, 1) (fp32). CPU tensors."""
+    seed = cfg.seed if seed is None else seed
+    g = torch.Generator().manual_seed(seed * 7919 + 17)
+    s = cfg.d ** -0.5
+    shape = (cfg.B, cfg.T, cfg.H, cfg.d)
+    out = {
+        "q": (_randn_chunked(shape, g, torch.float32) * s).to(torch.bfloat16),
+        "k": (_randn_chunked(shape, g, torch.float32) * s).to(torch.bfloat16),
+        "v": _randn_chunked(shape, g, torch.bfloat16),
+        "gate": cfg.gate_lo + (1 - cfg.gate_lo) * torch.rand((cfg.B, cfg.H, cfg.nchunks),
+                                                             generator=g),
+        "state": torch.randn((cfg.B, cfg.H, cfg.d, cfg.d), generator=g),
+    }
+    return out
