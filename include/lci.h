@@ -364,29 +364,44 @@ LCI_API lci_status lci_index_select_noalloc(const void* q_c, const void* k_c, lc
                                             void* stream);
 
 /*
- * Workspace bytes lci_sparse_decode needs for these sizes.
+ * Workspace bytes lci_sparse_decode needs for these sizes and this block table
+ * (nb_max is the table's max_blocks).
  */
 LCI_API lci_status lci_sparse_decode_workspace_size(int32_t batch, int32_t S, int32_t H_i,
-                                                    int32_t d_c, int32_t nb_max, int32_t topk,
-                                                    size_t* bytes);
+                                                    int32_t d_c, int32_t topk, int32_t H_q,
+                                                    const lci_block_table* table, size_t* bytes);
 
 /*
  * One decode step in one call: lci_index_select (one-row-at-a-time schedule)
- * followed by lci_sparse_attn, with identical results, block ids included.
- * [GPU-stack] "Separate Paths for Prefill and Decode" asks that decode overlap
- * index selection with the cache reads; here the indexer publishes each query
- * row as soon as its block ids are final, and the attention kernel, launched
- * behind it (programmatic dependent launch), starts on a row as soon as that
- * row is published, while later rows are still being scored.
+ * followed by lci_sparse_attn, with identical block ids and outputs within the
+ * attention tolerance. [GPU-stack] "Separate Paths for Prefill and Decode" asks
+ * that decode pipeline index prefetching with incremental aggregation; [Hetero]
+ * §IV that index retrieval and attention be pipelined to hide retrieval
+ * latency. For bf16 keys of H_i*d_c = 1024 features and the decode attention
+ * shapes (head_dim 128, block_size a multiple of 64, at most 16 query heads per
+ * KV head) the step is ONE persistent launch: CTAs claim scoring chunks from a
+ * global counter, the last chunk of a row selects the row's blocks and
+ * publishes it, and CTAs then claim attention splits of published rows while
+ * later rows are still being scored; the last split of a (row, KV head) pair
+ * to finish combines the splits. Other shapes run the indexer and the
+ * attention kernel back to back, each row's attention starting as soon as the
+ * indexer publishes the row.
  * Arguments are those of the two calls; k_c's nb_max must equal the table's
  * max_blocks and all floating inputs share one dtype. The workspace holds the
- * indexer's scratch and per-row publication flags: zero-fill it before its
- * first call and again before using it with other sizes or after a call that
- * failed on the device; every successful call leaves it ready for the next.
- * The flags are cleared by each call itself before its attention kernel can
- * start, so a flag left set by an earlier call is never taken for a new
+ * scratch, per-row publication flags and the per-call counters: zero-fill it
+ * before its first call and again before using it with other sizes or after a
+ * call that failed on the device; every successful call leaves it ready for
+ * the next. A flag left set by an earlier call is never taken for a new
  * publication. Calls sharing a workspace must not overlap in time.
  */
+/*
+ * How many kernel launches lci_sparse_decode makes for these sizes: 1 (the
+ * one-launch persistent step) or 2 (indexer, then attention), assuming
+ * 16-byte aligned pools.
+ */
+LCI_API lci_status lci_sparse_decode_launches(int32_t H_i, int32_t d_c, int32_t H_q,
+                                              const lci_block_table* table, int32_t* launches);
+
 LCI_API lci_status lci_sparse_decode(const void* q_c, const void* k_c, lci_dtype dtype,
                                      int32_t batch, int32_t S, int32_t H_i, int32_t d_c,
                                      int32_t nb_max, const int32_t* d_ctx_len,

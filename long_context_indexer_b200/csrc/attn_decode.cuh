@@ -58,6 +58,109 @@ __device__ __forceinline__ uint32_t tile_off(int r, int c) {
     return (uint32_t)((c >> 3) * dec::kBox + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
+// One 64-token K/V tile (two 64x64 boxes of K then of V, 128-byte swizzle, at
+// shared address kbase) for consumer warp w, which takes tokens 16w..16w+15:
+// S = Q K^T with mma.m16n8k16, the online softmax update of (m, l) for the
+// fragment's two head rows, and O += P V. t0 is the tile's first token;
+// tokens after `last` are masked (their V is never read into the MMA).
+__device__ __forceinline__ void dec_consume_tile(uint32_t kbase, int w, int g8, int q4, int t0,
+                                                 long long last, float scale_log2,
+                                                 const uint4 (&qa)[4], const uint4 (&qb)[4],
+                                                 float& m_a, float& m_b, float& l_a, float& l_b,
+                                                 float (&o)[2][8][4]) {
+    using namespace dec;
+    const long long wt0 = (long long)t0 + 16 * w;  // first token of this warp
+    if (wt0 <= last) {
+        const uint32_t vbase = kbase + 2 * kBox;
+        // S = Q K^T over this warp's 16 tokens (two n-tiles of 8)
+        float sacc[2][4];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sacc[j][e] = 0.f;
+            const int tr = 16 * w + 8 * j + tok_perm(g8);
+#pragma unroll
+            for (int sl = 0; sl < 4; ++sl) {
+                const uint4 kk = lds128(kbase + tile_off(tr, 4 * sl + q4));
+                mma_bf16_16816(sacc[j], qa[sl].x, qb[sl].x, qa[sl].y, qb[sl].y, kk.x, kk.y);
+                mma_bf16_16816(sacc[j], qa[sl].z, qb[sl].z, qa[sl].w, qb[sl].w, kk.z, kk.w);
+            }
+        }
+        // tokens of the C-fragment columns: n = 2*q4, 2*q4+1 of each n-tile
+        const int c0 = tok_perm(2 * q4), c1 = tok_perm(2 * q4 + 1);
+        const bool partial = wt0 + 15 > last;
+        float x[2][4];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const long long ta = wt0 + 8 * j + c0, tb = wt0 + 8 * j + c1;
+            x[j][0] = (partial && ta > last) ? -INFINITY : sacc[j][0] * scale_log2;
+            x[j][1] = (partial && tb > last) ? -INFINITY : sacc[j][1] * scale_log2;
+            x[j][2] = (partial && ta > last) ? -INFINITY : sacc[j][2] * scale_log2;
+            x[j][3] = (partial && tb > last) ? -INFINITY : sacc[j][3] * scale_log2;
+        }
+        float mx_a = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+        float mx_b = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
+        mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
+        mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
+        mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
+        mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
+        const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
+        const float base_a = mn_a == -INFINITY ? 0.f : mn_a;
+        const float base_b = mn_b == -INFINITY ? 0.f : mn_b;
+        const float corr_a = exp2f(m_a - base_a), corr_b = exp2f(m_b - base_b);
+        m_a = mn_a;
+        m_b = mn_b;
+        float pr[2][4];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            pr[j][0] = exp2f(x[j][0] - base_a);
+            pr[j][1] = exp2f(x[j][1] - base_a);
+            pr[j][2] = exp2f(x[j][2] - base_b);
+            pr[j][3] = exp2f(x[j][3] - base_b);
+        }
+        l_a = l_a * corr_a + (pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1]);
+        l_b = l_b * corr_b + (pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3]);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                o[h][i][0] *= corr_a;
+                o[h][i][1] *= corr_a;
+                o[h][i][2] *= corr_b;
+                o[h][i][3] *= corr_b;
+            }
+        const uint32_t pa0 = pack_bf16x2(pr[0][0], pr[0][1]);
+        const uint32_t pa1 = pack_bf16x2(pr[0][2], pr[0][3]);
+        const uint32_t pa2 = pack_bf16x2(pr[1][0], pr[1][1]);
+        const uint32_t pa3 = pack_bf16x2(pr[1][2], pr[1][3]);
+        // V rows of the k positions 2q4, 2q4+1, 2q4+8, 2q4+9
+        const int r0 = 16 * w + c0, r1 = 16 * w + c1, r2 = r0 + 8, r3 = r1 + 8;
+        // masked tokens must not reach the MMA (their V may be unset memory)
+        const bool z0 = partial && wt0 + c0 > last, z1 = partial && wt0 + c1 > last;
+        const bool z2 = partial && wt0 + 8 + c0 > last, z3 = partial && wt0 + 8 + c1 > last;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint4 va = lds128(vbase + tile_off(r0, 8 * h + g8));
+            uint4 vb = lds128(vbase + tile_off(r1, 8 * h + g8));
+            uint4 vc = lds128(vbase + tile_off(r2, 8 * h + g8));
+            uint4 vd = lds128(vbase + tile_off(r3, 8 * h + g8));
+            if (z0) va = make_uint4(0, 0, 0, 0);
+            if (z1) vb = make_uint4(0, 0, 0, 0);
+            if (z2) vc = make_uint4(0, 0, 0, 0);
+            if (z3) vd = make_uint4(0, 0, 0, 0);
+            const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
+            const uint32_t wc[4] = {vc.x, vc.y, vc.z, vc.w}, wd[4] = {vd.x, vd.y, vd.z, vd.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t sel = (i & 1) ? 0x7632u : 0x5410u;
+                const uint32_t b0 = __byte_perm(wa[i >> 1], wb[i >> 1], sel);
+                const uint32_t b1 = __byte_perm(wc[i >> 1], wd[i >> 1], sel);
+                mma_bf16_16816(o[h][i], pa0, pa1, pa2, pa3, b0, b1);
+            }
+        }
+    }
+}
+
 template <int kStages>
 __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -211,97 +314,9 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
             const int st = it % kStages;
             const bool ok = mbar_wait(&full_bar[st], (it / kStages) & 1);
             const int t0 = info[st];
-            const long long wt0 = (long long)t0 + 16 * w;  // first token of this warp
-            if (ok && t0 >= 0 && wt0 <= last) {
-                const uint32_t kbase = smem_u32(smem + st * kStageBytes);
-                const uint32_t vbase = kbase + 2 * kBox;
-                // S = Q K^T over this warp's 16 tokens (two n-tiles of 8)
-                float sacc[2][4];
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) sacc[j][e] = 0.f;
-                    const int tr = 16 * w + 8 * j + tok_perm(g8);
-#pragma unroll
-                    for (int sl = 0; sl < 4; ++sl) {
-                        const uint4 kk = lds128(kbase + tile_off(tr, 4 * sl + q4));
-                        mma_bf16_16816(sacc[j], qa[sl].x, qb[sl].x, qa[sl].y, qb[sl].y, kk.x, kk.y);
-                        mma_bf16_16816(sacc[j], qa[sl].z, qb[sl].z, qa[sl].w, qb[sl].w, kk.z, kk.w);
-                    }
-                }
-                // tokens of the C-fragment columns: n = 2*q4, 2*q4+1 of each n-tile
-                const int c0 = tok_perm(2 * q4), c1 = tok_perm(2 * q4 + 1);
-                const bool partial = wt0 + 15 > last;
-                float x[2][4];
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const long long ta = wt0 + 8 * j + c0, tb = wt0 + 8 * j + c1;
-                    x[j][0] = (partial && ta > last) ? -INFINITY : sacc[j][0] * scale_log2;
-                    x[j][1] = (partial && tb > last) ? -INFINITY : sacc[j][1] * scale_log2;
-                    x[j][2] = (partial && ta > last) ? -INFINITY : sacc[j][2] * scale_log2;
-                    x[j][3] = (partial && tb > last) ? -INFINITY : sacc[j][3] * scale_log2;
-                }
-                float mx_a = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
-                float mx_b = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
-                mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
-                mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
-                mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
-                mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
-                const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
-                const float base_a = mn_a == -INFINITY ? 0.f : mn_a;
-                const float base_b = mn_b == -INFINITY ? 0.f : mn_b;
-                const float corr_a = exp2f(m_a - base_a), corr_b = exp2f(m_b - base_b);
-                m_a = mn_a;
-                m_b = mn_b;
-                float pr[2][4];
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    pr[j][0] = exp2f(x[j][0] - base_a);
-                    pr[j][1] = exp2f(x[j][1] - base_a);
-                    pr[j][2] = exp2f(x[j][2] - base_b);
-                    pr[j][3] = exp2f(x[j][3] - base_b);
-                }
-                l_a = l_a * corr_a + (pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1]);
-                l_b = l_b * corr_b + (pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3]);
-#pragma unroll
-                for (int h = 0; h < 2; ++h)
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        o[h][i][0] *= corr_a;
-                        o[h][i][1] *= corr_a;
-                        o[h][i][2] *= corr_b;
-                        o[h][i][3] *= corr_b;
-                    }
-                const uint32_t pa0 = pack_bf16x2(pr[0][0], pr[0][1]);
-                const uint32_t pa1 = pack_bf16x2(pr[0][2], pr[0][3]);
-                const uint32_t pa2 = pack_bf16x2(pr[1][0], pr[1][1]);
-                const uint32_t pa3 = pack_bf16x2(pr[1][2], pr[1][3]);
-                // V rows of the k positions 2q4, 2q4+1, 2q4+8, 2q4+9
-                const int r0 = 16 * w + c0, r1 = 16 * w + c1, r2 = r0 + 8, r3 = r1 + 8;
-                // masked tokens must not reach the MMA (their V may be unset memory)
-                const bool z0 = partial && wt0 + c0 > last, z1 = partial && wt0 + c1 > last;
-                const bool z2 = partial && wt0 + 8 + c0 > last, z3 = partial && wt0 + 8 + c1 > last;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint4 va = lds128(vbase + tile_off(r0, 8 * h + g8));
-                    uint4 vb = lds128(vbase + tile_off(r1, 8 * h + g8));
-                    uint4 vc = lds128(vbase + tile_off(r2, 8 * h + g8));
-                    uint4 vd = lds128(vbase + tile_off(r3, 8 * h + g8));
-                    if (z0) va = make_uint4(0, 0, 0, 0);
-                    if (z1) vb = make_uint4(0, 0, 0, 0);
-                    if (z2) vc = make_uint4(0, 0, 0, 0);
-                    if (z3) vd = make_uint4(0, 0, 0, 0);
-                    const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
-                    const uint32_t wc[4] = {vc.x, vc.y, vc.z, vc.w}, wd[4] = {vd.x, vd.y, vd.z, vd.w};
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const uint32_t sel = (i & 1) ? 0x7632u : 0x5410u;
-                        const uint32_t b0 = __byte_perm(wa[i >> 1], wb[i >> 1], sel);
-                        const uint32_t b1 = __byte_perm(wc[i >> 1], wd[i >> 1], sel);
-                        mma_bf16_16816(o[h][i], pa0, pa1, pa2, pa3, b0, b1);
-                    }
-                }
-            }
+            if (ok && t0 >= 0)
+                dec_consume_tile(smem_u32(smem + st * kStageBytes), w, g8, q4, t0, last, scale_log2,
+                                 qa, qb, m_a, m_b, l_a, l_b, o);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty_bar[st]);
         }

@@ -16,9 +16,11 @@
 //   P  = exp2(S*c - m)    rows whose query did not select the unit's block, and
 //                         tokens after the query's position, get P = 0
 //   O += P V              tcgen05.mma with A = P read from TMEM, B = V read
-//                         MN-major from shared memory
-// Q stays in shared memory for the whole tile; S (two buffers), P (two
-// buffers) and O live in TMEM (128 + 256 + 128 = 512 columns). Rows of one
+//                         MN-major from shared memory (S = Q K^T reads Q from
+//                         TMEM too)
+// Q (as bf16 pairs, the MMA's A operand), S (two buffers, each also holding
+// its stage's P once read) and O live in TMEM; shared memory holds only the
+// K and V rings (three stages each). Rows of one
 // MMA belong to different queries, so a K/V tile is read once per tile instead
 // of once per query.
 //
@@ -48,16 +50,18 @@ constexpr int kRows = 128;             // MMA rows per tile
 constexpr int kStageTok = 128;         // tokens per stage (two 64-token units)
 constexpr int kHalf = 128 * 128;       // one 64-dim half of a 128-row tile: 16 KiB
 constexpr int kTileBytes = 2 * kHalf;  // 128 rows x 128 dims bf16: 32 KiB
-constexpr int kKStages = 2, kVStages = 2;
+constexpr int kKStages = 3, kVStages = 3;
 constexpr int kMaxWords = 512;         // block bitmap words: nb_max <= 16384
 constexpr int kMaxUnion = 1024;        // distinct blocks per tile (QT * topk)
 constexpr int kSoftWarps = 8;            // two threads per MMA row
 constexpr int kThreads = 64 + 32 * kSoftWarps;
-constexpr int kColO = 0, kColS = 128, kColP = 384, kTmemCols = 512;
+// TMEM columns: O [128 rows x 128 dims] fp32, two S buffers [128 x 128 tokens]
+// fp32 whose first 64 columns then hold the stage's P as bf16 pairs, and Q
+// [128 x 128 dims] as bf16 pairs (the A operand of S = Q K^T)
+constexpr int kColO = 0, kColS = 128, kColQ = 384, kTmemCols = 512;
 constexpr float kLazy = 8.0f;          // rescale when the maximum grows past m + 8
 // shared memory layout (offsets from a 1024-byte aligned base)
-constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kTileBytes;
+constexpr int kOffK = 0;
 constexpr int kOffV = kOffK + kKStages * kTileBytes;
 constexpr int kOffUnion = kOffV + kVStages * kTileBytes;
 constexpr int kUnionBytes = 2 * kMaxWords * 4 + 3 * kMaxUnion * 4;
@@ -266,24 +270,38 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
     const int nstages = (nunits + 1) / 2;
     const long long ctx = ctx_len[b];
 
-    // ---------------- Q tile -> shared memory (swizzled, K-major) ----------------
-    if (warp >= 2) {
-        const int r = (warp & 3) * 32 + lane, hf = (warp - 2) >> 2;
-        const int qi = r / G, s = s0 + qi;
-        const uint4* src = reinterpret_cast<const uint4*>(
-            q + (((size_t)b * S + s) * H_q + (size_t)g * G + (r - qi * G)) * kHD);
-        unsigned char* qs = smem + kOffQ;
-#pragma unroll
-        for (int c = 8 * hf; c < 8 * hf + 8; ++c) {
-            const uint4 v = s < S ? src[c] : make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(qs + pfa_off(r, c)) = v;
-        }
-        fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // ---------------- Q tile -> TMEM (the A operand of S = Q K^T) ----------------
+    // The softmax warps store their row halves (bf16 pairs: column c holds dims
+    // 2c, 2c+1); the MMA warp waits for them on named barrier 5. The producer
+    // starts its loads meanwhile.
+    constexpr int kQBarrier = 5, kQThreads = 32 + 32 * kSoftWarps;
+    if (warp >= 2) {
+        const int quarter = warp & 3, hf = (warp - 2) >> 2;
+        const int r = quarter * 32 + lane;
+        const int qi = r / G, s = s0 + qi;
+        const uint4* src = reinterpret_cast<const uint4*>(
+            q + (((size_t)b * S + s) * H_q + (size_t)g * G + (r - qi * G)) * kHD);
+        uint32_t qv[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint4 v = s < S ? src[8 * hf + c] : make_uint4(0, 0, 0, 0);
+            qv[4 * c] = v.x;
+            qv[4 * c + 1] = v.y;
+            qv[4 * c + 2] = v.z;
+            qv[4 * c + 3] = v.w;
+        }
+        tmem_st32(tmem_base + ((uint32_t)(quarter * 32) << 16) + kColQ + hf * 32, qv);
+        tmem_wait_st();
+        tc_fence_before();
+        named_barrier_sync(kQBarrier, kQThreads);
+    } else if (warp == 1) {
+        named_barrier_sync(kQBarrier, kQThreads);
+        tc_fence_after();
+    }
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -341,7 +359,6 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            const uint32_t qa = smem_u32(smem + kOffQ);
             auto pv = [&](int j) -> bool {
                 const int vs = j % kVStages;
                 if (!mbar_wait(&pfull[j & 1], (j >> 1) & 1) ||
@@ -353,7 +370,7 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
                 const uint32_t vb = smem_u32(smem + kOffV + vs * kTileBytes);
 #pragma unroll
                 for (int kt = 0; kt < kStageTok / 16; ++kt)  // 16 tokens per MMA
-                    tc_mma_tmem_a(tmem_base + kColO, tmem_base + kColP + (j & 1) * 64 + kt * 8,
+                    tc_mma_tmem_a(tmem_base + kColO, tmem_base + kColS + (j & 1) * 128 + kt * 8,
                                   sw128_desc_mn(vb + kt * 2048, kHalf), kIdescPV,
                                   (j > 0 || kt > 0) ? 1u : 0u);
                 tc_commit(&vempty[vs]);
@@ -374,8 +391,8 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
 #pragma unroll
                 for (int kk = 0; kk < kHD / 16; ++kk) {  // 16 dims per MMA
                     const uint32_t off = (kk >> 2) * kHalf;
-                    tc_mma(d, sw128_desc(qa + off) + 2 * (kk & 3), sw128_desc(kb + off) + 2 * (kk & 3),
-                           kIdescQK, kk > 0 ? 1u : 0u);
+                    tc_mma_tmem_a(d, tmem_base + kColQ + kk * 8, sw128_desc(kb + off) + 2 * (kk & 3),
+                                  kIdescQK, kk > 0 ? 1u : 0u);
                 }
                 tc_commit(&kempty[ks]);
                 tc_commit(&sfull[i & 1]);
@@ -453,7 +470,9 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
             int* xo = xok + (i & 1) * 256;
             xm[hf * 128 + r] = mx;
             xo[hf * 128 + r] = my_ok;
+            tc_fence_before();  // this half's S loads are ordered before the partner's P stores
             named_barrier_sync(bar_id, 64);
+            tc_fence_after();
             if (!__all_sync(0xffffffffu, my_ok && xo[(hf ^ 1) * 128 + r])) {
                 *s_abort = 1;
                 break;
@@ -498,7 +517,9 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
 #pragma unroll
                     for (int e = 0; e < 16; ++e) pk[e] = 0u;
                 }
-                tmem_st16(lane_addr + kColP + (i & 1) * 64 + hf * 32 + ch * 16, pk);
+                // P overwrites the S buffer's first 64 columns: both halves
+                // have read their S columns (the barrier above)
+                tmem_st16(lane_addr + kColS + (i & 1) * 128 + hf * 32 + ch * 16, pk);
             }
             tmem_wait_st();
             // V rows of an absent unit and of tokens past the context length

@@ -21,6 +21,7 @@
 #include "common.cuh"
 #include "compress.cuh"
 #include "cp_merge.cuh"
+#include "decode_fused.cuh"
 #include "index_gemv.cuh"
 #include "index_prefill.cuh"
 #include "state_scan.cuh"
@@ -1034,25 +1035,115 @@ extern "C" {
 
 struct DecodePlan {
     IndexPlan ix;
-    size_t off_ready, bytes;
+    bool fused;                 // the one-launch persistent kernel
+    int nsplit;                 // attention splits per (row, KV head) pair (fused)
+    size_t off_ready, off_split, off_sync, off_part, bytes;
 };
 
-DecodePlan plan_decode(int32_t batch, int32_t S, int32_t K, int32_t nb_max, size_t esz) {
+// The one-launch kernel covers bf16 keys of 1024 features (2 KiB per block)
+// over the decode attention kernel's shapes.
+bool fused_decode_fits(lci_dtype dtype, int32_t K, const lci_block_table* t, int32_t H_q,
+                       const void* k_pool, const void* v_pool) {
+    return dtype == LCI_BF16 && K == 1024 && decode_kernel_fits(t, H_q, k_pool, v_pool);
+}
+
+DecodePlan plan_decode(int32_t batch, int32_t S, int32_t K, int32_t nb_max, size_t esz,
+                       int32_t topk, const lci_block_table* t, int32_t H_q, bool fused) {
     DecodePlan d{};
     d.ix = plan_index(batch, S, K, nb_max, esz);
+    d.fused = fused;
     const size_t rows = (size_t)batch * S;
     d.off_ready = align_up(d.ix.bytes);
-    d.bytes = d.off_ready + align_up(rows * sizeof(unsigned int));
+    size_t end = d.off_ready + align_up(rows * sizeof(unsigned int));
+    if (fused) {
+        // splits: about two attention items per SM, at least two 64-token tiles each
+        const long long pairs = (long long)rows * t->num_kv_heads;
+        const int nunits = topk * (t->block_size / 64);
+        long long want = (2 * 148 + pairs - 1) / pairs;
+        if (want > 32) want = 32;
+        if (want > nunits / 2) want = nunits / 2;
+        if (want < 1) want = 1;
+        const int per = (int)((nunits + want - 1) / want);
+        d.nsplit = (nunits + per - 1) / per;
+        d.off_split = end;
+        d.off_sync = d.off_split + align_up((size_t)pairs * sizeof(unsigned int));
+        d.off_part = d.off_sync + kAlign;
+        end = d.off_part + align_up((size_t)pairs * d.nsplit * lci::fdec::kPartFloats * sizeof(float));
+    }
+    (void)H_q;
+    d.bytes = end;
     return d;
 }
 
 lci_status lci_sparse_decode_workspace_size(int32_t batch, int32_t S, int32_t H_i, int32_t d_c,
-                                            int32_t nb_max, int32_t topk, size_t* bytes) {
-    if (!bytes) return fail(LCI_ERR_INVALID_ARG, "sparse_decode_workspace_size: null output");
-    lci_status st = check_index_args(batch, S, H_i, d_c, nb_max, topk, LCI_BF16);
+                                            int32_t topk, int32_t H_q,
+                                            const lci_block_table* table, size_t* bytes) {
+    if (!bytes || !table)
+        return fail(LCI_ERR_INVALID_ARG, "sparse_decode_workspace_size: null argument");
+    lci_status st = check_index_args(batch, S, H_i, d_c, table->max_blocks, topk, LCI_BF16);
     if (st != LCI_OK && st != LCI_ERR_UNSUPPORTED) return st;
-    *bytes = plan_decode(batch, S, H_i * d_c, nb_max, 2).bytes;  // same for both types
+    st = check_attn_args(batch, S, H_q, table, topk);
+    if (st != LCI_OK) return st;
+    const int K = H_i * d_c;
+    // enough for either schedule (the fused one is chosen when the call fits it)
+    const bool fused = table->dtype == LCI_BF16 && K == 1024 &&
+                       fused_decode_fits(LCI_BF16, K, table, H_q, nullptr, nullptr);
+    *bytes = plan_decode(batch, S, K, table->max_blocks, 2, topk, table, H_q, fused).bytes;
     return ok();
+}
+
+lci_status lci_sparse_decode_launches(int32_t H_i, int32_t d_c, int32_t H_q,
+                                      const lci_block_table* table, int32_t* launches) {
+    if (!table || !launches) return fail(LCI_ERR_INVALID_ARG, "sparse_decode_launches: null argument");
+    if (H_i <= 0 || d_c <= 0 || H_q <= 0 || H_q % table->num_kv_heads != 0)
+        return fail(LCI_ERR_INVALID_ARG, "sparse_decode_launches: bad sizes");
+    *launches = fused_decode_fits(table->dtype, H_i * d_c, table, H_q, nullptr, nullptr) ? 1 : 2;
+    return ok();
+}
+
+lci_status launch_decode_fused(const void* q_c, const void* k_c, int32_t batch, int32_t S,
+                               int32_t nb_max, const int32_t* ctx_len, const int32_t* q_start,
+                               int32_t topk, const void* q, int32_t H_q, const void* k_pool,
+                               const void* v_pool, const lci_block_table* t, float scale,
+                               int32_t* ids, void* out, char* w, const DecodePlan& pl,
+                               cudaStream_t st) {
+    if ((long long)pl.ix.chunk_blocks * 2048 > lci::fdec::kChunkBytes)
+        return fail(LCI_ERR_UNSUPPORTED, "sparse_decode: chunk of %d blocks too large",
+                    pl.ix.chunk_blocks);
+    CUtensorMap tm_k, tm_v;
+    lci_status s = pool_maps(t, k_pool, v_pool, &tm_k, &tm_v);
+    if (s != LCI_OK) return s;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    static int num_sms = 148;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(lci::sparse_decode_fused_kernel,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        lci::fdec::kSmemBytes);
+        int dev = 0;
+        if (attr_err == cudaSuccess) attr_err = cudaGetDevice(&dev);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    });
+    if (attr_err != cudaSuccess)
+        return fail(LCI_ERR_CUDA, "sparse_decode: %s", cudaGetErrorString(attr_err));
+    const int rows = batch * S;
+    const long long items = (long long)rows * pl.ix.nchunks +
+                            (long long)rows * t->num_kv_heads * pl.nsplit;
+    if (items >= (1ll << 31)) return fail(LCI_ERR_UNSUPPORTED, "sparse_decode: too many work items");
+    const int grid = (int)std::min<long long>(num_sms, items);
+    const float scale_log2 = scale * 1.4426950408889634f;
+    lci::sparse_decode_fused_kernel<<<grid, lci::fdec::kThreads, lci::fdec::kSmemBytes, st>>>(
+        static_cast<const __nv_bfloat16*>(q_c), static_cast<const __nv_bfloat16*>(k_c), S, nb_max,
+        t->block_size, ctx_len, q_start, topk, pl.ix.chunk_blocks, pl.ix.nchunks,
+        reinterpret_cast<float*>(w + pl.ix.off_scores), reinterpret_cast<uint32_t*>(w + pl.ix.off_chunk_max),
+        reinterpret_cast<unsigned int*>(w + pl.ix.off_counters), ids, tm_k, tm_v,
+        static_cast<const __nv_bfloat16*>(q), t->d_table, t->num_pages, t->num_kv_heads, H_q,
+        scale_log2, static_cast<__nv_bfloat16*>(out), pl.nsplit,
+        reinterpret_cast<float*>(w + pl.off_part), reinterpret_cast<unsigned int*>(w + pl.off_split),
+        reinterpret_cast<unsigned int*>(w + pl.off_ready), reinterpret_cast<unsigned int*>(w + pl.off_sync),
+        rows);
+    return check_launch("sparse_decode");
 }
 
 lci_status lci_sparse_decode(const void* q_c, const void* k_c, lci_dtype dtype, int32_t batch,
@@ -1075,7 +1166,9 @@ lci_status lci_sparse_decode(const void* q_c, const void* k_c, lci_dtype dtype, 
     if (!aligned16(q_c) || !aligned16(k_c))
         return fail(LCI_ERR_INVALID_ARG, "sparse_decode: q_c and k_c must be 16-byte aligned");
     const int K = H_i * d_c;
-    const DecodePlan pl = plan_decode(batch, S, K, nb_max, dtype_size(dtype));
+    const bool fused = fused_decode_fits(dtype, K, table, H_q, k_pool, v_pool);
+    const DecodePlan pl = plan_decode(batch, S, K, nb_max, dtype_size(dtype), topk, table, H_q,
+                                      fused);
     if (!workspace || workspace_bytes < pl.bytes ||
         (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
         return fail(LCI_ERR_WORKSPACE, "sparse_decode: workspace needs %zu bytes, 256-byte aligned "
@@ -1084,6 +1177,9 @@ lci_status lci_sparse_decode(const void* q_c, const void* k_c, lci_dtype dtype, 
     if (!std::isfinite(scale)) return fail(LCI_ERR_INVALID_ARG, "sparse_decode: non-finite scale");
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     char* w = static_cast<char*>(workspace);
+    if (pl.fused)
+        return launch_decode_fused(q_c, k_c, batch, S, nb_max, d_ctx_len, d_q_start, topk, q, H_q,
+                                   k_pool, v_pool, table, scale, d_ids, out, w, pl, cs);
     if (dtype == LCI_BF16 && decode_kernel_fits(table, H_q, k_pool, v_pool)) {
         // rows are published one by one and attended as soon as they are ready
         unsigned int* ready = reinterpret_cast<unsigned int*>(w + pl.off_ready);

@@ -47,7 +47,7 @@ SIGNATURES = {
     "lci_sparse_attn": (_st, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _f32,
                               _st, _vp, _vp, _sz, _vp]),
     "lci_get_device_status": (_st, [_vp]),
-    "lci_sparse_decode_workspace_size": (_st, [_i32, _i32, _i32, _i32, _i32, _i32,
+    "lci_sparse_decode_workspace_size": (_st, [_i32, _i32, _i32, _i32, _i32, _i32, _vp,
                                                ctypes.POINTER(_sz)]),
     "lci_sparse_decode": (_st, [_vp, _vp, _st, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp,
                                 _i32, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _sz, _vp]),
@@ -56,6 +56,7 @@ SIGNATURES = {
     "lci_sparse_attn_pipelined": (_st, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp,
                                         _f32, _vp, _vp, _vp]),
     "lci_set_wait_limit_ns": (_st, [ctypes.c_uint64]),
+    "lci_sparse_decode_launches": (_st, [_i32, _i32, _i32, _vp, ctypes.POINTER(_i32)]),
     "lci_gated_state_scan": (_st, [_vp, _vp, _vp, _st, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                    _i32, _vp, _vp]),
     "lci_block_scores_at": (_st, [_vp, _vp, _st, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _vp,
@@ -316,16 +317,25 @@ def sparse_attn(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, tab
 _decode_ws_sizes: Dict[Tuple[int, ...], int] = {}
 
 
-def sparse_decode_workspace_size(B, S, H_i, d_c, nb_max, topk) -> int:
-    key = (B, S, H_i, d_c, nb_max, topk)
+def sparse_decode_workspace_size(B, S, H_i, d_c, topk, H_q, table: BlockTable) -> int:
+    key = (B, S, H_i, d_c, topk, H_q, table.max_blocks, table.num_kv_heads, table.block_size,
+           table.head_dim, str(table.dtype))
     n = _decode_ws_sizes.get(key)
     if n is None:
         c = ctypes.c_size_t()
-        _check(load_library().lci_sparse_decode_workspace_size(B, S, H_i, d_c, nb_max, topk,
-                                                               ctypes.byref(c)),
+        _check(load_library().lci_sparse_decode_workspace_size(B, S, H_i, d_c, topk, H_q,
+                                                               table.handle, ctypes.byref(c)),
                "lci_sparse_decode_workspace_size")
         n = _decode_ws_sizes[key] = c.value
     return n
+
+
+def sparse_decode_launches(H_i: int, d_c: int, H_q: int, table: BlockTable) -> int:
+    """Kernel launches of one sparse_decode call: 1 (one persistent launch) or 2."""
+    n = ctypes.c_int32()
+    _check(load_library().lci_sparse_decode_launches(H_i, d_c, H_q, table.handle, ctypes.byref(n)),
+           "lci_sparse_decode_launches")
+    return n.value
 
 
 def sparse_decode(q_c: torch.Tensor, k_c: torch.Tensor, ctx_len: torch.Tensor,
@@ -348,9 +358,10 @@ def sparse_decode(q_c: torch.Tensor, k_c: torch.Tensor, ctx_len: torch.Tensor,
         ids = torch.empty((B, S, topk), dtype=torch.int32, device=q_c.device)
     if out is None:
         out = torch.empty_like(q)
-    need = sparse_decode_workspace_size(B, S, H_i, d_c, nb_max, topk)
+    need = sparse_decode_workspace_size(B, S, H_i, d_c, topk, H_q, table)
     if ws is None:
-        ws = workspace(q_c.device, need, f"sparse_decode:{B}x{S}x{nb_max}:{H_i * d_c}")
+        ws = workspace(q_c.device, need, f"sparse_decode:{B}x{S}x{nb_max}:{H_i * d_c}:{topk}:"
+                                         f"{H_q}x{table.num_kv_heads}x{table.block_size}")
     _check(load_library().lci_sparse_decode(
         _dev(q_c, "q_c", None, 4), _dev(k_c, "k_c", q_c.dtype, 4), _dtype_code(q_c), B, S, H_i,
         d_c, nb_max, _dev(ctx_len, "ctx_len", torch.int32, 1),

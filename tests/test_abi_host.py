@@ -127,9 +127,10 @@ def test_sparse_decode_host_checks(lib):
     assert lib.lci_create_block_table(FAKE, 2, 8, 20, 64, 1, 128, 1, ctypes.byref(h)) == 0
     try:
         need = ctypes.c_size_t()
-        assert lib.lci_sparse_decode_workspace_size(2, 1, 8, 128, 8, 4, ctypes.byref(need)) == 0
+        assert lib.lci_sparse_decode_workspace_size(2, 1, 8, 128, 4, 16, h, ctypes.byref(need)) == 0
         assert need.value > 0
-        assert lib.lci_sparse_decode_workspace_size(2, 1, 8, 128, 8, 4, None) == INVALID
+        assert lib.lci_sparse_decode_workspace_size(2, 1, 8, 128, 4, 16, h, None) == INVALID
+        assert lib.lci_sparse_decode_workspace_size(2, 1, 8, 128, 4, 16, None, ctypes.byref(need)) == INVALID
 
         def dec(**kw):
             a = dict(q_c=FAKE, k_c=FAKE, dtype=1, B=2, S=1, H_i=8, d_c=128, nb_max=8, ctx=FAKE,

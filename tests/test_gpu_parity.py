@@ -307,3 +307,32 @@ def test_decode_attention_deep_ring_uneven_splits(B, H_kv):
                                      d["q"], d["k_pool"], d["v_pool"], bt)
     torch.cuda.synchronize()
     assert torch.equal(ids_f, ids) and torch.equal(out_f, out)
+
+
+@pytest.mark.parametrize("name", ["decode", "long", "1m_decode"])
+def test_one_launch_decode_step_over_many_calls(name):
+    """The one-launch decode step (persistent CTAs claiming scoring chunks, then
+    attention splits) keeps its per-call counters and epoch in the workspace:
+    ten calls in a row on one workspace, interleaved with calls of another
+    size on another workspace, give the oracle's ids and outputs every time."""
+    cfg = CONFIGS[name]
+    w = generate(cfg)
+    d = upload(w)
+    bt = lci.create_block_table(d["block_table"], d["k_pool"])
+    other = SMALL.replace(H_i=8, d_c=128, S=3, q_start=997)
+    wo = generate(other)
+    do = upload(wo)
+    bto = lci.create_block_table(do["block_table"], do["k_pool"])
+    ref_ids, ref_out = oracle_rows(cfg, w)
+    ref_ids_o, ref_out_o = oracle_rows(other, wo)
+    for _ in range(10):
+        ids, out = lci.sparse_decode(d["q_c"], d["k_c"], d["ctx_len"], d["q_start"], cfg.topk,
+                                     d["q"], d["k_pool"], d["v_pool"], bt)
+        ids_o, out_o = lci.sparse_decode(do["q_c"], do["k_c"], do["ctx_len"], do["q_start"],
+                                         other.topk, do["q"], do["k_pool"], do["v_pool"], bto)
+    torch.cuda.synchronize()
+    lci.get_device_status()
+    assert torch.equal(ids.cpu().reshape(-1, cfg.topk), ref_ids)
+    assert_out_close(out.reshape(-1, cfg.H_q, cfg.hd), ref_out, torch.bfloat16, name)
+    assert torch.equal(ids_o.cpu().reshape(-1, other.topk), ref_ids_o)
+    assert_out_close(out_o.reshape(-1, other.H_q, other.hd), ref_out_o, torch.bfloat16, "other")

@@ -76,6 +76,6 @@ def test_state_scan_rejects_unsupported_shapes():
     cfg = SCAN_CONFIGS["scan_small"]
     d = {k: v.cuda() for k, v in generate_scan(cfg).items()}
     with pytest.raises(lci.LciError) as e:
-        lci.gated_state_scan(d["q"], d["k"], d["v"], d["gate"].repeat(1, 1, 2)[:, :, :5], d["state"],
-                             chunk=64)
+        lci.gated_state_scan(d["q"], d["k"], d["v"], d["gate"].repeat(1, 1, 2)[:, :, :5].contiguous(),
+                             d["state"], chunk=64)
     assert e.value.status == 2

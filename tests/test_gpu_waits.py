@@ -64,14 +64,16 @@ def test_unpublished_rows_time_out_and_report_timeout():
     assert torch.equal(ids2, ids) and torch.equal(out2, out_ref)
 
 
-def test_fused_decode_after_a_timed_out_consumer():
-    """After a consumer gave up, the one-call decode step on a workspace whose
-    flags were left set still waits for this call's own publications."""
-    cfg = CONFIGS["decode"]
+def test_two_kernel_decode_after_a_timed_out_consumer():
+    """After a consumer gave up, the two-kernel form of the one-call decode
+    step (block keys of 512 features, which the one-launch kernel does not
+    take) on a workspace whose flags were left set still waits for this call's
+    own publications."""
+    cfg = CONFIGS["decode"].replace(H_i=4)
     d = upload(generate(cfg))
     _, ids_ref, out_ref = run_gpu(cfg, d)
     bt = lci.create_block_table(d["block_table"], d["k_pool"])
-    need = lci.sparse_decode_workspace_size(cfg.B, cfg.S, cfg.H_i, cfg.d_c, cfg.NB, cfg.topk)
+    need = lci.sparse_decode_workspace_size(cfg.B, cfg.S, cfg.H_i, cfg.d_c, cfg.topk, cfg.H_q, bt)
     ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
     # Every publication flag left set, as after a consumer that gave up while
     # its producer published late. The arrival counters (the first 256 bytes,
