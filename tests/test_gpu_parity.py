@@ -264,13 +264,18 @@ def test_fused_decode_step_matches_two_calls_and_oracle(name):
     d = upload(w)
     _, ids2, out2 = run_gpu(cfg, d)
     bt = lci.create_block_table(d["block_table"], d["k_pool"])
-    for _ in range(3):  # the per-row flags must reset between calls
+    first = None
+    for _ in range(3):  # the per-call state must reset between calls
         ids, out = lci.sparse_decode(d["q_c"], d["k_c"], d["ctx_len"], d["q_start"], cfg.topk,
                                      d["q"], d["k_pool"], d["v_pool"], bt)
         torch.cuda.synchronize()
         lci.get_device_status()
         assert torch.equal(ids, ids2)
-        assert torch.equal(out, out2)
+        # the one-launch step splits and combines the attention its own way:
+        # within the tolerance of the two-call result, and run to run identical
+        assert (out.float() - out2.float()).abs().max().item() <= TOL[cfg.torch_dtype]
+        first = out.clone() if first is None else first
+        assert torch.equal(out, first)
     ref_ids, ref_out = oracle_rows(cfg, w)
     assert torch.equal(ids.cpu().reshape(-1, cfg.topk), ref_ids)
     assert_out_close(out.reshape(-1, cfg.H_q, cfg.hd), ref_out, cfg.torch_dtype, name)
@@ -306,7 +311,8 @@ def test_decode_attention_deep_ring_uneven_splits(B, H_kv):
     ids_f, out_f = lci.sparse_decode(d["q_c"], d["k_c"], d["ctx_len"], d["q_start"], cfg.topk,
                                      d["q"], d["k_pool"], d["v_pool"], bt)
     torch.cuda.synchronize()
-    assert torch.equal(ids_f, ids) and torch.equal(out_f, out)
+    assert torch.equal(ids_f, ids)
+    assert_out_close(out_f.reshape(-1, cfg.H_q, cfg.hd), ref_out, cfg.torch_dtype, "one call")
 
 
 @pytest.mark.parametrize("name", ["decode", "long", "1m_decode"])
