@@ -377,15 +377,10 @@ LCI_API lci_status lci_sparse_decode_workspace_size(int32_t batch, int32_t S, in
  * attention tolerance. [GPU-stack] "Separate Paths for Prefill and Decode" asks
  * that decode pipeline index prefetching with incremental aggregation; [Hetero]
  * §IV that index retrieval and attention be pipelined to hide retrieval
- * latency. For bf16 keys of H_i*d_c = 1024 features and the decode attention
- * shapes (head_dim 128, block_size a multiple of 64, at most 16 query heads per
- * KV head) the step is ONE persistent launch: CTAs claim scoring chunks from a
- * global counter, the last chunk of a row selects the row's blocks and
- * publishes it, and CTAs then claim attention splits of published rows while
- * later rows are still being scored; the last split of a (row, KV head) pair
- * to finish combines the splits. Other shapes run the indexer and the
- * attention kernel back to back, each row's attention starting as soon as the
- * indexer publishes the row.
+ * latency. The indexer publishes each query row as soon as its block ids are
+ * final, and the attention kernel, launched behind it (programmatic dependent
+ * launch), starts on a row as soon as that row is published, while later rows
+ * are still being scored.
  * Arguments are those of the two calls; k_c's nb_max must equal the table's
  * max_blocks and all floating inputs share one dtype. The workspace holds the
  * scratch, per-row publication flags and the per-call counters: zero-fill it
@@ -394,14 +389,6 @@ LCI_API lci_status lci_sparse_decode_workspace_size(int32_t batch, int32_t S, in
  * the next. A flag left set by an earlier call is never taken for a new
  * publication. Calls sharing a workspace must not overlap in time.
  */
-/*
- * How many kernel launches lci_sparse_decode makes for these sizes: 1 (the
- * one-launch persistent step) or 2 (indexer, then attention), assuming
- * 16-byte aligned pools.
- */
-LCI_API lci_status lci_sparse_decode_launches(int32_t H_i, int32_t d_c, int32_t H_q,
-                                              const lci_block_table* table, int32_t* launches);
-
 LCI_API lci_status lci_sparse_decode(const void* q_c, const void* k_c, lci_dtype dtype,
                                      int32_t batch, int32_t S, int32_t H_i, int32_t d_c,
                                      int32_t nb_max, const int32_t* d_ctx_len,
@@ -475,6 +462,32 @@ LCI_API lci_status lci_gated_state_scan(const void* q, const void* k, const void
  * wait ran out since the last call; otherwise LCI_ERR_DEVICE_BOUNDS when a
  * device bounds check fired. lci_last_error() lists every flag that was set.
  */
+/*
+ * The same decode step as lci_sparse_decode in ONE persistent launch: about
+ * one CTA per SM claims work items from a global counter, first the scoring
+ * chunks of the query rows (the last chunk of a row to finish selects the
+ * row's blocks and publishes it), then attention splits of (row, KV head)
+ * pairs whose rows are published, while later rows are still being scored;
+ * the last split of a pair to finish combines the splits. A CTA claims
+ * attention work only after every scoring item has been claimed by a running
+ * CTA, and scoring never waits, so the launch completes whatever the
+ * residency. Same arguments, results (ids identical, outputs within the
+ * attention tolerance) and workspace as lci_sparse_decode; the workspace also
+ * keeps the per-call counters and an epoch, which every call leaves ready for
+ * the next. Supported (else LCI_ERR_UNSUPPORTED): bf16, H_i*d_c = 1024,
+ * head_dim 128, block_size a multiple of 64, at most 16 query heads per KV
+ * head, 16-byte aligned pools.
+ */
+LCI_API lci_status lci_sparse_decode_persistent(const void* q_c, const void* k_c, lci_dtype dtype,
+                                                int32_t batch, int32_t S, int32_t H_i,
+                                                int32_t d_c, int32_t nb_max,
+                                                const int32_t* d_ctx_len, const int32_t* d_q_start,
+                                                int32_t topk, const void* q, int32_t H_q,
+                                                const void* k_pool, const void* v_pool,
+                                                const lci_block_table* table, float scale,
+                                                int32_t* d_ids, void* out, void* workspace,
+                                                size_t workspace_bytes, void* stream);
+
 LCI_API lci_status lci_get_device_status(void* stream);
 
 #ifdef __cplusplus

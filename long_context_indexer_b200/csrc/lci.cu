@@ -1092,15 +1092,6 @@ lci_status lci_sparse_decode_workspace_size(int32_t batch, int32_t S, int32_t H_
     return ok();
 }
 
-lci_status lci_sparse_decode_launches(int32_t H_i, int32_t d_c, int32_t H_q,
-                                      const lci_block_table* table, int32_t* launches) {
-    if (!table || !launches) return fail(LCI_ERR_INVALID_ARG, "sparse_decode_launches: null argument");
-    if (H_i <= 0 || d_c <= 0 || H_q <= 0 || H_q % table->num_kv_heads != 0)
-        return fail(LCI_ERR_INVALID_ARG, "sparse_decode_launches: bad sizes");
-    *launches = fused_decode_fits(table->dtype, H_i * d_c, table, H_q, nullptr, nullptr) ? 1 : 2;
-    return ok();
-}
-
 lci_status launch_decode_fused(const void* q_c, const void* k_c, int32_t batch, int32_t S,
                                int32_t nb_max, const int32_t* ctx_len, const int32_t* q_start,
                                int32_t topk, const void* q, int32_t H_q, const void* k_pool,
@@ -1146,12 +1137,14 @@ lci_status launch_decode_fused(const void* q_c, const void* k_c, int32_t batch, 
     return check_launch("sparse_decode");
 }
 
-lci_status lci_sparse_decode(const void* q_c, const void* k_c, lci_dtype dtype, int32_t batch,
-                             int32_t S, int32_t H_i, int32_t d_c, int32_t nb_max,
-                             const int32_t* d_ctx_len, const int32_t* d_q_start, int32_t topk,
-                             const void* q, int32_t H_q, const void* k_pool, const void* v_pool,
-                             const lci_block_table* table, float scale, int32_t* d_ids, void* out,
-                             void* workspace, size_t workspace_bytes, void* stream) {
+static lci_status sparse_decode_impl(const void* q_c, const void* k_c, lci_dtype dtype,
+                                     int32_t batch, int32_t S, int32_t H_i, int32_t d_c,
+                                     int32_t nb_max, const int32_t* d_ctx_len,
+                                     const int32_t* d_q_start, int32_t topk, const void* q,
+                                     int32_t H_q, const void* k_pool, const void* v_pool,
+                                     const lci_block_table* table, float scale, int32_t* d_ids,
+                                     void* out, void* workspace, size_t workspace_bytes,
+                                     void* stream, bool one_launch) {
     if (!q_c || !k_c || !d_ctx_len || !d_q_start || !d_ids || !q || !k_pool || !v_pool || !out)
         return fail(LCI_ERR_INVALID_ARG, "sparse_decode: null pointer argument");
     lci_status st = check_index_args(batch, S, H_i, d_c, nb_max, topk, dtype);
@@ -1166,7 +1159,11 @@ lci_status lci_sparse_decode(const void* q_c, const void* k_c, lci_dtype dtype, 
     if (!aligned16(q_c) || !aligned16(k_c))
         return fail(LCI_ERR_INVALID_ARG, "sparse_decode: q_c and k_c must be 16-byte aligned");
     const int K = H_i * d_c;
-    const bool fused = fused_decode_fits(dtype, K, table, H_q, k_pool, v_pool);
+    const bool fused = one_launch;
+    if (one_launch && !fused_decode_fits(dtype, K, table, H_q, k_pool, v_pool))
+        return fail(LCI_ERR_UNSUPPORTED, "sparse_decode_persistent: needs bf16 keys of H_i*d_c = "
+                    "1024, bf16 pools of head_dim 128, block_size a multiple of 64, at most 16 "
+                    "query heads per KV head and 16-byte aligned pools");
     const DecodePlan pl = plan_decode(batch, S, K, nb_max, dtype_size(dtype), topk, table, H_q,
                                       fused);
     if (!workspace || workspace_bytes < pl.bytes ||
@@ -1206,6 +1203,30 @@ lci_status lci_sparse_decode(const void* q_c, const void* k_c, lci_dtype dtype, 
                                   d_q_start, scale, out, cs);
     return launch_attn_simt<__nv_bfloat16>(q, batch, S, H_q, k_pool, v_pool, table, d_ids, topk,
                                            d_ctx_len, d_q_start, scale, out, cs);
+}
+
+lci_status lci_sparse_decode(const void* q_c, const void* k_c, lci_dtype dtype, int32_t batch,
+                             int32_t S, int32_t H_i, int32_t d_c, int32_t nb_max,
+                             const int32_t* d_ctx_len, const int32_t* d_q_start, int32_t topk,
+                             const void* q, int32_t H_q, const void* k_pool, const void* v_pool,
+                             const lci_block_table* table, float scale, int32_t* d_ids, void* out,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+    return sparse_decode_impl(q_c, k_c, dtype, batch, S, H_i, d_c, nb_max, d_ctx_len, d_q_start,
+                              topk, q, H_q, k_pool, v_pool, table, scale, d_ids, out, workspace,
+                              workspace_bytes, stream, false);
+}
+
+lci_status lci_sparse_decode_persistent(const void* q_c, const void* k_c, lci_dtype dtype,
+                                        int32_t batch, int32_t S, int32_t H_i, int32_t d_c,
+                                        int32_t nb_max, const int32_t* d_ctx_len,
+                                        const int32_t* d_q_start, int32_t topk, const void* q,
+                                        int32_t H_q, const void* k_pool, const void* v_pool,
+                                        const lci_block_table* table, float scale, int32_t* d_ids,
+                                        void* out, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+    return sparse_decode_impl(q_c, k_c, dtype, batch, S, H_i, d_c, nb_max, d_ctx_len, d_q_start,
+                              topk, q, H_q, k_pool, v_pool, table, scale, d_ids, out, workspace,
+                              workspace_bytes, stream, true);
 }
 
 lci_status lci_get_device_status(void* stream) {

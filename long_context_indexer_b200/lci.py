@@ -56,7 +56,9 @@ SIGNATURES = {
     "lci_sparse_attn_pipelined": (_st, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp,
                                         _f32, _vp, _vp, _vp]),
     "lci_set_wait_limit_ns": (_st, [ctypes.c_uint64]),
-    "lci_sparse_decode_launches": (_st, [_i32, _i32, _i32, _vp, ctypes.POINTER(_i32)]),
+    "lci_sparse_decode_persistent": (_st, [_vp, _vp, _st, _i32, _i32, _i32, _i32, _i32, _vp, _vp,
+                                           _i32, _vp, _i32, _vp, _vp, _vp, _f32, _vp, _vp, _vp,
+                                           _sz, _vp]),
     "lci_gated_state_scan": (_st, [_vp, _vp, _vp, _st, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                    _i32, _vp, _vp]),
     "lci_block_scores_at": (_st, [_vp, _vp, _st, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _vp,
@@ -330,19 +332,11 @@ def sparse_decode_workspace_size(B, S, H_i, d_c, topk, H_q, table: BlockTable) -
     return n
 
 
-def sparse_decode_launches(H_i: int, d_c: int, H_q: int, table: BlockTable) -> int:
-    """Kernel launches of one sparse_decode call: 1 (one persistent launch) or 2."""
-    n = ctypes.c_int32()
-    _check(load_library().lci_sparse_decode_launches(H_i, d_c, H_q, table.handle, ctypes.byref(n)),
-           "lci_sparse_decode_launches")
-    return n.value
-
-
 def sparse_decode(q_c: torch.Tensor, k_c: torch.Tensor, ctx_len: torch.Tensor,
                   q_start: torch.Tensor, topk: int, q: torch.Tensor, k_pool: torch.Tensor,
                   v_pool: torch.Tensor, table: BlockTable, scale: float = 0.0,
                   ids: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-                  ws: Optional[torch.Tensor] = None, stream=None):
+                  ws: Optional[torch.Tensor] = None, stream=None, persistent: bool = False):
     """index_select + sparse_attn in one call (rows attended as they are selected).
 
     Returns (ids [B, S, topk] int32, out [B, S, H_q, hd])."""
@@ -362,14 +356,14 @@ def sparse_decode(q_c: torch.Tensor, k_c: torch.Tensor, ctx_len: torch.Tensor,
     if ws is None:
         ws = workspace(q_c.device, need, f"sparse_decode:{B}x{S}x{nb_max}:{H_i * d_c}:{topk}:"
                                          f"{H_q}x{table.num_kv_heads}x{table.block_size}")
-    _check(load_library().lci_sparse_decode(
+    name = "lci_sparse_decode_persistent" if persistent else "lci_sparse_decode"
+    _check(getattr(load_library(), name)(
         _dev(q_c, "q_c", None, 4), _dev(k_c, "k_c", q_c.dtype, 4), _dtype_code(q_c), B, S, H_i,
         d_c, nb_max, _dev(ctx_len, "ctx_len", torch.int32, 1),
         _dev(q_start, "q_start", torch.int32, 1), topk, _dev(q, "q", q_c.dtype, 4), H_q,
         _dev(k_pool, "k_pool", q_c.dtype), _dev(v_pool, "v_pool", q_c.dtype), table.handle,
         float(scale), _dev(ids, "ids", torch.int32, 3), _dev(out, "out", q_c.dtype, 4),
-        _dev(ws, "workspace"), ws.numel() * ws.element_size(), _stream(stream)),
-        "lci_sparse_decode")
+        _dev(ws, "workspace"), ws.numel() * ws.element_size(), _stream(stream)), name)
     return ids, out
 
 
@@ -562,6 +556,53 @@ def get_wait_limit_ns() -> int:
     v = ctypes.c_uint64()
     _check(load_library().lci_get_wait_limit_ns(ctypes.byref(v)), "lci_get_wait_limit_ns")
     return v.value
+
+
+class SparseDecodeStep:
+    """A decode step prepared once, for a loop that calls it every step: the
+    tensors are checked and their device pointers taken here, the workspace is
+    allocated, and each call makes only the lci_sparse_decode C call on the
+    given stream (the caller updates the buffers' contents between calls, e.g.
+    by copying the new tokens' queries into q_c and q)."""
+
+    def __init__(self, q_c: torch.Tensor, k_c: torch.Tensor, ctx_len: torch.Tensor,
+                 q_start: torch.Tensor, topk: int, q: torch.Tensor, k_pool: torch.Tensor,
+                 v_pool: torch.Tensor, table: BlockTable, scale: float = 0.0,
+                 ids: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                 ws: Optional[torch.Tensor] = None, stream=None, persistent: bool = False):
+        B, S, H_i, d_c = q_c.shape
+        nb_max = k_c.shape[1]
+        H_q = q.shape[2]
+        if tuple(q.shape[:2]) != (B, S):
+            raise ValueError("lci: q must be [B, S, H_q, hd] with q_c's B and S")
+        if tuple(k_pool.shape) != (table.num_pages, table.num_kv_heads, table.block_size,
+                                   table.head_dim) or v_pool.shape != k_pool.shape:
+            raise ValueError("lci: pools do not match the block table")
+        self.ids = torch.empty((B, S, topk), dtype=torch.int32, device=q_c.device) \
+            if ids is None else ids
+        self.out = torch.empty_like(q) if out is None else out
+        need = sparse_decode_workspace_size(B, S, H_i, d_c, topk, H_q, table)
+        self.ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=q_c.device) \
+            if ws is None else ws
+        if self.ws.numel() * self.ws.element_size() < need:
+            raise ValueError("lci: workspace too small")
+        self._keep = (q_c, k_c, ctx_len, q_start, q, k_pool, v_pool, table)
+        self._name = "lci_sparse_decode_persistent" if persistent else "lci_sparse_decode"
+        self._fn = getattr(load_library(), self._name)
+        self._stream = _stream(stream)
+        self._args = (
+            _dev(q_c, "q_c", None, 4), _dev(k_c, "k_c", q_c.dtype, 4), _dtype_code(q_c), B, S, H_i,
+            d_c, nb_max, _dev(ctx_len, "ctx_len", torch.int32, 1),
+            _dev(q_start, "q_start", torch.int32, 1), topk, _dev(q, "q", q_c.dtype, 4), H_q,
+            _dev(k_pool, "k_pool", q_c.dtype), _dev(v_pool, "v_pool", q_c.dtype), table.handle,
+            ctypes.c_float(scale), _dev(self.ids, "ids", torch.int32, 3),
+            _dev(self.out, "out", q_c.dtype, 4), _dev(self.ws, "workspace"),
+            ctypes.c_size_t(self.ws.numel() * self.ws.element_size()), self._stream)
+
+    def __call__(self) -> None:
+        rc = self._fn(*self._args)
+        if rc != LCI_OK:
+            _check(rc, self._name)
 
 
 def get_device_status(stream=None) -> None:

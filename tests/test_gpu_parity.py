@@ -254,12 +254,15 @@ def test_unwritten_cache_slots_never_reach_the_output(S, q0):
     assert_out_close(out.reshape(-1, cfg.H_q, cfg.hd), ref_out, torch.bfloat16, "nan-tail")
 
 
+@pytest.mark.parametrize("persistent", [False, True])
 @pytest.mark.parametrize("name", ["decode", "small", "small_f32", "1m_decode"])
-def test_fused_decode_step_matches_two_calls_and_oracle(name):
+def test_fused_decode_step_matches_two_calls_and_oracle(name, persistent):
     """lci_sparse_decode (rows attended as soon as they are selected) gives the
     block ids and outputs of index_select + sparse_attn, call after call."""
     cfg = {"decode": CONFIGS["decode"], "1m_decode": CONFIGS["1m_decode"], "small": SMALL,
            "small_f32": SMALL.replace(dtype="f32")}[name]
+    if persistent and name.startswith("small"):
+        pytest.skip("the one-launch step takes 1024-feature bf16 keys")
     w = generate(cfg)
     d = upload(w)
     _, ids2, out2 = run_gpu(cfg, d)
@@ -267,7 +270,7 @@ def test_fused_decode_step_matches_two_calls_and_oracle(name):
     first = None
     for _ in range(3):  # the per-call state must reset between calls
         ids, out = lci.sparse_decode(d["q_c"], d["k_c"], d["ctx_len"], d["q_start"], cfg.topk,
-                                     d["q"], d["k_pool"], d["v_pool"], bt)
+                                     d["q"], d["k_pool"], d["v_pool"], bt, persistent=persistent)
         torch.cuda.synchronize()
         lci.get_device_status()
         assert torch.equal(ids, ids2)
@@ -308,11 +311,13 @@ def test_decode_attention_deep_ring_uneven_splits(B, H_kv):
     assert torch.equal(ids.cpu().reshape(-1, cfg.topk), ref_ids)
     assert_out_close(out.reshape(-1, cfg.H_q, cfg.hd), ref_out, cfg.torch_dtype, "deep ring")
     bt = lci.create_block_table(d["block_table"], d["k_pool"])
-    ids_f, out_f = lci.sparse_decode(d["q_c"], d["k_c"], d["ctx_len"], d["q_start"], cfg.topk,
-                                     d["q"], d["k_pool"], d["v_pool"], bt)
-    torch.cuda.synchronize()
-    assert torch.equal(ids_f, ids)
-    assert_out_close(out_f.reshape(-1, cfg.H_q, cfg.hd), ref_out, cfg.torch_dtype, "one call")
+    for persistent in (False, True):
+        ids_f, out_f = lci.sparse_decode(d["q_c"], d["k_c"], d["ctx_len"], d["q_start"], cfg.topk,
+                                         d["q"], d["k_pool"], d["v_pool"], bt,
+                                         persistent=persistent)
+        torch.cuda.synchronize()
+        assert torch.equal(ids_f, ids)
+        assert_out_close(out_f.reshape(-1, cfg.H_q, cfg.hd), ref_out, cfg.torch_dtype, "one call")
 
 
 @pytest.mark.parametrize("name", ["decode", "long", "1m_decode"])
@@ -333,12 +338,35 @@ def test_one_launch_decode_step_over_many_calls(name):
     ref_ids_o, ref_out_o = oracle_rows(other, wo)
     for _ in range(10):
         ids, out = lci.sparse_decode(d["q_c"], d["k_c"], d["ctx_len"], d["q_start"], cfg.topk,
-                                     d["q"], d["k_pool"], d["v_pool"], bt)
+                                     d["q"], d["k_pool"], d["v_pool"], bt, persistent=True)
         ids_o, out_o = lci.sparse_decode(do["q_c"], do["k_c"], do["ctx_len"], do["q_start"],
-                                         other.topk, do["q"], do["k_pool"], do["v_pool"], bto)
+                                         other.topk, do["q"], do["k_pool"], do["v_pool"], bto,
+                                         persistent=True)
     torch.cuda.synchronize()
     lci.get_device_status()
     assert torch.equal(ids.cpu().reshape(-1, cfg.topk), ref_ids)
     assert_out_close(out.reshape(-1, cfg.H_q, cfg.hd), ref_out, torch.bfloat16, name)
     assert torch.equal(ids_o.cpu().reshape(-1, other.topk), ref_ids_o)
     assert_out_close(out_o.reshape(-1, other.H_q, other.hd), ref_out_o, torch.bfloat16, "other")
+
+
+def test_prepared_decode_step_matches_the_plain_call():
+    """SparseDecodeStep takes its pointers once and launches with them every
+    call; after the inputs are overwritten in place it sees the new values."""
+    cfg = CONFIGS["decode"].replace(B=8, ctx=8192, q_start=8191, spare_pages=8)
+    w = generate(cfg)
+    d = upload(w)
+    bt = lci.create_block_table(d["block_table"], d["k_pool"])
+    step = lci.SparseDecodeStep(d["q_c"], d["k_c"], d["ctx_len"], d["q_start"], cfg.topk, d["q"],
+                                d["k_pool"], d["v_pool"], bt)
+    for seed in (0, 1):
+        if seed:
+            d["q_c"].copy_(torch.flip(d["q_c"], dims=[0]))
+            d["q"].copy_(torch.flip(d["q"], dims=[0]))
+        step()
+        ids, out = lci.sparse_decode(d["q_c"], d["k_c"], d["ctx_len"], d["q_start"], cfg.topk,
+                                     d["q"], d["k_pool"], d["v_pool"], bt)
+        torch.cuda.synchronize()
+        lci.get_device_status()
+        assert torch.equal(step.ids, ids)
+        assert torch.equal(step.out, out)
