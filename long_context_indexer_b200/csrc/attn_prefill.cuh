@@ -124,6 +124,18 @@ __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// 64 consecutive 32-bit columns of this thread's TMEM lane, one load.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]), "+r"(r[32]), "+r"(r[33]), "+r"(r[34]), "+r"(r[35]), "+r"(r[36]), "+r"(r[37]), "+r"(r[38]), "+r"(r[39]), "+r"(r[40]), "+r"(r[41]), "+r"(r[42]), "+r"(r[43]), "+r"(r[44]), "+r"(r[45]), "+r"(r[46]), "+r"(r[47]), "+r"(r[48]), "+r"(r[49]), "+r"(r[50]), "+r"(r[51]), "+r"(r[52]), "+r"(r[53]), "+r"(r[54]), "+r"(r[55]), "+r"(r[56]), "+r"(r[57]), "+r"(r[58]), "+r"(r[59]), "+r"(r[60]), "+r"(r[61]), "+r"(r[62]), "+r"(r[63])
+                 :
+                 : "memory");
+}
+
 // Byte offset of (row r, 16-byte chunk c of its 128 dims) in a 128-row tile
 // stored as two 64-dim halves with the 128-byte swizzle.
 __device__ __forceinline__ uint32_t pfa_off(int r, int c) {
@@ -441,27 +453,24 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
             const bool waited = mbar_wait(&sfull[i & 1], (i >> 1) & 1);
             const int my_ok = waited && !*s_abort;
             tc_fence_after();
-            uint32_t sv[2][32];
+            uint32_t sv[64];
             float mx = -INFINITY;
             const bool warp_any = __any_sync(0xffffffffu, nval > 0);
             if (warp_any) {
-                tmem_ld32(lane_addr + kColS + (i & 1) * 128 + hf * 64, sv[0]);
-                tmem_ld32(lane_addr + kColS + (i & 1) * 128 + hf * 64 + 32, sv[1]);
-                if (nval == 64) {
+                tmem_ld64(lane_addr + kColS + (i & 1) * 128 + hf * 64, sv);
+                if (nval < 64) {
 #pragma unroll
-                    for (int ch = 0; ch < 2; ++ch)
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sv[ch][e]));
-                } else {
-#pragma unroll
-                    for (int ch = 0; ch < 2; ++ch)
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const bool ok = ch * 32 + e < nval;
-                            sv[ch][e] = ok ? sv[ch][e] : __float_as_uint(-INFINITY);
-                            mx = fmaxf(mx, __uint_as_float(sv[ch][e]));
-                        }
+                    for (int e = 0; e < 64; ++e)
+                        sv[e] = e < nval ? sv[e] : __float_as_uint(-INFINITY);
                 }
+                // eight independent running maxima, then a tree
+                float pm[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) pm[k] = __uint_as_float(sv[k]);
+#pragma unroll
+                for (int e = 8; e < 64; ++e) pm[e & 7] = fmaxf(pm[e & 7], __uint_as_float(sv[e]));
+                mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                           fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
             }
             // the row maximum of the stage (raw scores; the scale is positive),
             // and whether both halves may go on: one decision for the pair of
@@ -499,28 +508,28 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
                 }
                 l *= corr;
             }
-            // P = 2^(s*c - m) as bf16 pairs into this stage's P buffer
+            // P = 2^(s*c - m) as bf16 pairs; it overwrites the S buffer's first
+            // 64 columns (both halves have read their S columns: the barrier above)
             const float neg_m = -m_ref;
+            uint32_t pk[32];
+            if (nval > 0) {
+                float ps[8];
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-                uint32_t pk[16];
-                if (nval > 0) {
+                for (int k = 0; k < 8; ++k) ps[k] = 0.f;
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        // masked entries hold -inf: 2^-inf = 0
-                        const float a = fast_exp2(fmaf(__uint_as_float(sv[ch][2 * e]), scale_log2, neg_m));
-                        const float bb = fast_exp2(fmaf(__uint_as_float(sv[ch][2 * e + 1]), scale_log2, neg_m));
-                        l += a + bb;
-                        pk[e] = pack_bf16x2(a, bb);
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                for (int e = 0; e < 32; ++e) {
+                    // masked entries hold -inf: 2^-inf = 0
+                    const float a = fast_exp2(fmaf(__uint_as_float(sv[2 * e]), scale_log2, neg_m));
+                    const float bb = fast_exp2(fmaf(__uint_as_float(sv[2 * e + 1]), scale_log2, neg_m));
+                    ps[e & 7] += a + bb;
+                    pk[e] = pack_bf16x2(a, bb);
                 }
-                // P overwrites the S buffer's first 64 columns: both halves
-                // have read their S columns (the barrier above)
-                tmem_st16(lane_addr + kColS + (i & 1) * 128 + hf * 32 + ch * 16, pk);
+                l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) pk[e] = 0u;
             }
+            tmem_st32(lane_addr + kColS + (i & 1) * 128 + hf * 32, pk);
             tmem_wait_st();
             // V rows of an absent unit and of tokens past the context length
             // must be zero before the P V MMA reads them (this thread: token row
