@@ -208,6 +208,7 @@ class Pipeline:
         nd = lci.sparse_decode_workspace_size(cfg.B, cfg.S, cfg.H_i, cfg.d_c, cfg.topk, cfg.H_q,
                                               self.bt)
         self.ws_d = torch.zeros(max(nd, 256), dtype=torch.uint8, device=device)
+        self.ws_p = torch.zeros(max(nd, 256), dtype=torch.uint8, device=device)
         self.one_call = cfg.S == 1 and not cfg.compress
         self.launches_per_step = (1 if cfg.compress else 0) + 2
 
@@ -223,6 +224,7 @@ class Pipeline:
         other.ws_i = torch.zeros_like(self.ws_i)
         other.ws_a = torch.zeros_like(self.ws_a)
         other.ws_d = torch.zeros_like(self.ws_d)
+        other.ws_p = torch.zeros_like(self.ws_p)
         other.launches_per_step = self.launches_per_step
         other.one_call = self.one_call
         return other
@@ -284,6 +286,13 @@ class Pipeline:
         d, c = self.d, self.cfg
         self.lci.sparse_attn(d["q"], d["k_pool"], d["v_pool"], self.bt, self.ids, d["ctx_len"],
                              d["q_start"], out=self.out, ws=self.ws_a)
+
+    def step_persistent(self):
+        """The same decode step as one persistent launch."""
+        d, c = self.d, self.cfg
+        self.lci.sparse_decode(d["q_c"], self.k_c, d["ctx_len"], d["q_start"], c.topk, d["q"],
+                               d["k_pool"], d["v_pool"], self.bt, ids=self.ids, out=self.out,
+                               ws=self.ws_p, persistent=True)
 
     def step(self):
         c = self.cfg
@@ -456,7 +465,15 @@ def measure(cfg, steps, warmup, device, rank=0, seed_offset=0, with_e2e=True):
     t_step = time_graph(g_step, n_rep, warm) / R
     t_idx = time_graph(g_idx, n_rep, warm) / R
     t_att = time_graph(g_att, n_rep, warm) / R
+    t_pers = None
+    if pipe.one_call and cfg.H_i * cfg.d_c == 1024 and cfg.dtype == "bf16":
+        for p in reps.pipes:
+            p.step_persistent()
+        g_pers = capture([p.step_persistent for p in reps.pipes])
+        t_pers = time_graph(g_pers, n_rep, warm) / R
+        del g_pers
     res = {"pipe": pipe, "t_index_ms": t_idx, "t_attn_ms": t_att, "t_step_ms": t_step,
+           "t_persistent_ms": t_pers,
            "t_total_ms": t_step * steps, "alg": alg, "replicas": R,
            "cycle_mb": reps.cycle_bytes / 2**20, "launches": pipe.launches_per_step * steps}
     if with_e2e:
@@ -511,6 +528,7 @@ def config_entry(cfg, r, pk):
     ti, ta = r["t_index_ms"] * 1e-3, r["t_attn_ms"] * 1e-3
     e = {
         "ms_step": r["t_step_ms"], "ms_index": r["t_index_ms"], "ms_attn": r["t_attn_ms"],
+        "ms_step_one_launch": r["t_persistent_ms"],
         "tokens_per_s": rows / (r["t_step_ms"] * 1e-3),
         "index_gbs": a["index_bytes"] / ti / 1e9,
         "index_tflops": a["index_flops"] / ti / 1e12,
@@ -674,7 +692,8 @@ def main():
                           "frac": step_gbs / pk["hbm_gbs"]},
         "kernels_ms": {k: v["ms"] for k, v in kernels.items()},
         "itemized_ms": {"index_select alone": res["t_index_ms"],
-                        "sparse_attn alone": res["t_attn_ms"]},
+                        "sparse_attn alone": res["t_attn_ms"],
+                        "one-launch persistent step": res["t_persistent_ms"]},
         "e2e": {"value": e2e_value, "unit": "tokens/s", **res["e2e_bytes"]},
         "gpu_launches": res["launches"],
         "clocks": clk.summary(),

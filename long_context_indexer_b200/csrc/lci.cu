@@ -1037,7 +1037,9 @@ struct DecodePlan {
     IndexPlan ix;
     bool fused;                 // the one-launch persistent kernel
     int nsplit;                 // attention splits per (row, KV head) pair (fused)
-    size_t off_ready, off_split, off_sync, off_part, bytes;
+    size_t off_ready;           // publication flags of the two-kernel form (0 / 1)
+    size_t off_pready;          // publication flags of the one-launch form (call epochs)
+    size_t off_split, off_sync, off_part, bytes;
 };
 
 // The one-launch kernel covers bf16 keys of 1024 features (2 KiB per block)
@@ -1065,7 +1067,10 @@ DecodePlan plan_decode(int32_t batch, int32_t S, int32_t K, int32_t nb_max, size
         if (want < 1) want = 1;
         const int per = (int)((nunits + want - 1) / want);
         d.nsplit = (nunits + per - 1) / per;
-        d.off_split = end;
+        // the one-launch form keeps its own flags: the two-kernel form leaves
+        // its flags at 1, which is an epoch value the one-launch form waits for
+        d.off_pready = end;
+        d.off_split = d.off_pready + align_up(rows * sizeof(unsigned int));
         d.off_sync = d.off_split + align_up((size_t)pairs * sizeof(unsigned int));
         d.off_part = d.off_sync + kAlign;
         end = d.off_part + align_up((size_t)pairs * d.nsplit * lci::fdec::kPartFloats * sizeof(float));
@@ -1132,7 +1137,7 @@ lci_status launch_decode_fused(const void* q_c, const void* k_c, int32_t batch, 
         static_cast<const __nv_bfloat16*>(q), t->d_table, t->num_pages, t->num_kv_heads, H_q,
         scale_log2, static_cast<__nv_bfloat16*>(out), pl.nsplit,
         reinterpret_cast<float*>(w + pl.off_part), reinterpret_cast<unsigned int*>(w + pl.off_split),
-        reinterpret_cast<unsigned int*>(w + pl.off_ready), reinterpret_cast<unsigned int*>(w + pl.off_sync),
+        reinterpret_cast<unsigned int*>(w + pl.off_pready), reinterpret_cast<unsigned int*>(w + pl.off_sync),
         rows);
     return check_launch("sparse_decode");
 }

@@ -370,3 +370,25 @@ def test_prepared_decode_step_matches_the_plain_call():
         lci.get_device_status()
         assert torch.equal(step.ids, ids)
         assert torch.equal(step.out, out)
+
+
+def test_both_decode_forms_share_one_workspace():
+    """The two-kernel and the one-launch decode forms alternate on one
+    workspace: neither takes the other's publication flags for its own."""
+    cfg = CONFIGS["decode"].replace(B=20, H_kv=2, ctx=6000, q_start=5999, topk=11, spare_pages=8)
+    w = generate(cfg)
+    d = upload(w)
+    ref_ids, ref_out = oracle_rows(cfg, w)
+    bt = lci.create_block_table(d["block_table"], d["k_pool"])
+    need = lci.sparse_decode_workspace_size(cfg.B, cfg.S, cfg.H_i, cfg.d_c, cfg.topk, cfg.H_q, bt)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for persistent in (False, True, True, False, True):
+        ids = torch.full((cfg.B, 1, cfg.topk), 12345, dtype=torch.int32, device="cuda")
+        ids, out = lci.sparse_decode(d["q_c"], d["k_c"], d["ctx_len"], d["q_start"], cfg.topk,
+                                     d["q"], d["k_pool"], d["v_pool"], bt, ids=ids, ws=ws,
+                                     persistent=persistent)
+        torch.cuda.synchronize()
+        lci.get_device_status()
+        assert torch.equal(ids.cpu().reshape(-1, cfg.topk), ref_ids), persistent
+        assert_out_close(out.reshape(-1, cfg.H_q, cfg.hd), ref_out, cfg.torch_dtype,
+                         f"persistent={persistent}")
