@@ -44,7 +44,7 @@ constexpr int kChunkBytes = 32768;
 constexpr int kRingBytes = kStages * dec::kStageBytes;  // 192 KiB
 constexpr int kOffSel = kRingBytes;
 constexpr int kOffBar = kOffSel + (int)((sizeof(SelectSmem) + 1023) / 1024 * 1024);
-constexpr int kSmemBytes = kOffBar + 512 + 1024;  // barriers and control words fit in 512 bytes
+constexpr int kSmemBytes = kOffBar + 512 + 1024;
 constexpr int kPartFloats = 2 * dec::kRows + dec::kRows * dec::kHD;  // m, l, o[16][128]
 // sync words in the workspace
 enum { kEpoch = 0, kClaim = 1, kExit = 2 };
@@ -102,20 +102,11 @@ __global__ void __launch_bounds__(fdec::kThreads, 1) sparse_decode_fused_kernel(
     __syncthreads();
 
     // ======================= scoring (A1 + A2) =======================
-    // Thread 0 claims scoring items kBufs at a time (one atomic per batch) and
-    // issues their bulk copies into free buffers; claimed items at or past
-    // items_a are attention items of this CTA, kept in s_own. A row's arrival
-    // on its counter is checked one item later, so the atomic's round trip
-    // overlaps the next item's work; the row's select then runs.
-    // s_ctl[0]: tail, s_ctl[1]: more scoring claims, s_ctl[2]: a row to select
-    // (or -1), s_ctl[6]: number of own attention items, s_own[..]: those items
-    int* s_own = s_ctl + 8 + 1;  // [kBufs], after s_max
+    // s_ctl[0]: items claimed and loading (tail), s_ctl[1]: the first claimed
+    // attention item (or items_total), s_ctl[2]: the select flag
     int head = 0, tail = 0;
     bool more = true;
-    int n_own = 0;
-    int pend_row = -1;           // thread 0: the row whose arrival is pending
-    unsigned pend_prev = 0u;     // thread 0: the counter value it returned
-    int batch_next = 0, batch_end = 0;  // thread 0: unissued claimed items
+    int first_b = items_total;
     auto chunk_range = [&](int w, int& row, int& chunk, int& j0, int& j1, int& vis) {
         row = w / nchunks;
         chunk = w - row * nchunks;
@@ -126,21 +117,12 @@ __global__ void __launch_bounds__(fdec::kThreads, 1) sparse_decode_fused_kernel(
     };
     for (;;) {
         if (tid == 0) {
-            // the pending row's arrival: was it the row's last chunk?
-            int sel_row = -1;
-            if (pend_row >= 0 && pend_prev == (unsigned)(nchunks - 1)) sel_row = pend_row;
-            pend_row = -1;
-            while (tail - head < fdec::kBufs && (batch_next < batch_end || more)) {
-                if (batch_next == batch_end) {
-                    const int w0 = (int)atomicAdd(sync_words + fdec::kClaim, (unsigned)fdec::kBufs);
-                    batch_next = w0;
-                    batch_end = w0 + fdec::kBufs;
-                    if (batch_end >= items_a) more = false;
-                }
-                const int w = batch_next++;
+            while (more && tail - head < fdec::kBufs) {
+                const int w = (int)atomicAdd(sync_words + fdec::kClaim, 1u);
                 if (w >= items_a) {
-                    if (w < items_total) s_own[n_own++] = w;
-                    continue;
+                    more = false;
+                    first_b = w;
+                    break;
                 }
                 const int slot = tail % fdec::kBufs;
                 s_item[slot] = w;
@@ -160,27 +142,13 @@ __global__ void __launch_bounds__(fdec::kThreads, 1) sparse_decode_fused_kernel(
                 ++tail;
             }
             s_ctl[0] = tail;
-            s_ctl[2] = sel_row;
-            s_ctl[6] = n_own;
+            s_ctl[1] = more ? -1 : first_b;
         }
         __syncthreads();
         tail = s_ctl[0];
-        const int sel_row = s_ctl[2];
-        if (sel_row >= 0) {
-            // the row's last chunk arrived: select its blocks and publish it
-            __threadfence();
-            if (tid == 0) row_counter[sel_row] = 0u;
-            const int b = sel_row / S, s = sel_row - b * S;
-            const int vis = visible_blocks((long long)__ldg(&q_start[b]) + s, __ldg(&ctx_len[b]), bs,
-                                           nb_max);
-            cta_topk_select<fdec::kThreads>(scores + (size_t)sel_row * nb_max,
-                                            chunk_max + (size_t)sel_row * nchunks, vis,
-                                            chunk_blocks, topk, ids + (size_t)sel_row * topk, sel);
-            __syncthreads();
-            if (tid == 0) {
-                __threadfence();
-                st_release_gpu(ready + sel_row, epoch);
-            }
+        if (s_ctl[1] >= 0) {
+            more = false;
+            first_b = s_ctl[1];
         }
         if (head == tail) break;
         const int slot = head % fdec::kBufs;
@@ -214,23 +182,28 @@ __global__ void __launch_bounds__(fdec::kThreads, 1) sparse_decode_fused_kernel(
                 }
             }
         }
-        __threadfence();  // this CTA's scores before its arrival on the row
         __syncthreads();  // the buffer is read; the chunk maximum is final
         ++head;
         if (tid == 0) {
             if (j0 < j1) chunk_max[(size_t)row * nchunks + chunk] = *s_max;
             __threadfence();
-            pend_prev = atomicAdd(&row_counter[row], 1u);  // checked next iteration
-            pend_row = row;
+            const unsigned prev = atomicAdd(&row_counter[row], 1u);
+            s_ctl[2] = prev == (unsigned)(nchunks - 1);
+        }
+        __syncthreads();
+        if (s_ctl[2]) {
+            // the row's last chunk: select its blocks and publish the row
+            __threadfence();
+            if (tid == 0) row_counter[row] = 0u;
+            cta_topk_select<fdec::kThreads>(row_scores, chunk_max + (size_t)row * nchunks, vis,
+                                            chunk_blocks, topk, ids + (size_t)row * topk, sel);
+            __syncthreads();
+            if (tid == 0) {
+                __threadfence();
+                st_release_gpu(ready + row, epoch);
+            }
         }
     }
-    // the first attention item: an own one, else a fresh claim
-    const int n_own_b = s_ctl[6];
-    __syncthreads();
-    if (tid == 0)
-        s_ctl[5] = n_own_b > 0 ? s_own[0] : (int)atomicAdd(sync_words + fdec::kClaim, 1u);
-    __syncthreads();
-    const int first_b = s_ctl[5];
 
     // ======================= attention (A3 + A4) =======================
     // The scoring buffers were read by generic loads; the ring is written by
@@ -240,7 +213,6 @@ __global__ void __launch_bounds__(fdec::kThreads, 1) sparse_decode_fused_kernel(
     const int g8 = lane >> 2, q4 = lane & 3;
     int it_base = 0;  // ring iterations so far (phases continue across items)
     int w = first_b;
-    int own_i = 1;               // next own attention item
     float* wo = reinterpret_cast<float*>(smem);           // combine scratch (ring is idle)
     constexpr int kSlots = 64, kElems = kSlots * 32;
     float* wm = wo + kConsumers * kElems;
@@ -251,9 +223,7 @@ __global__ void __launch_bounds__(fdec::kThreads, 1) sparse_decode_fused_kernel(
     while (w < items_total) {
         // claim the next item now: the atomic's round trip overlaps this item
         int next_w = 0;
-        if (tid == 0)
-            next_w = own_i < n_own_b ? s_own[own_i] : (int)atomicAdd(sync_words + fdec::kClaim, 1u);
-        ++own_i;
+        if (tid == 0) next_w = (int)atomicAdd(sync_words + fdec::kClaim, 1u);
         const int wb = w - items_a;
         const int pair = wb / nsplit, split = wb - pair * nsplit;
         const int row = pair / H_kv, g = pair - row * H_kv;
