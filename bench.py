@@ -396,46 +396,30 @@ def time_graph(g, reps, warmup):
 
 def time_e2e(pipes, steps, warmup):
     """End-to-end time (ms) of `steps` steps issued eagerly through the public
-    binding, as a user calls it: every step copies its inputs in from pinned
-    host memory, runs the library calls (argument checks, tensor-map lookups,
-    launches) and copies its results back to pinned host memory. Uploads and
-    read-backs run on a copy stream, double-buffered over the replicas, so
-    step i+1's upload overlaps step i's kernels. Device time between events on
-    the compute stream, after both streams are drained."""
-    comp = torch.cuda.current_stream()
-    copy = torch.cuda.Stream()
-    R = len(pipes)
+    binding, as a serving loop calls it: every step copies its inputs in from
+    pinned host memory, makes the library call (the prepared decode step: one C
+    call launching the kernels, tensor maps cached in the block table) and
+    copies its results back to pinned host memory, all on one stream, rotating
+    over the replicas. Device time between events on that stream."""
     for p in pipes:
         p.prepare_e2e()
-    up = [torch.cuda.Event() for _ in range(R)]
-    ran = [torch.cuda.Event() for _ in range(R)]
-    back = [torch.cuda.Event() for _ in range(R)]
+    R = len(pipes)
 
     def run(n):
         for i in range(n):
-            p, j = pipes[i % R], i % R
-            with torch.cuda.stream(copy):
-                copy.wait_event(back[j])  # this replica's previous read-back is done
-                p._d_in.copy_(p._h_in, non_blocking=True)
-                up[j].record(copy)
-            comp.wait_event(up[j])
+            p = pipes[i % R]
+            p._d_in.copy_(p._h_in, non_blocking=True)
             p.e2e_launch()
-            ran[j].record(comp)
-            with torch.cuda.stream(copy):
-                copy.wait_event(ran[j])
-                p._h_out.copy_(p._d_out, non_blocking=True)
-                back[j].record(copy)
+            p._h_out.copy_(p._d_out, non_blocking=True)
 
     run(max(warmup, R))
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if SAMPLER is not None:
         SAMPLER.active = True
-    e0.record(comp)
-    copy.wait_event(e0)
+    e0.record()
     run(steps)
-    comp.wait_stream(copy)
-    e1.record(comp)
+    e1.record()
     torch.cuda.synchronize()
     if SAMPLER is not None:
         SAMPLER.active = False

@@ -12,8 +12,10 @@
 //   update   S^T  += V_c^T K_c   A = V_c (MN-major), B = K_c (MN-major), D = S^T
 //   readout  O^T   = S^T Q_c^T   A = S^T from TMEM as bf16 (hi and lo halves,
 //                                 S = hi + lo to about 2^-17), B = Q_c (K-major)
-// The gate is applied by the 128 state threads (one TMEM lane = one dv row
-// each) when they split S^T for the readout, so it never waits on memory.
+// The gate is applied by the state warps (two threads per TMEM lane = dv row,
+// 64 dk columns each) when they split S^T for the readout, so it never waits
+// on memory. The output goes through two TMEM buffers: output warps write
+// chunk c while the state warps split the state of chunk c+1.
 // Q, K and V chunks stream in by TMA (4-D tensor maps over [B][T][H][128],
 // zero fill past T) through a two-stage ring; the output is written in fp32.
 #pragma once
@@ -32,7 +34,11 @@ constexpr int kHalf = 128 * 128;     // 128 rows x 64 columns of bf16: 16 KiB
 constexpr int kTile = 2 * kHalf;     // 128 x 128 bf16: 32 KiB
 constexpr int kStages = 2;
 constexpr int kStageBytes = 3 * kTile;  // Q, K, V
-constexpr int kThreads = 192;
+// warps: 0 TMA, 1 MMA, 2..9 state (two per TMEM lane quarter, 64 dk columns
+// each), 10..13 output (one per lane quarter)
+constexpr int kStateWarps = 8, kOutWarps = 4;
+constexpr int kThreads = 64 + 32 * (kStateWarps + kOutWarps);
+// TMEM columns: S^T fp32, its bf16 hi and lo halves, two output buffers
 constexpr int kColS = 0, kColHi = 128, kColLo = 192, kColO = 256, kTmemCols = 512;
 constexpr int kOffBar = kStages * kStageBytes;
 constexpr int kSmemBytes = kOffBar + 256 + 1024;
@@ -63,11 +69,12 @@ __global__ void __launch_bounds__(gss::kThreads, 1) gated_state_scan_kernel(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);  // [kStages]
     uint64_t* empty = full + kStages;                                // [kStages]
-    uint64_t* s0ready = empty + kStages;   // initial state in TMEM (4 warps)
+    uint64_t* s0ready = empty + kStages;   // initial state in TMEM (state warps)
     uint64_t* upd_done = s0ready + 1;      // update MMAs of a chunk completed
-    uint64_t* cdone = upd_done + 1;        // hi/lo written and S^T gated (4 warps)
-    uint64_t* out_ready = cdone + 1;       // readout MMAs of a chunk completed
-    uint64_t* drain = out_ready + 1;
+    uint64_t* cdone = upd_done + 1;        // hi/lo written and S^T gated (state warps)
+    uint64_t* out_ready = cdone + 1;       // [2] readout MMAs into output buffer b completed
+    uint64_t* ofree = out_ready + 2;       // [2] output buffer b read out (output warps)
+    uint64_t* drain = ofree + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -81,10 +88,13 @@ __global__ void __launch_bounds__(gss::kThreads, 1) gated_state_scan_kernel(
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 1);
         }
-        mbar_init(s0ready, 4);
+        mbar_init(s0ready, kStateWarps);
         mbar_init(upd_done, 1);
-        mbar_init(cdone, 4);
-        mbar_init(out_ready, 1);
+        mbar_init(cdone, kStateWarps);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&out_ready[i], 1);
+            mbar_init(&ofree[i], kOutWarps);
+        }
         mbar_init(drain, 1);
         *s_abort = 0;
         fence_mbar_init();
@@ -145,7 +155,8 @@ __global__ void __launch_bounds__(gss::kThreads, 1) gated_state_scan_kernel(
             };
             bool fine = nchunks == 0 || (mbar_wait(s0ready, 0) && update(0));
             for (int c = 0; c < nchunks && fine; ++c) {
-                if (*s_abort || !mbar_wait(cdone, c & 1)) {
+                if (*s_abort || !mbar_wait(cdone, c & 1) ||
+                    (c >= 2 && !mbar_wait(&ofree[c & 1], ((c >> 1) - 1) & 1))) {
                     fine = false;
                     break;
                 }
@@ -159,12 +170,12 @@ __global__ void __launch_bounds__(gss::kThreads, 1) gated_state_scan_kernel(
 #pragma unroll
                     for (int kk = 0; kk < kD / 16; ++kk) {
                         const uint32_t off = (kk >> 2) * kHalf;
-                        tc_mma_tmem_a(tmem_base + kColO, a + kk * 8,
+                        tc_mma_tmem_a(tmem_base + kColO + (c & 1) * 128, a + kk * 8,
                                       sw128_desc(qb + off) + 2 * (kk & 3), kIdescRead,
                                       (part | kk) != 0 ? 1u : 0u);
                     }
                 }
-                tc_commit(out_ready);
+                tc_commit(&out_ready[c & 1]);
                 tc_commit(&empty[st]);
                 if (c + 1 < nchunks) fine = update(c + 1);
             }
@@ -173,83 +184,95 @@ __global__ void __launch_bounds__(gss::kThreads, 1) gated_state_scan_kernel(
             mbar_wait(drain, 0);
         }
     } else {
-        // ---------------- state threads: one dv row of S^T each ----------------
         const int quarter = warp & 3;
         const int i = quarter * 32 + lane;  // dv index = TMEM lane
         const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
         const size_t st_base = (size_t)bh * kD * kD;
-        // S^T[i][:] = gate[0] * S0[:][i]
-        {
-            const float g0 = nchunks > 0 ? g_row[0] : 1.f;
+        if (warp < 2 + kStateWarps) {
+            // ---------------- state warps: dk columns 64*hf .. 64*hf+63 of row i ----------------
+            const int hf = (warp - 2) >> 2;
+            {   // S^T[i][:] = gate[0] * S0[:][i]
+                const float g0 = nchunks > 0 ? g_row[0] : 1.f;
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                uint32_t v[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    v[e] = __float_as_uint(g0 * state_in[st_base + (size_t)(ch * 32 + e) * kD + i]);
-                tmem_st32(lane_addr + kColS + ch * 32, v);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(s0ready);
-        }
-        for (int c = 0; c < nchunks; ++c) {
-            const bool w1 = mbar_wait(upd_done, c & 1);
-            if (!__all_sync(0xffffffffu, w1 && !*s_abort)) {
-                *s_abort = 1;
-                break;
-            }
-            tc_fence_after();
-            const bool last = c + 1 == nchunks;
-            const float gn = last ? 1.f : g_row[c + 1];
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                uint32_t v[32];
-                tmem_ld32(lane_addr + kColS + ch * 32, v);
-                uint32_t hi[16], lo[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float x0 = __uint_as_float(v[2 * e]), x1 = __uint_as_float(v[2 * e + 1]);
-                    const __nv_bfloat162 hp = __floats2bfloat162_rn(x0, x1);
-                    const float2 hf = __bfloat1622float2(hp);
-                    hi[e] = *reinterpret_cast<const uint32_t*>(&hp);
-                    lo[e] = pack_bf16x2(x0 - hf.x, x1 - hf.y);
-                }
-                tmem_st16(lane_addr + kColHi + ch * 16, hi);
-                tmem_st16(lane_addr + kColLo + ch * 16, lo);
-                if (last) {
-                    // the final state, S[:][i]
+                for (int ch = 0; ch < 2; ++ch) {
+                    uint32_t v[32];
+                    const int d0 = hf * 64 + ch * 32;
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
-                        state_out[st_base + (size_t)(ch * 32 + e) * kD + i] = __uint_as_float(v[e]);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(gn * __uint_as_float(v[e]));
-                    tmem_st32(lane_addr + kColS + ch * 32, v);
+                        v[e] = __float_as_uint(g0 * state_in[st_base + (size_t)(d0 + e) * kD + i]);
+                    tmem_st32(lane_addr + kColS + d0, v);
                 }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(s0ready);
             }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(cdone);
-            // the chunk's output O^T[i][t] -> out[b][t][h][i]
-            const bool w2 = mbar_wait(out_ready, c & 1);
-            if (!__all_sync(0xffffffffu, w2 && !*s_abort)) {
-                *s_abort = 1;
-                break;
-            }
-            tc_fence_after();
-            const int t0 = c * kC;
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                uint32_t v[32];
-                tmem_ld32(lane_addr + kColO + ch * 32, v);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int t = t0 + ch * 32 + e;
-                    if (t < T) out[(((size_t)b * T + t) * H + h) * kD + i] = __uint_as_float(v[e]);
+            for (int c = 0; c < nchunks; ++c) {
+                const bool w1 = mbar_wait(upd_done, c & 1);
+                if (!__all_sync(0xffffffffu, w1 && !*s_abort)) {
+                    *s_abort = 1;
+                    break;
                 }
+                tc_fence_after();
+                const bool last = c + 1 == nchunks;
+                const float gn = last ? 1.f : g_row[c + 1];
+#pragma unroll
+                for (int ch = 0; ch < 2; ++ch) {
+                    const int d0 = hf * 64 + ch * 32;
+                    uint32_t v[32];
+                    tmem_ld32(lane_addr + kColS + d0, v);
+                    uint32_t hi[16], lo[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float x0 = __uint_as_float(v[2 * e]), x1 = __uint_as_float(v[2 * e + 1]);
+                        const __nv_bfloat162 hp = __floats2bfloat162_rn(x0, x1);
+                        const float2 hf2 = __bfloat1622float2(hp);
+                        hi[e] = *reinterpret_cast<const uint32_t*>(&hp);
+                        lo[e] = pack_bf16x2(x0 - hf2.x, x1 - hf2.y);
+                    }
+                    tmem_st16(lane_addr + kColHi + d0 / 2, hi);
+                    tmem_st16(lane_addr + kColLo + d0 / 2, lo);
+                    if (last) {
+                        // the final state, S[:][i]
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            state_out[st_base + (size_t)(d0 + e) * kD + i] = __uint_as_float(v[e]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(gn * __uint_as_float(v[e]));
+                        tmem_st32(lane_addr + kColS + d0, v);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(cdone);
+            }
+        } else {
+            // ---------------- output warps: O^T[i][t] -> out[b][t][h][i] ----------------
+            for (int c = 0; c < nchunks; ++c) {
+                const bool w2 = mbar_wait(&out_ready[c & 1], (c >> 1) & 1);
+                if (!__all_sync(0xffffffffu, w2 && !*s_abort)) {
+                    *s_abort = 1;
+                    break;
+                }
+                tc_fence_after();
+                const int t0 = c * kC;
+                float* ob = out + (((size_t)b * T + t0) * H + h) * kD + i;
+                const size_t tstride = (size_t)H * kD;
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t v[32];
+                    tmem_ld32(lane_addr + kColO + (c & 1) * 128 + ch * 32, v);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int t = ch * 32 + e;
+                        if (t0 + t < T) ob[(size_t)t * tstride] = __uint_as_float(v[e]);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ofree[c & 1]);
             }
         }
     }
