@@ -25,8 +25,8 @@
 // of once per query.
 //
 // Warps: 0 TMA producer (K and V rings, 128-byte swizzle), 1 MMA issuer (one
-// thread), 2..17 softmax: four threads per MMA row (TMEM lane), each taking 32
-// tokens of a stage and 32 of the output dims. The softmax is online
+// thread), 2..9 softmax: two threads per MMA row (TMEM lane), each taking one
+// 64-token unit of a stage and 64 of the output dims. The softmax is online
 // with a lazy rescale: a row's reference maximum m moves only when a stage's
 // maximum exceeds it by more than 8 (log2 units), so P <= 2^8 and O is
 // rescaled in TMEM only then (after the previous P V has completed). The
@@ -53,8 +53,7 @@ constexpr int kTileBytes = 2 * kHalf;  // 128 rows x 128 dims bf16: 32 KiB
 constexpr int kKStages = 3, kVStages = 3;
 constexpr int kMaxWords = 512;         // block bitmap words: nb_max <= 16384
 constexpr int kMaxUnion = 1024;        // distinct blocks per tile (QT * topk)
-constexpr int kParts = 4;                // threads per MMA row (32 stage columns each)
-constexpr int kSoftWarps = 4 * kParts;
+constexpr int kSoftWarps = 8;            // two threads per MMA row
 constexpr int kThreads = 64 + 32 * kSoftWarps;
 // TMEM columns: O [128 rows x 128 dims] fp32, two S buffers [128 x 128 tokens]
 // fp32 whose first 64 columns then hold the stage's P as bf16 pairs, and Q
@@ -67,11 +66,10 @@ constexpr int kOffV = kOffK + kKStages * kTileBytes;
 constexpr int kOffUnion = kOffV + kVStages * kTileBytes;
 constexpr int kUnionBytes = 2 * kMaxWords * 4 + 3 * kMaxUnion * 4;
 constexpr int kOffBar = kOffUnion + kUnionBytes;
-// exchange between a row's threads: [3][kParts][128] floats (two stage buffers
-// of partial maxima, then the partial sums) and [2][kParts][128] ints (wait
-// outcomes)
+// exchange between a row's two threads: [3][2][128] floats (two stage buffers
+// of row maxima, then the row sums) and [2][2][128] ints (wait outcomes)
 constexpr int kOffXchg = kOffBar + 256;
-constexpr int kSmemBytes = kOffXchg + 3 * kParts * 128 * 4 + 2 * kParts * 128 * 4 + 1024 /*alignment slack*/;
+constexpr int kSmemBytes = kOffXchg + 3 * 2 * 128 * 4 + 2 * 2 * 128 * 4 + 1024 /*alignment slack*/;
 // instruction descriptors: D fp32, A and B bf16, M = 128, N = 128;
 // S = Q K^T with both operands K-major, O += P V with V (B) MN-major
 constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(128 >> 3) << 17) |
@@ -294,21 +292,21 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
     // starts its loads meanwhile.
     constexpr int kQBarrier = 5, kQThreads = 32 + 32 * kSoftWarps;
     if (warp >= 2) {
-        const int quarter = warp & 3, part = (warp - 2) >> 2;
+        const int quarter = warp & 3, hf = (warp - 2) >> 2;
         const int r = quarter * 32 + lane;
         const int qi = r / G, s = s0 + qi;
         const uint4* src = reinterpret_cast<const uint4*>(
             q + (((size_t)b * S + s) * H_q + (size_t)g * G + (r - qi * G)) * kHD);
-        uint32_t qv[16];
+        uint32_t qv[32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const uint4 v = s < S ? src[4 * part + c] : make_uint4(0, 0, 0, 0);
+        for (int c = 0; c < 8; ++c) {
+            const uint4 v = s < S ? src[8 * hf + c] : make_uint4(0, 0, 0, 0);
             qv[4 * c] = v.x;
             qv[4 * c + 1] = v.y;
             qv[4 * c + 2] = v.z;
             qv[4 * c + 3] = v.w;
         }
-        tmem_st16(tmem_base + ((uint32_t)(quarter * 32) << 16) + kColQ + part * 16, qv);
+        tmem_st32(tmem_base + ((uint32_t)(quarter * 32) << 16) + kColQ + hf * 32, qv);
         tmem_wait_st();
         tc_fence_before();
         named_barrier_sync(kQBarrier, kQThreads);
@@ -419,16 +417,13 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
             mbar_wait(drain, 0);
         }
     } else {
-        // ---------------- softmax and epilogue: kParts threads per MMA row ----------------
-        // Thread (r, part) owns stage columns 32*part .. 32*part+31 of row r
-        // (tokens 32*(part&1) .. +31 of unit slot part>>1) and output dims
-        // 32*part .. 32*part+31. A row's threads agree on its maximum through
-        // shared memory and a named barrier of their kParts warps (ids 1..4,
-        // one per TMEM lane quarter); every decision that changes control flow
-        // is taken the same way by all of them, so their barriers always match.
-        constexpr int kCols = 128 / kParts;
+        // ---------------- softmax and epilogue: two threads per MMA row ----------------
+        // Thread (r, hf) owns row r's tokens of unit slot hf (stage columns
+        // 64*hf .. 64*hf+63) and output dims 64*hf .. 64*hf+63. The two halves
+        // of a row agree on its maximum through shared memory and a named
+        // barrier of their two warps (ids 1..4, one per TMEM lane quarter).
         const int quarter = warp & 3;
-        const int part = (warp - 2) >> 2;
+        const int hf = (warp - 2) >> 2;
         const int r = quarter * 32 + lane;
         const int bar_id = 1 + quarter;
         const int qi = r / G, s = s0 + qi;
@@ -436,34 +431,36 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
         const long long last = s < S ? (p < ctx - 1 ? p : ctx - 1) : -1;
         const uint32_t qbit = 1u << qi;
         const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
-        float* xchg = reinterpret_cast<float*>(smem + kOffXchg);    // [3][kParts][128]
-        int* xok = reinterpret_cast<int*>(xchg + 3 * kParts * 128);  // [2][kParts][128]
-        float m_ref = -INFINITY;  // reference maximum (log2 units), the same in every part
-        float l = 0.f;            // this part's share of the row sum
-        const int slot = (part * kCols) >> 6, slot_off = (part * kCols) & 63;
+        float* xchg = reinterpret_cast<float*>(smem + kOffXchg);  // [3][2][128]
+        int* xok = reinterpret_cast<int*>(xchg + 3 * 2 * 128);      // [2][2][128]
+        float m_ref = -INFINITY;  // reference maximum (log2 units), the same in both halves
+        float l = 0.f;            // this half's share of the row sum
         for (int i = 0; i < nstages; ++i) {
-            // this part's tokens: whether the row takes their unit and how many
-            // of them the row may see
-            const int u = 2 * i + slot;
-            int nval = 0;
+            // this half's unit: its first token, whether the row takes it, and
+            // how many of its 64 tokens the row may see
+            const int u = 2 * i + hf;
+            int t0 = 0, nval = 0;
             if (u < nunits) {
                 const int blk = u / upb, sub = u - blk * upb;
-                if (upage[blk] >= 0 && (umask[blk] & qbit) != 0u) {
-                    const long long nv = last - ((long long)ublk[blk] * bs + sub * 64 + slot_off) + 1;
-                    nval = nv <= 0 ? 0 : (nv < kCols ? (int)nv : kCols);
+                if (upage[blk] >= 0) {
+                    t0 = ublk[blk] * bs + sub * 64;
+                    if ((umask[blk] & qbit) != 0u && (long long)t0 <= last) {
+                        const long long nv = last - t0 + 1;
+                        nval = nv < 64 ? (int)nv : 64;
+                    }
                 }
             }
             const bool waited = mbar_wait(&sfull[i & 1], (i >> 1) & 1);
             const int my_ok = waited && !*s_abort;
             tc_fence_after();
-            uint32_t sv[kCols];
+            uint32_t sv[64];
             float mx = -INFINITY;
             const bool warp_any = __any_sync(0xffffffffu, nval > 0);
             if (warp_any) {
-                tmem_ld32(lane_addr + kColS + (i & 1) * 128 + part * kCols, sv);
-                if (nval < kCols) {
+                tmem_ld64(lane_addr + kColS + (i & 1) * 128 + hf * 64, sv);
+                if (nval < 64) {
 #pragma unroll
-                    for (int e = 0; e < kCols; ++e)
+                    for (int e = 0; e < 64; ++e)
                         sv[e] = e < nval ? sv[e] : __float_as_uint(-INFINITY);
                 }
                 // eight independent running maxima, then a tree
@@ -471,31 +468,25 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
 #pragma unroll
                 for (int k = 0; k < 8; ++k) pm[k] = __uint_as_float(sv[k]);
 #pragma unroll
-                for (int e = 8; e < kCols; ++e) pm[e & 7] = fmaxf(pm[e & 7], __uint_as_float(sv[e]));
+                for (int e = 8; e < 64; ++e) pm[e & 7] = fmaxf(pm[e & 7], __uint_as_float(sv[e]));
                 mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
                            fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
             }
             // the row maximum of the stage (raw scores; the scale is positive),
-            // and whether every part may go on
-            float* xm = xchg + (i & 1) * kParts * 128;
-            int* xo = xok + (i & 1) * kParts * 128;
-            xm[part * 128 + r] = mx;
-            xo[part * 128 + r] = my_ok;
-            tc_fence_before();  // this part's S loads are ordered before the others' P stores
-            named_barrier_sync(bar_id, 32 * kParts);
+            // and whether both halves may go on: one decision for the pair of
+            // warps, so their named barriers always match
+            float* xm = xchg + (i & 1) * 256;
+            int* xo = xok + (i & 1) * 256;
+            xm[hf * 128 + r] = mx;
+            xo[hf * 128 + r] = my_ok;
+            tc_fence_before();  // this half's S loads are ordered before the partner's P stores
+            named_barrier_sync(bar_id, 64);
             tc_fence_after();
-            float mrow = -INFINITY;
-            int all_ok = 1;
-#pragma unroll
-            for (int k = 0; k < kParts; ++k) {
-                mrow = fmaxf(mrow, xm[k * 128 + r]);
-                all_ok &= xo[k * 128 + r];
-            }
-            if (!__all_sync(0xffffffffu, all_ok)) {
+            if (!__all_sync(0xffffffffu, my_ok && xo[(hf ^ 1) * 128 + r])) {
                 *s_abort = 1;
                 break;
             }
-            mrow *= scale_log2;
+            const float mrow = fmaxf(mx, xm[(hf ^ 1) * 128 + r]) * scale_log2;
             // lazy reference: move m only when the stage's maximum passes m + 8
             float corr = 1.f;
             if (mrow > m_ref + kLazy) {
@@ -503,27 +494,30 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
                 m_ref = mrow;
             }
             if (__any_sync(0xffffffffu, corr != 1.f)) {
-                // O holds earlier stages of this row: rescale this part's
+                // O holds earlier stages of this row: rescale this half's
                 // columns once the previous P V has landed
                 if (!mbar_wait(obar, (i - 1) & 1)) *s_abort = 1;
                 tc_fence_after();
-                uint32_t ov[32];
-                tmem_ld32(lane_addr + kColO + part * 32, ov);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
-                tmem_st32(lane_addr + kColO + part * 32, ov);
+                for (int ch = 0; ch < 2; ++ch) {
+                    uint32_t ov[32];
+                    tmem_ld32(lane_addr + kColO + hf * 64 + ch * 32, ov);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
+                    tmem_st32(lane_addr + kColO + hf * 64 + ch * 32, ov);
+                }
                 l *= corr;
             }
             // P = 2^(s*c - m) as bf16 pairs; it overwrites the S buffer's first
-            // 64 columns (every part has read its S columns: the barrier above)
+            // 64 columns (both halves have read their S columns: the barrier above)
             const float neg_m = -m_ref;
-            uint32_t pk[kCols / 2];
+            uint32_t pk[32];
             if (nval > 0) {
                 float ps[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) ps[k] = 0.f;
 #pragma unroll
-                for (int e = 0; e < kCols / 2; ++e) {
+                for (int e = 0; e < 32; ++e) {
                     // masked entries hold -inf: 2^-inf = 0
                     const float a = fast_exp2(fmaf(__uint_as_float(sv[2 * e]), scale_log2, neg_m));
                     const float bb = fast_exp2(fmaf(__uint_as_float(sv[2 * e + 1]), scale_log2, neg_m));
@@ -533,13 +527,13 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
                 l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
             } else {
 #pragma unroll
-                for (int e = 0; e < kCols / 2; ++e) pk[e] = 0u;
+                for (int e = 0; e < 32; ++e) pk[e] = 0u;
             }
-            tmem_st16(lane_addr + kColS + (i & 1) * 128 + part * (kCols / 2), pk);
+            tmem_st32(lane_addr + kColS + (i & 1) * 128 + hf * 32, pk);
             tmem_wait_st();
             // V rows of an absent unit and of tokens past the context length
             // must be zero before the P V MMA reads them (this thread: token row
-            // r of the stage, dims 32*part .. 32*part+31)
+            // r of the stage, dims 64*hf .. 64*hf+63)
             bool v_absent[2];
             long long v_t0[2];
             bool stage_tail = false;  // the same for every thread
@@ -565,7 +559,7 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
                 if (mine_absent || mine_t0 + (r & 63) >= ctx) {
                     unsigned char* vt = smem + kOffV + vs * kTileBytes;
 #pragma unroll
-                    for (int cc = 4 * part; cc < 4 * part + 4; ++cc)
+                    for (int cc = 8 * hf; cc < 8 * hf + 8; ++cc)
                         *reinterpret_cast<uint4*>(vt + pfa_off(r, cc)) = make_uint4(0, 0, 0, 0);
                 }
                 fence_proxy_async_smem();
@@ -575,38 +569,40 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
             if (lane == 0) mbar_arrive(&pfull[i & 1]);
         }
         // ---------------- epilogue: O / l -> bf16 ----------------
-        float* xl = xchg + 2 * kParts * 128;
-        xl[part * 128 + r] = l;
-        named_barrier_sync(bar_id, 32 * kParts);
-        float ltot = 0.f;
-#pragma unroll
-        for (int k = 0; k < kParts; ++k) ltot += xl[k * 128 + r];
+        float* xl = xchg + 2 * 256;
+        xl[hf * 128 + r] = l;
+        named_barrier_sync(bar_id, 64);
+        const float ltot = l + xl[(hf ^ 1) * 128 + r];
         if (nstages > 0 && !*s_abort) {
             if (!mbar_wait(ofin, 0)) *s_abort = 1;
             tc_fence_after();
         }
         const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
         // log2-sum-exp2 of the scaled logits, for combining partial results
-        if (lse != nullptr && s < S && part == 0)
+        if (lse != nullptr && s < S && hf == 0)
             lse[((size_t)b * S + s) * H_q + (size_t)g * G + (r - qi * G)] =
                 ltot > 0.f ? m_ref + __log2f(ltot) : -INFINITY;
         __nv_bfloat16* orow = out + (((size_t)b * S + s) * H_q + (size_t)g * G + (r - qi * G)) * kHD;
-        uint32_t ov[32];
-        if (nstages > 0) {
-            tmem_ld32(lane_addr + kColO + part * 32, ov);
-        } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = 0u;
-        }
-        if (s < S) {
-            uint32_t pk[16];
+        for (int ch = 0; ch < 2; ++ch) {
+            uint32_t ov[32];
+            if (nstages > 0) {
+                tmem_ld32(lane_addr + kColO + hf * 64 + ch * 32, ov);
+            } else {
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-                pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv);
-            uint4* dst = reinterpret_cast<uint4*>(orow + part * 32);
+                for (int e = 0; e < 32; ++e) ov[e] = 0u;
+            }
+            if (s < S) {
+                uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv,
+                                        __uint_as_float(ov[2 * e + 1]) * inv);
+                uint4* dst = reinterpret_cast<uint4*>(orow + hf * 64 + ch * 32);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            }
         }
     }
     tc_fence_before();
