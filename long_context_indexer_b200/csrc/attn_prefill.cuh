@@ -54,7 +54,8 @@ constexpr int kKStages = 3, kVStages = 3;
 constexpr int kMaxWords = 512;         // block bitmap words: nb_max <= 16384
 constexpr int kMaxUnion = 1024;        // distinct blocks per tile (QT * topk)
 constexpr int kSoftWarps = 8;            // two threads per MMA row
-constexpr int kThreads = 64 + 32 * kSoftWarps;
+constexpr int kVWarp = 2 + kSoftWarps;     // V producer (warp 0 produces K)
+constexpr int kThreads = 64 + 32 * kSoftWarps + 32;
 // TMEM columns: O [128 rows x 128 dims] fp32, two S buffers [128 x 128 tokens]
 // fp32 whose first 64 columns then hold the stage's P as bf16 pairs, and Q
 // [128 x 128 dims] as bf16 pairs (the A operand of S = Q K^T)
@@ -291,7 +292,7 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
     // 2c, 2c+1); the MMA warp waits for them on named barrier 5. The producer
     // starts its loads meanwhile.
     constexpr int kQBarrier = 5, kQThreads = 32 + 32 * kSoftWarps;
-    if (warp >= 2) {
+    if (warp >= 2 && warp < kVWarp) {
         const int quarter = warp & 3, hf = (warp - 2) >> 2;
         const int r = quarter * 32 + lane;
         const int qi = r / G, s = s0 + qi;
@@ -315,11 +316,19 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
         tc_fence_after();
     }
 
-    if (warp == 0) {
-        // ---------------- TMA producer ----------------
+    if (warp == 0 || warp == kVWarp) {
+        // ---------------- TMA producers: K (warp 0) and V (the last warp) ----------------
+        // Separate producers let K run ahead of the V ring, whose slots free
+        // only after the softmax and P V of their stage.
+        const bool is_k = warp == 0;
+        const int nst = is_k ? kKStages : kVStages;
+        uint64_t* fullb = is_k ? kfull : vfull;
+        uint64_t* emptyb = is_k ? kempty : vempty;
+        const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
+        unsigned char* ring = smem + (is_k ? kOffK : kOffV);
         if (lane == 0) {
             for (int i = 0; i < nstages; ++i) {
-                const int ks = i % kKStages, vs = i % kVStages;
+                const int st = i % nst;
                 int ys[2];
                 int nload = 0;
                 for (int c = 0; c < 2; ++c) {
@@ -336,35 +345,20 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
                 }
                 const uint32_t bytes = (uint32_t)nload * 2u * 8192u;
                 if (*s_abort) break;
-                if (i >= kKStages && !mbar_wait(&kempty[ks], ((i / kKStages) - 1) & 1)) {
+                if (i >= nst && !mbar_wait(&emptyb[st], ((i / nst) - 1) & 1)) {
                     *s_abort = 1;
                     break;
                 }
-                unsigned char* kd = smem + kOffK + ks * kTileBytes;
+                unsigned char* dst = ring + st * kTileBytes;
                 if (bytes) {
-                    mbar_arrive_expect_tx(&kfull[ks], bytes);
+                    mbar_arrive_expect_tx(&fullb[st], bytes);
                     for (int c = 0; c < 2; ++c)
                         if (ys[c] >= 0) {
-                            tma_load_2d(kd + c * 8192, &tm_k, 0, ys[c], &kfull[ks]);
-                            tma_load_2d(kd + kHalf + c * 8192, &tm_k, 64, ys[c], &kfull[ks]);
+                            tma_load_2d(dst + c * 8192, tm, 0, ys[c], &fullb[st]);
+                            tma_load_2d(dst + kHalf + c * 8192, tm, 64, ys[c], &fullb[st]);
                         }
                 } else {
-                    mbar_arrive(&kfull[ks]);
-                }
-                if (i >= kVStages && !mbar_wait(&vempty[vs], ((i / kVStages) - 1) & 1)) {
-                    *s_abort = 1;
-                    break;
-                }
-                unsigned char* vd = smem + kOffV + vs * kTileBytes;
-                if (bytes) {
-                    mbar_arrive_expect_tx(&vfull[vs], bytes);
-                    for (int c = 0; c < 2; ++c)
-                        if (ys[c] >= 0) {
-                            tma_load_2d(vd + c * 8192, &tm_v, 0, ys[c], &vfull[vs]);
-                            tma_load_2d(vd + kHalf + c * 8192, &tm_v, 64, ys[c], &vfull[vs]);
-                        }
-                } else {
-                    mbar_arrive(&vfull[vs]);
+                    mbar_arrive(&fullb[st]);
                 }
             }
         }
