@@ -162,14 +162,8 @@ __global__ void __launch_bounds__(NT) index_gemv_select_kernel(
     __threadfence();
     if (tid == 0) counters[row] = 0u;
     SelectSmem& sel = *reinterpret_cast<SelectSmem*>(dyn_smem);
-    if (vis <= kWarpSelMax && topk <= kWarpSelTopk) {
-        // a short row: one warp selects without CTA barriers (the other warps
-        // wait for it only when the row is published to a consumer)
-        if (warp == 0) warp_topk_select(row_scores, vis, topk, ids + (size_t)row * topk, sel);
-    } else {
-        cta_topk_select<NT>(row_scores, chunk_max + (size_t)row * nchunks, vis, chunk_blocks,
-                            topk, ids + (size_t)row * topk, sel);
-    }
+    cta_topk_select<NT>(row_scores, chunk_max + (size_t)row * nchunks, vis, chunk_blocks, topk,
+                        ids + (size_t)row * topk, sel);
     if (ready != nullptr) {  // publish the row to a consumer running concurrently
         __syncthreads();
         if (tid == 0) {

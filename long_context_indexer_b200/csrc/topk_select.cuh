@@ -307,104 +307,3 @@ __device__ void cta_topk_select(const float* scores, const uint32_t* chunk_max, 
 }
 
 }  // namespace lci
-
-namespace lci {
-
-constexpr int kWarpSelMax = 1024;   // candidates the one-warp select takes (32 per lane)
-constexpr int kWarpSelTopk = 64;    // and winners (2 per lane)
-
-// Exact top-k of scores[0..n) by (score desc, index asc), written in rank order
-// to out[0..topk) with -1 padding, by ONE warp (n <= kWarpSelMax, topk <=
-// kWarpSelTopk): the order-preserving keys go to shared memory once, a
-// four-pass radix select finds the k-th largest key (a warp-private 256-bin
-// histogram per pass, no CTA barrier), then the winners are ranked among
-// themselves. Keys are visited in index order (j outer, lane inner), which is
-// how ties at the threshold are taken.
-__device__ void warp_topk_select(const float* scores, int n, int topk, int32_t* out,
-                                 SelectSmem& sm) {
-    const int lane = threadIdx.x & 31;
-    for (int i = lane; i < n; i += 32) sm.cand_key[i] = load_key(scores, i);
-    __syncwarp();
-    const int k = n < topk ? n : topk;
-    uint32_t prefix = 0u, mask = 0u;
-    int remaining = k;
-#pragma unroll 1
-    for (int shift = 24; shift >= 0 && k > 0; shift -= 8) {
-        for (int b = lane; b < 256; b += 32) sm.hist[b] = 0u;
-        __syncwarp();
-        for (int i = lane; i < n; i += 32) {
-            const uint32_t u = sm.cand_key[i];
-            if ((u & mask) == prefix) atomicAdd(&sm.hist[(u >> shift) & 255u], 1u);
-        }
-        __syncwarp();
-        // lane l owns bins 255-8l .. 248-8l (descending)
-        int c[8], lsum = 0;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            c[q] = (int)sm.hist[255 - 8 * lane - q];
-            lsum += c[q];
-        }
-        int incl = lsum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += t;
-        }
-        const int excl = incl - lsum;
-        int bin = -1, above = 0;
-        if (excl < remaining && remaining <= incl) {
-            int cum = excl;
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                if (bin < 0 && cum + c[q] >= remaining) {
-                    bin = 255 - 8 * lane - q;
-                    above = cum;
-                }
-                cum += c[q];
-            }
-        }
-        const unsigned owner = __ballot_sync(0xffffffffu, bin >= 0);
-        const int src = __ffs(owner) - 1;
-        bin = __shfl_sync(0xffffffffu, bin, src);
-        above = __shfl_sync(0xffffffffu, above, src);
-        remaining -= above;
-        prefix |= (uint32_t)bin << shift;
-        mask |= 255u << shift;
-        __syncwarp();
-    }
-    // winners: keys above the threshold, then the lowest-index keys equal to it
-    const uint32_t T = prefix;
-    int taken = 0, eq_taken = 0;
-    for (int base = 0; base < n && k > 0; base += 32) {
-        const int i = base + lane;
-        const uint32_t u = i < n ? sm.cand_key[i] : 0u;
-        const bool gt = i < n && u > T;
-        const bool eq = i < n && u == T;
-        const unsigned eq_b = __ballot_sync(0xffffffffu, eq);
-        const int eq_rank = eq_taken + __popc(eq_b & ((1u << lane) - 1u));
-        const bool take = gt || (eq && eq_rank < remaining);
-        const unsigned tb = __ballot_sync(0xffffffffu, take);
-        if (take) {
-            const int slot = taken + __popc(tb & ((1u << lane) - 1u));
-            sm.win_key[slot] = u;
-            sm.win_id[slot] = i;
-        }
-        taken += __popc(tb);
-        eq_taken += __popc(eq_b);
-    }
-    __syncwarp();
-    // rank the k winners among themselves: (key desc, index asc)
-    for (int e = lane; e < k; e += 32) {
-        const uint32_t ke = sm.win_key[e];
-        const int ie = sm.win_id[e];
-        int rank = 0;
-        for (int f = 0; f < k; ++f) {
-            const uint32_t kf = sm.win_key[f];
-            rank += (kf > ke) || (kf == ke && sm.win_id[f] < ie);
-        }
-        out[rank] = ie;
-    }
-    for (int i = k + lane; i < topk; i += 32) out[i] = -1;
-}
-
-}  // namespace lci
