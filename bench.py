@@ -51,10 +51,39 @@ def parse():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default=HEADLINE, choices=sorted(CONFIGS))
+    ap.add_argument("--config", default=HEADLINE, choices=sorted(CONFIGS) + ["scan"])
     ap.add_argument("--no-extra", action="store_true", help="skip the other configurations")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="run the workload's step --steps times without timing or output "
+                         "(for profiler captures); --config scan runs the state scan, "
+                         "--persistent the one-launch decode step")
+    ap.add_argument("--persistent", action="store_true")
     return ap.parse_args()
+
+
+def run_profile(args):
+    """The step of one workload, --steps times, nothing timed or printed but a
+    status line: a small, self-contained command for ncu captures."""
+    import long_context_indexer_b200 as lci
+    torch.cuda.set_device(0)
+    if args.config == "scan":
+        cfg = SCAN_CONFIGS["scan"].replace(B=2)
+        d = {k: v.cuda() for k, v in generate_scan(cfg).items()}
+        for _ in range(args.steps):
+            lci.gated_state_scan(d["q"], d["k"], d["v"], d["gate"], d["state"], cfg.C)
+    else:
+        cfg = CONFIGS[args.config]
+        pipe = Pipeline(cfg, generate(cfg), torch.device("cuda", 0))
+        for _ in range(args.steps):
+            if args.persistent:
+                pipe.step_persistent()
+            else:
+                pipe.step()
+    torch.cuda.synchronize()
+    lci.get_device_status()
+    print(f"profile run: {args.config}{' persistent' if args.persistent else ''} x{args.steps} ok")
+    return 0
 
 
 def peaks():
@@ -610,6 +639,12 @@ def run_reference(args):
 
 def main():
     args = parse()
+    if args.profile:
+        return run_profile(args)
+    if args.config == "scan":
+        print("bench.py: --config scan is for --profile runs; the scan is measured in every "
+              "default run (state_scan in the JSON line)", file=sys.stderr)
+        return 2
     if args.impl == "reference":
         return run_reference(args)
     world, rank, local = dist_setup(args)
