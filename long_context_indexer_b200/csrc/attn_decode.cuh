@@ -21,9 +21,10 @@
 // load bank-conflict free and needs no ldmatrix.
 //
 // Combine: the four warps merge through shared memory into a CTA partial
-// (max, sum, unnormalised O); the CTAs of a cluster then merge their partials
-// through distributed shared memory, each CTA finishing a slice of the output.
-// No global workspace and no atomics.
+// (max, sum, unnormalised O) held in registers; the CTAs of a cluster then
+// store each slice of their partial into the CTA that finishes that slice
+// (distributed shared memory), so one cluster barrier separates the exchange
+// from the final merge. No global workspace and no atomics.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -46,11 +47,53 @@ constexpr int kBox = 64 * 64 * 2;  // one 64x64 bf16 box = 8 KiB
 constexpr int kStageBytes = 4 * kBox;  // K: 2 boxes, V: 2 boxes
 constexpr int kMaxSplit = 8;
 constexpr int kRows = 16;          // query heads per MMA (padded)
-// shared memory: stages, then barriers and metadata
-constexpr int smem_bytes(int stages) { return stages * kStageBytes + 1024 /*align*/ + 256; }
+constexpr int kSlots = 64;         // fp32 accumulators per consumer thread
+constexpr int kWoStride = 68;      // floats per lane of a warp partial (16-byte access, no conflicts)
+constexpr int kMetaBytes = 256;    // barriers and unit info after the ring
+// Slots of one cluster CTA's slice of the output (a multiple of 4), and the
+// padded per-lane pitch of a received slice (4 mod 8 floats: 16-byte
+// accesses of 8 consecutive lanes hit distinct banks).
+__host__ __device__ constexpr int slice_slots(int nsplit) {
+    return ((kSlots + nsplit - 1) / nsplit + 3) & ~3;
+}
+__host__ __device__ constexpr int slice_pitch(int sp) { return sp + ((12 - (sp & 7)) & 7); }
+constexpr int recv_floats() {
+    int m = 0;
+    for (int n = 2; n <= kMaxSplit; ++n) {
+        const int f = n * 32 * slice_pitch(slice_slots(n));
+        m = f > m ? f : m;
+    }
+    return m;
+}
+constexpr int kRecvFloats = recv_floats();  // slices received from the cluster
+// shared memory: ring stages, barriers and metadata, received slices and the
+// sources' (max, sum) per head
+constexpr int smem_bytes(int stages) {
+    return stages * kStageBytes + 1024 /*align*/ + kMetaBytes +
+           (kRecvFloats + kMaxSplit * kRows * 2) * 4;
+}
+static_assert(kConsumers * (32 * kWoStride + 2 * kRows) * 4 <= 3 * kStageBytes,
+              "warp partials fit in the ring");
 }  // namespace dec
 
 __device__ __forceinline__ int tok_perm(int x) { return x ^ ((x & 1) << 2); }
+
+// Four consecutive bf16 outputs: one 8-byte store when the output is 8-byte
+// aligned, else four 2-byte stores.
+__device__ __forceinline__ void store_bf16x4(__nv_bfloat16* p, float a, float b, float c, float d,
+                                             bool vec) {
+    if (vec) {
+        uint2 w;
+        w.x = pack_bf16x2(a, b);
+        w.y = pack_bf16x2(c, d);
+        *reinterpret_cast<uint2*>(p) = w;
+    } else {
+        p[0] = __float2bfloat16_rn(a);
+        p[1] = __float2bfloat16_rn(b);
+        p[2] = __float2bfloat16_rn(c);
+        p[3] = __float2bfloat16_rn(d);
+    }
+}
 
 // Byte offset of (row r, 16-byte chunk c of the 128-dim row) inside one K or V
 // tile stored as two 64x64 boxes with the 128-byte swizzle.
@@ -201,6 +244,9 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
         prefetch_tensormap(&tm_v);
     }
     __syncthreads();
+    // first half of the barrier that guarantees every CTA of the cluster runs
+    // before any distributed shared memory store (the wait is at the combine)
+    if (nsplit > 1) cluster_arrive_relaxed();
 
     // Per-thread fragment coordinates.
     const int g8 = lane >> 2, q4 = lane & 3;
@@ -323,21 +369,23 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
     }
     __syncthreads();  // every stage consumed: the ring memory is free
 
-    // ---------------- combine the four warps ----------------
-    // Partials stay in the accumulator fragment layout: slot o = 32*h + 4*i + e
-    // of lane l holds head (l>>2) + 8*(e>>1), dim 64*h + 16*(l&3) + 8*(e&1) + i.
-    // Every exchange below is a conflict-free [slot][lane] access.
-    constexpr int kSlots = 64;                 // fp32 accumulators per thread
-    constexpr int kElems = kSlots * 32;        // = 16 heads x 128 dims
-    float* wo = reinterpret_cast<float*>(smem);          // [kConsumers][kSlots][32]
-    float* wm = wo + kConsumers * kElems;                 // [kConsumers][16]
-    float* wl = wm + kConsumers * kRows;                  // [kConsumers][16]
-    float* wf = wl + kConsumers * kRows;                  // [kConsumers][16] weights
-    float* cm = wf + kConsumers * kRows;                  // [16] CTA max
-    float* cl = cm + kRows;                               // [16] CTA sum
-    float* co = cl + kRows;                               // [kSlots][32] CTA partial
-    float* xf = co + kElems;                              // [kMaxSplit][16]
-    float* xl = xf + kMaxSplit * kRows;                   // [16]
+    // ---------------- combine ----------------
+    // Accumulator slot o = 32*h + 4*i + e of lane l holds head (l>>2) + 8*(e>>1),
+    // dim 64*h + 16*(l&3) + 8*(e&1) + i (the mma C-fragment layout).
+    // 1. Each consumer warp leaves (max, sum, unnormalised O) in the free ring
+    //    memory; consumer thread (w, l) then merges slots 16w..16w+15 of lane l
+    //    over the four warps into the CTA partial, in registers.
+    // 2. A lone CTA normalises and writes the output. In a cluster, each CTA
+    //    stores every slice of its partial into the CTA owning that slice
+    //    (distributed shared memory), one cluster barrier publishes the stores,
+    //    and every owner merges its slice over the cluster from its own memory.
+    float* wo = reinterpret_cast<float*>(smem);             // [warp][lane][kWoStride]
+    float* wm = wo + kConsumers * 32 * kWoStride;           // [warp][16] running max
+    float* wl = wm + kConsumers * kRows;                    // [warp][16] running sum
+    float* ro = reinterpret_cast<float*>(smem + kStages * kStageBytes + kMetaBytes);
+    float* rml = ro + kRecvFloats;                          // [source CTA][16][max, sum]
+    __nv_bfloat16* orow = out + ((size_t)row * H_q + (size_t)g * G) * kHD;
+    const bool vec_out = (reinterpret_cast<uintptr_t>(out) & 7u) == 0u;
     if (warp < kConsumers) {
         l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
         l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
@@ -349,94 +397,148 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
             wl[warp * kRows + g8] = l_a;
             wl[warp * kRows + g8 + 8] = l_b;
         }
-        float* dst = wo + warp * kElems + lane;
+        float4* dst = reinterpret_cast<float4*>(wo + (warp * 32 + lane) * kWoStride);
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) dst[(32 * h + 4 * i + e) * 32] = o[h][i][e];
+                dst[8 * h + i] = make_float4(o[h][i][0], o[h][i][1], o[h][i][2], o[h][i][3]);
     }
     __syncthreads();
-    if (tid < kRows) {
-        float M = -INFINITY;
-#pragma unroll
-        for (int w2 = 0; w2 < kConsumers; ++w2) M = fmaxf(M, wm[w2 * kRows + tid]);
-        const float base = M == -INFINITY ? 0.f : M;
-        float L = 0.f;
+    const int sp = slice_slots(nsplit), pitch = slice_pitch(sp);
+    if (nsplit > 1) cluster_wait();  // every CTA of the cluster has started
+    if (warp < kConsumers) {
+        // heads of this lane's slots: e = 0, 1 -> ha; e = 2, 3 -> hb
+        const int ha = g8, hb = g8 + 8;
+        float Ma = -INFINITY, Mb = -INFINITY;
 #pragma unroll
         for (int w2 = 0; w2 < kConsumers; ++w2) {
-            const float f = exp2f(wm[w2 * kRows + tid] - base);
-            wf[w2 * kRows + tid] = f;
-            L += f * wl[w2 * kRows + tid];
+            Ma = fmaxf(Ma, wm[w2 * kRows + ha]);
+            Mb = fmaxf(Mb, wm[w2 * kRows + hb]);
         }
-        cm[tid] = M;
-        cl[tid] = L;
-        // log2-sum-exp2 of the scaled logits, for combining partial results
-        if (lse != nullptr && nsplit == 1 && tid < G)
-            lse[(size_t)row * H_q + (size_t)g * G + tid] = L > 0.f ? M + log2f(L) : -INFINITY;
-    }
-    __syncthreads();
-    __nv_bfloat16* orow = out + ((size_t)row * H_q + (size_t)g * G) * kHD;
-    for (int sidx = tid; sidx < kElems; sidx += kThreads) {
-        const int ln = sidx & 31, oi = sidx >> 5, e = oi & 3;
-        const int head = (ln >> 2) + 8 * (e >> 1);
-        float acc = 0.f;
+        const float ba = Ma == -INFINITY ? 0.f : Ma, bb = Mb == -INFINITY ? 0.f : Mb;
+        float fa[kConsumers], fb[kConsumers], La = 0.f, Lb = 0.f;
 #pragma unroll
-        for (int w2 = 0; w2 < kConsumers; ++w2) acc += wf[w2 * kRows + head] * wo[w2 * kElems + sidx];
+        for (int w2 = 0; w2 < kConsumers; ++w2) {
+            fa[w2] = exp2f(wm[w2 * kRows + ha] - ba);
+            fb[w2] = exp2f(wm[w2 * kRows + hb] - bb);
+            La += fa[w2] * wl[w2 * kRows + ha];
+            Lb += fb[w2] * wl[w2 * kRows + hb];
+        }
+        float4 acc[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w2 = 0; w2 < kConsumers; ++w2) {
+            const float4* src = reinterpret_cast<const float4*>(wo + (w2 * 32 + lane) * kWoStride) + 4 * warp;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float4 v = src[j];
+                acc[j].x += fa[w2] * v.x;
+                acc[j].y += fa[w2] * v.y;
+                acc[j].z += fb[w2] * v.z;
+                acc[j].w += fb[w2] * v.w;
+            }
+        }
         if (nsplit == 1) {
-            if (head < G) {
-                const int dim = 64 * (oi >> 5) + 16 * (ln & 3) + 8 * (e & 1) + ((oi >> 2) & 7);
-                const float L = cl[head];
-                orow[head * kHD + dim] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
+            // slots 16w + 4j + e: h = w >> 1, i = (4w + j) & 7, so group j of
+            // component e lands on dim 64h + 16*q4 + 8*(e&1) + ((4w) & 7) + j
+            const float ia = La > 0.f ? 1.f / La : 0.f, ib = Lb > 0.f ? 1.f / Lb : 0.f;
+            const int d0 = 64 * (warp >> 1) + 16 * q4 + ((4 * warp) & 7);
+            if (ha < G) {
+                store_bf16x4(orow + ha * kHD + d0, acc[0].x * ia, acc[1].x * ia, acc[2].x * ia,
+                             acc[3].x * ia, vec_out);
+                store_bf16x4(orow + ha * kHD + d0 + 8, acc[0].y * ia, acc[1].y * ia, acc[2].y * ia,
+                             acc[3].y * ia, vec_out);
+            }
+            if (hb < G) {
+                store_bf16x4(orow + hb * kHD + d0, acc[0].z * ib, acc[1].z * ib, acc[2].z * ib,
+                             acc[3].z * ib, vec_out);
+                store_bf16x4(orow + hb * kHD + d0 + 8, acc[0].w * ib, acc[1].w * ib, acc[2].w * ib,
+                             acc[3].w * ib, vec_out);
+            }
+            // log2-sum-exp2 of the scaled logits, for combining partial results
+            if (lse != nullptr && warp == 0 && q4 == 0) {
+                float* lrow = lse + (size_t)row * H_q + (size_t)g * G;
+                if (ha < G) lrow[ha] = La > 0.f ? Ma + log2f(La) : -INFINITY;
+                if (hb < G) lrow[hb] = Lb > 0.f ? Mb + log2f(Lb) : -INFINITY;
             }
         } else {
-            co[sidx] = acc;
+            namespace cg = cooperative_groups;
+            cg::cluster_group cluster = cg::this_cluster();
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int slot = 16 * warp + 4 * j;
+                const int owner = slot / sp;
+                float* dst = cluster.map_shared_rank(ro, owner) +
+                             (size_t)(split * 32 + lane) * pitch + (slot - owner * sp);
+                *reinterpret_cast<float4*>(dst) = acc[j];
+            }
+            if (warp == 0 && q4 == 0) {
+                for (int c = 0; c < nsplit; ++c) {
+                    float* d = cluster.map_shared_rank(rml, c) + split * 2 * kRows;
+                    *reinterpret_cast<float2*>(d + 2 * ha) = make_float2(Ma, La);
+                    *reinterpret_cast<float2*>(d + 2 * hb) = make_float2(Mb, Lb);
+                }
+            }
         }
     }
     if (nsplit == 1) return;
-
-    // ---------------- combine the CTAs of the cluster (DSMEM) ----------------
-    cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
-    if (tid < kRows) {
-        float mc[kMaxSplit];
-        float M = -INFINITY;
+    cluster_arrive();
+    cluster_wait();
+    // This CTA owns slots [split*sp, split*sp + sp) of every lane.
+    const int s0 = split * sp;
+    const int ngroups = s0 < kSlots ? (min(kSlots, s0 + sp) - s0) / 4 : 0;
+    for (int e = tid; e < ngroups * 32; e += kThreads) {
+        const int ln = e & 31, gq = e >> 5;
+        const int slot = s0 + 4 * gq;
+        const int ha = ln >> 2, hb = ha + 8;
+        float Ma = -INFINITY, Mb = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < kMaxSplit; ++c) {
-            mc[c] = c < nsplit ? cluster.map_shared_rank(cm, c)[tid] : -INFINITY;
-            M = fmaxf(M, mc[c]);
+        for (int r = 0; r < kMaxSplit; ++r) {
+            if (r < nsplit) {
+                Ma = fmaxf(Ma, rml[(r * kRows + ha) * 2]);
+                Mb = fmaxf(Mb, rml[(r * kRows + hb) * 2]);
+            }
         }
+        const float ba = Ma == -INFINITY ? 0.f : Ma, bb = Mb == -INFINITY ? 0.f : Mb;
+        float La = 0.f, Lb = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int r = 0; r < kMaxSplit; ++r) {
+            if (r < nsplit) {
+                const float2 xa = *reinterpret_cast<const float2*>(rml + (r * kRows + ha) * 2);
+                const float2 xb = *reinterpret_cast<const float2*>(rml + (r * kRows + hb) * 2);
+                const float fa = exp2f(xa.x - ba), fb = exp2f(xb.x - bb);
+                La += fa * xa.y;
+                Lb += fb * xb.y;
+                const float4 v = *reinterpret_cast<const float4*>(ro + (size_t)(r * 32 + ln) * pitch + 4 * gq);
+                acc.x += fa * v.x;
+                acc.y += fa * v.y;
+                acc.z += fb * v.z;
+                acc.w += fb * v.w;
+            }
+        }
+        const float ia = La > 0.f ? 1.f / La : 0.f, ib = Lb > 0.f ? 1.f / Lb : 0.f;
+        const int d = 64 * (slot >> 5) + 16 * (ln & 3) + ((slot >> 2) & 7);
+        if (ha < G) {
+            orow[ha * kHD + d] = __float2bfloat16_rn(acc.x * ia);
+            orow[ha * kHD + d + 8] = __float2bfloat16_rn(acc.y * ia);
+        }
+        if (hb < G) {
+            orow[hb * kHD + d] = __float2bfloat16_rn(acc.z * ib);
+            orow[hb * kHD + d + 8] = __float2bfloat16_rn(acc.w * ib);
+        }
+    }
+    if (lse != nullptr && split == 0 && tid < G) {
+        float M = -INFINITY;
+        for (int r = 0; r < nsplit; ++r) M = fmaxf(M, rml[(r * kRows + tid) * 2]);
         const float base = M == -INFINITY ? 0.f : M;
         float L = 0.f;
-#pragma unroll
-        for (int c = 0; c < kMaxSplit; ++c) {
-            const float f = c < nsplit ? exp2f(mc[c] - base) : 0.f;
-            xf[c * kRows + tid] = f;
-            if (c < nsplit) L += f * cluster.map_shared_rank(cl, c)[tid];
-        }
-        xl[tid] = L > 0.f ? 1.f / L : 0.f;
-        if (lse != nullptr && split == 0 && tid < G)
-            lse[(size_t)row * H_q + (size_t)g * G + tid] = L > 0.f ? M + log2f(L) : -INFINITY;
+        for (int r = 0; r < nsplit; ++r)
+            L += exp2f(rml[(r * kRows + tid) * 2] - base) * rml[(r * kRows + tid) * 2 + 1];
+        lse[(size_t)row * H_q + (size_t)g * G + tid] = L > 0.f ? M + log2f(L) : -INFINITY;
     }
-    __syncthreads();
-    const int chunk = (kElems + nsplit - 1) / nsplit;
-    const int e0 = split * chunk, e1 = min(kElems, e0 + chunk);
-    for (int sidx = e0 + tid; sidx < e1; sidx += kThreads) {
-        const int ln = sidx & 31, oi = sidx >> 5, e = oi & 3;
-        const int head = (ln >> 2) + 8 * (e >> 1);
-        float v[kMaxSplit];
-#pragma unroll
-        for (int c = 0; c < kMaxSplit; ++c) v[c] = c < nsplit ? cluster.map_shared_rank(co, c)[sidx] : 0.f;
-        float acc = 0.f;
-#pragma unroll
-        for (int c = 0; c < kMaxSplit; ++c) acc += xf[c * kRows + head] * v[c];
-        if (head < G) {
-            const int dim = 64 * (oi >> 5) + 16 * (ln & 3) + 8 * (e & 1) + ((oi >> 2) & 7);
-            orow[head * kHD + dim] = __float2bfloat16_rn(acc * xl[head]);
-        }
-    }
-    cluster.sync();  // keep this CTA's partial alive until every reader is done
 }
 
 }  // namespace lci

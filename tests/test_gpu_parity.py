@@ -320,6 +320,23 @@ def test_decode_attention_deep_ring_uneven_splits(B, H_kv):
         assert_out_close(out_f.reshape(-1, cfg.H_q, cfg.hd), ref_out, cfg.torch_dtype, "one call")
 
 
+@pytest.mark.parametrize("B,H_kv,topk", [(300, 1, 3), (150, 1, 4), (100, 1, 4), (40, 1, 4),
+                                         (1, 1, 5), (3, 2, 5), (1, 1, 6), (1, 1, 7), (2, 1, 9)])
+def test_decode_attention_every_cluster_size(B, H_kv, topk):
+    """Decode shapes that split each (row, KV head) pair over 1 to 8 CTAs of a
+    cluster (the split count follows from the pairs and the units per pair):
+    300 pairs run one CTA each, 150 and 100 pairs clusters of 2 and 3, 40 pairs
+    of 4, and single rows with 5, 6, 7 or 9 units clusters of 5 to 8, whose
+    output slices are uneven. H_kv = 2 leaves half of the 16 MMA rows unused."""
+    cfg = CONFIGS["decode"].replace(name="splits", B=B, H_kv=H_kv, ctx=1000, q_start=999,
+                                    topk=topk, spare_pages=4)
+    w = generate(cfg)
+    _, ids, out = run_gpu(cfg, upload(w))
+    ref_ids, ref_out = oracle_rows(cfg, w)
+    assert torch.equal(ids.cpu().reshape(-1, cfg.topk), ref_ids)
+    assert_out_close(out.reshape(-1, cfg.H_q, cfg.hd), ref_out, cfg.torch_dtype, "cluster splits")
+
+
 @pytest.mark.parametrize("name", ["decode", "long", "1m_decode"])
 def test_one_launch_decode_step_over_many_calls(name):
     """The one-launch decode step (persistent CTAs claiming scoring chunks, then
