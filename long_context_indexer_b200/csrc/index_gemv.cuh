@@ -32,6 +32,21 @@ __device__ __forceinline__ float dot_chunk(const uint4& raw, const float* q, __n
            d.x * q[6] + d.y * q[7];
 }
 
+// Dot product of 16 bytes of a key with 16 bytes of the query, both packed.
+__device__ __forceinline__ float dot16(const uint4& k, const uint4& q, float) {
+    return __uint_as_float(k.x) * __uint_as_float(q.x) + __uint_as_float(k.y) * __uint_as_float(q.y) +
+           __uint_as_float(k.z) * __uint_as_float(q.z) + __uint_as_float(k.w) * __uint_as_float(q.w);
+}
+
+__device__ __forceinline__ float dot16(const uint4& k, const uint4& q, __nv_bfloat16) {
+    const float2 a = bf16x2_to_f32(k.x), b = bf16x2_to_f32(k.y);
+    const float2 c = bf16x2_to_f32(k.z), d = bf16x2_to_f32(k.w);
+    const float2 qa = bf16x2_to_f32(q.x), qb = bf16x2_to_f32(q.y);
+    const float2 qc = bf16x2_to_f32(q.z), qd = bf16x2_to_f32(q.w);
+    return a.x * qa.x + a.y * qa.y + b.x * qb.x + b.y * qb.y + c.x * qc.x + c.y * qc.y +
+           d.x * qd.x + d.y * qd.y;
+}
+
 // KV > 0: every block key is KV*32 16-byte chunks (2 KiB for KV = 4) and lane l
 // always owns chunks l + 32*c, so its slice of the query row lives in
 // registers. KV == 0: any size, query row staged in shared memory.
@@ -156,6 +171,138 @@ __global__ void __launch_bounds__(NT) index_gemv_select_kernel(
     if (tid == 0) {
         const unsigned prev = atomicAdd(&counters[row], 1u);
         s_last = (prev == (unsigned)(nchunks - 1));
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    if (tid == 0) counters[row] = 0u;
+    SelectSmem& sel = *reinterpret_cast<SelectSmem*>(dyn_smem);
+    cta_topk_select<NT>(row_scores, chunk_max + (size_t)row * nchunks, vis, chunk_blocks, topk,
+                        ids + (size_t)row * topk, sel);
+    if (ready != nullptr) {  // publish the row to a consumer running concurrently
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            st_release_gpu(ready + row, 1u);
+        }
+    }
+}
+
+// Streaming form for 2 KiB block keys (K = 1024 bf16 or 512 fp32), the decode
+// schedule. Grid rows x ncta (ncta fastest), sized by the host so that every
+// CTA is resident at once: CTA `part` of a row scores blocks
+// [part*cta_blocks, +cta_blocks) of the visible range, streaming them through
+// a two-stage ring of NW blocks (one per warp) filled by bulk copies, so its
+// loads stay in flight back to back instead of waiting for a later wave. It
+// records the maximum key of every `chunk_blocks` blocks (cta_blocks is a
+// multiple of chunk_blocks); the last CTA of the row selects as above.
+namespace ixs {
+constexpr int kStages = 2;
+constexpr int kRowBytes = 2048;
+template <int NT> constexpr int smem_bytes() {
+    return kStages * (NT / 32) * kRowBytes > (int)sizeof(SelectSmem) ? kStages * (NT / 32) * kRowBytes
+                                                                      : (int)sizeof(SelectSmem);
+}
+}  // namespace ixs
+
+template <typename T, int NT>
+__global__ void __launch_bounds__(NT) index_stream_select_kernel(
+    const T* __restrict__ q_c, const T* __restrict__ k_c, int S, int nb_max, int bs,
+    const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ q_start, int topk,
+    int chunk_blocks, int cta_blocks, int ncta, int nchunks, float* __restrict__ scores,
+    uint32_t* __restrict__ chunk_max, unsigned int* __restrict__ counters,
+    int32_t* __restrict__ ids, unsigned int* __restrict__ ready,
+    const int32_t* __restrict__ page_table, int num_pages) {
+    constexpr int NW = NT / 32;
+    constexpr int KV = ixs::kRowBytes / (16 * 32);  // 16-byte pieces per lane of a key
+    constexpr int kStageBytes = NW * ixs::kRowBytes;
+    constexpr int kMaxUnits = 64;  // chunk maxima one CTA records
+    extern __shared__ __align__(128) unsigned char dyn_smem[];
+    __shared__ uint64_t bars[ixs::kStages];
+    __shared__ uint32_t s_umax[kMaxUnits];
+    __shared__ int s_last;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int row = blockIdx.x / ncta, part = blockIdx.x - row * ncta;
+    // The row's publication flag starts every call cleared (see the kernel above).
+    if (ready != nullptr && part == 0) {
+        if (tid == 0) {
+            ready[row] = 0u;
+            __threadfence();
+        }
+        __syncthreads();
+    }
+    pdl_trigger();
+    const int b = row / S, s = row - b * S;
+    const long long p = (long long)__ldg(&q_start[b]) + s;
+    const int vis = visible_blocks(p, __ldg(&ctx_len[b]), bs, nb_max);
+    const int j0 = part * cta_blocks;
+    const int j1 = min(j0 + cta_blocks, vis);
+    const int nst = j0 < j1 ? (j1 - j0 + NW - 1) / NW : 0;  // stages of work
+    float* row_scores = scores + (size_t)row * nb_max;
+    const unsigned char* kbase = reinterpret_cast<const unsigned char*>(k_c);
+    // Stage `it` covers blocks j0 + it*NW .. +NW: one contiguous copy of k_c, or
+    // one copy per block at the block's page.
+    auto issue = [&](int it) {
+        const int a = j0 + it * NW, e = min(a + NW, j1);
+        unsigned char* dst = dyn_smem + (it % ixs::kStages) * kStageBytes;
+        uint64_t* bar = &bars[it % ixs::kStages];
+        mbar_arrive_expect_tx(bar, (uint32_t)((e - a) * ixs::kRowBytes));
+        if (page_table == nullptr) {
+            bulk_load(dst, kbase + ((size_t)b * nb_max + a) * ixs::kRowBytes,
+                      (uint32_t)((e - a) * ixs::kRowBytes), bar);
+        } else {
+            for (int j = a; j < e; ++j) {
+                int page = page_table[(size_t)b * nb_max + j];
+                if (page < 0 || page >= num_pages) {
+                    raise_status(kStatusBadPage);
+                    page = 0;  // keep the copy in bounds; the result is flagged
+                }
+                bulk_load(dst + (j - a) * ixs::kRowBytes, kbase + (size_t)page * ixs::kRowBytes,
+                          ixs::kRowBytes, bar);
+            }
+        }
+    };
+    if (tid == 0) {
+        for (int i = 0; i < ixs::kStages; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+        for (int it = 0; it < nst && it < ixs::kStages; ++it) issue(it);
+    }
+    for (int u = tid; u < kMaxUnits; u += NT) s_umax[u] = 0u;  // below every real key
+    // this lane's slice of the query row: pieces lane + 32*c, kept packed
+    uint4 qv[KV];
+    const uint4* qrow = reinterpret_cast<const uint4*>(q_c + (size_t)row * (ixs::kRowBytes / sizeof(T)));
+#pragma unroll
+    for (int c = 0; c < KV; ++c) qv[c] = __ldg(qrow + lane + 32 * c);
+    __syncthreads();
+    bool ok = true;
+    for (int it = 0; it < nst; ++it) {
+        const int st = it % ixs::kStages;
+        ok = ok && mbar_wait(&bars[st], (uint32_t)((it / ixs::kStages) & 1));
+        const int j = j0 + it * NW + warp;
+        if (ok && j < j1) {
+            const uint4* kr = reinterpret_cast<const uint4*>(dyn_smem + st * kStageBytes +
+                                                             warp * ixs::kRowBytes);
+            float acc = 0.f;
+#pragma unroll
+            for (int c = 0; c < KV; ++c) acc += dot16(kr[lane + 32 * c], qv[c], T());
+            acc = warp_sum(acc);
+            if (lane == 0) {
+                row_scores[j] = acc;
+                atomicMax(&s_umax[(j - j0) / chunk_blocks], score_key(acc));
+            }
+        }
+        __syncthreads();  // stage st is read: refill it
+        if (tid == 0 && ok && it + ixs::kStages < nst) issue(it + ixs::kStages);
+    }
+    if (j0 < j1) {
+        const int u0 = j0 / chunk_blocks, nu = (j1 - j0 + chunk_blocks - 1) / chunk_blocks;
+        for (int u = tid; u < nu; u += NT) chunk_max[(size_t)row * nchunks + u0 + u] = s_umax[u];
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        const unsigned prev = atomicAdd(&counters[row], 1u);
+        s_last = (prev == (unsigned)(ncta - 1));
     }
     __syncthreads();
     if (!s_last) return;

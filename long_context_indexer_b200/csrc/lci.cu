@@ -88,6 +88,10 @@ constexpr int kIndexMaxSmem = 65536 + 1024;
 struct IndexPlan {
     int chunk_blocks, nchunks;
     bool qreg;  // 2 KiB block keys: query slice in registers
+    // 2 KiB block keys take the streaming kernel: chunk maxima every s_chunk
+    // blocks, s_nchunks per row (never more than the layout holds)
+    bool stream;
+    int s_chunk, s_nchunks;
     size_t off_counters, off_scores, off_chunk_max, bytes;
     size_t smem;
 };
@@ -117,6 +121,10 @@ IndexPlan plan_index(int32_t batch, int32_t S, int32_t K, int32_t nb_max, size_t
     pl.off_chunk_max = pl.off_scores + align_up((size_t)rows * nb_max * sizeof(float));
     pl.bytes = pl.off_chunk_max + align_up((size_t)rows * nchunks_alloc * sizeof(uint32_t));
     pl.qreg = row_bytes == 2048;
+    pl.stream = row_bytes == 2048;
+    pl.s_chunk = std::max(8, index_chunk(rows, K, nb_max, 4));
+    while ((nb_max + pl.s_chunk - 1) / pl.s_chunk > lci::kMaxChunks) pl.s_chunk *= 2;
+    pl.s_nchunks = (nb_max + pl.s_chunk - 1) / pl.s_chunk;
     const size_t stage = (size_t)chunk * row_bytes + (pl.qreg ? 0 : (size_t)K * sizeof(float));
     const size_t sel = sizeof(lci::SelectSmem);
     pl.smem = stage > sel ? stage : sel;
@@ -142,12 +150,65 @@ lci_status check_index_args(int32_t batch, int32_t S, int32_t H_i, int32_t d_c, 
     return LCI_OK;
 }
 
+// CTAs of the streaming index kernel the device holds at once.
+template <typename T>
+int index_stream_slots() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    static std::mutex mu;
+    static int slots[64] = {0};
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= 64) return 0;
+    if (slots[dev] == 0) {
+        int sms = 0, per_sm = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                &per_sm, lci::index_stream_select_kernel<T, kIndexThreads>, kIndexThreads,
+                lci::ixs::smem_bytes<kIndexThreads>()) != cudaSuccess)
+            return 0;
+        slots[dev] = sms * std::max(1, per_sm);
+    }
+    return slots[dev];
+}
+
+template <typename T>
+lci_status launch_index_stream(const void* q_c, const void* k_c, int32_t batch, int32_t S,
+                               int32_t bs, int32_t nb_max, const int32_t* ctx_len,
+                               const int32_t* q_start, int32_t topk, int32_t* ids, void* ws,
+                               const IndexPlan& pl, cudaStream_t st, unsigned int* ready,
+                               const int32_t* page_table, int32_t num_pages) {
+    const long long rows = (long long)batch * S;
+    const int slots = index_stream_slots<T>();
+    if (slots <= 0) return fail(LCI_ERR_CUDA, "index_select: device query failed");
+    // Blocks per CTA: whole chunks, as few as keep every CTA resident at once,
+    // and at most 64 chunks (the chunk maxima one CTA records).
+    const long long per_row = std::max(1ll, slots / rows);
+    const long long units = (nb_max + pl.s_chunk - 1) / pl.s_chunk;
+    long long cta_units = (units + per_row - 1) / per_row;
+    cta_units = std::min(std::max(cta_units, 1ll), 64ll);
+    const int cta_blocks = (int)(cta_units * pl.s_chunk);
+    const int ncta = (nb_max + cta_blocks - 1) / cta_blocks;
+    const long long grid = rows * ncta;
+    if (grid >= (1ll << 31)) return fail(LCI_ERR_UNSUPPORTED, "index_select: grid too large");
+    char* w = static_cast<char*>(ws);
+    lci::index_stream_select_kernel<T, kIndexThreads>
+        <<<(unsigned)grid, kIndexThreads, lci::ixs::smem_bytes<kIndexThreads>(), st>>>(
+            static_cast<const T*>(q_c), static_cast<const T*>(k_c), S, nb_max, bs, ctx_len, q_start,
+            topk, pl.s_chunk, cta_blocks, ncta, pl.s_nchunks,
+            reinterpret_cast<float*>(w + pl.off_scores), reinterpret_cast<uint32_t*>(w + pl.off_chunk_max),
+            reinterpret_cast<unsigned int*>(w + pl.off_counters), ids, ready, page_table, num_pages);
+    return check_launch("index_select");
+}
+
 template <typename T>
 lci_status launch_index_gemv(const void* q_c, const void* k_c, int32_t batch, int32_t S, int32_t K,
                              int32_t bs, int32_t nb_max, const int32_t* ctx_len,
                              const int32_t* q_start, int32_t topk, int32_t* ids, void* ws,
                              const IndexPlan& pl, cudaStream_t st, unsigned int* ready = nullptr,
                              const int32_t* page_table = nullptr, int32_t num_pages = 0) {
+    if (pl.stream)
+        return launch_index_stream<T>(q_c, k_c, batch, S, bs, nb_max, ctx_len, q_start, topk, ids,
+                                      ws, pl, st, ready, page_table, num_pages);
     constexpr int KV = 2048 / (16 * 32);
     auto kern = pl.qreg ? lci::index_gemv_select_kernel<T, kIndexThreads, KV>
                         : lci::index_gemv_select_kernel<T, kIndexThreads, 0>;

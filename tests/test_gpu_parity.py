@@ -149,6 +149,38 @@ def test_ties_break_to_lower_block_id():
     assert torch.equal(ids.cpu().reshape(-1, cfg.topk), ref_ids)
 
 
+@pytest.mark.parametrize("ctx,topk,mode", [
+    (32768, 200, "grid"),    # k above the sorted-list pass: radix select over 512 blocks
+    (262144, 200, "grid"),   # the same over 4096 blocks
+    (262144, 64, "zero"),    # all scores equal: every chunk survives pruning -> radix select
+    (262144, 64, "few"),     # few distinct scores: ties at the pruning bound
+    (70400, 128, "grid"),    # 1100 blocks, k at the sorted pass's limit, pruned
+    (8192, 128, "grid"),     # k == n: all 128 visible blocks, in rank order
+    (65536, 1, "grid"),      # k == 1 over 1024 blocks (one sorted-list pass, 4 per lane)
+    (16384, 9, "grid"),      # 256 blocks: one composite per lane
+])
+def test_select_paths(ctx, topk, mode):
+    """Every branch of the CTA top-k: one sorted-list pass (32, 64 or 128
+    composites per warp), pruning by chunk maxima then a sorted-list pass, and
+    the exact radix select for large k or candidate sets that ties inflate."""
+    cfg = CONFIGS["decode"].replace(name="sel", B=2, ctx=ctx, q_start=ctx - 1, topk=topk)
+    w = generate(cfg, with_kv=False)
+    dt = w["q_c"].dtype
+    if mode == "zero":
+        w["q_c"].zero_()
+    elif mode == "few":
+        w["q_c"] = (w["q_c"] > 1).to(dt) * 0.0625
+        w["k_c"] = (w["k_c"] > 0).to(dt) * 0.0625
+    d = upload(w)
+    ids = lci.index_select(d["q_c"], d["k_c"], cfg.bs, d["ctx_len"], d["q_start"], topk)
+    torch.cuda.synchronize()
+    lci.get_device_status()
+    ref = oracle.index_select(w["q_c"], w["k_c"], cfg.bs, w["ctx_len"], w["q_start"], topk)
+    assert torch.equal(ids.cpu().reshape(-1, topk), ref.reshape(-1, topk))
+    if mode == "zero":
+        assert (ids.cpu().reshape(-1, topk) == torch.arange(topk, dtype=torch.int32)).all()
+
+
 def test_extreme_grid_values_are_exact():
     cfg = SMALL.replace(H_i=8, d_c=128, topk=6, S=2, q_start=998)
     w = generate(cfg)
