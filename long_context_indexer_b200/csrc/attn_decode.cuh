@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
     int num_pages, int H_kv, int bs, int S, int H_q, const int32_t* __restrict__ ids, int topk,
     const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ q_start, float scale_log2,
     __nv_bfloat16* __restrict__ out, int nsplit, const unsigned int* __restrict__ ready,
-    float* __restrict__ lse) {
+    float* __restrict__ lse, const unsigned long long* __restrict__ picks) {
     using namespace dec;
     namespace cg = cooperative_groups;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -282,14 +282,19 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
     // after writing the row's ids (bounded wait on this row's flag only). The
     // library's producer clears its flags itself before this grid can start. A
     // row whose flag never comes is skipped (zero output, time-out status).
+    // A producer may instead publish each pick as (block id, page) in
+    // picks[row][rank] (kPickPending until written): the producer warp then
+    // polls exactly the picks it needs, with no flag, id or table round trip.
     __shared__ int s_alive;
-    if (ready == nullptr) {
-        pdl_wait();
-    } else {
-        if (tid == 0) s_alive = wait_flag_set(ready + row) ? 1 : 0;
-        __syncthreads();
+    if (picks == nullptr) {
+        if (ready == nullptr) {
+            pdl_wait();
+        } else {
+            if (tid == 0) s_alive = wait_flag_set(ready + row) ? 1 : 0;
+            __syncthreads();
+        }
     }
-    const bool alive = ready == nullptr || s_alive != 0;
+    const bool alive = picks != nullptr || ready == nullptr || s_alive != 0;
 
     float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
     float o[2][8][4];
@@ -311,9 +316,17 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
             int t0 = -1, y = 0;
             if (u < u1 && alive) {
                 const int i = u / tiles_per_block, sub = u - i * tiles_per_block;
-                const int j = __ldcg(row_ids + i);
+                int j, page = -1;
+                if (picks != nullptr) {
+                    const unsigned long long v =
+                        wait_slot(picks + (size_t)row * topk + i, kPickPending, ~0ull);
+                    j = (int)(unsigned)(v >> 32);
+                    page = (int)(unsigned)(v & 0xffffffffull);
+                } else {
+                    j = __ldcg(row_ids + i);
+                    if (j >= 0 && j < nb_max) page = table[(size_t)b * nb_max + j];
+                }
                 if (j >= 0 && j < nb_max) {
-                    const int page = table[(size_t)b * nb_max + j];
                     if (page < 0 || page >= num_pages) {
                         raise_status(kStatusBadPage);
                     } else if ((long long)j * bs + sub * kTile <= last) {

@@ -18,6 +18,9 @@ enum : unsigned int {
     kStatusTimeout = 1u << 2,     // a bounded device wait gave up
 };
 
+// A published (block id << 32 | page) pick not yet written: both INT_MIN.
+constexpr unsigned long long kPickPending = 0x8000000080000000ull;
+
 // Limit of every bounded device wait, in nanoseconds of global time. Set from
 // the host (lci_set_wait_limit_ns) between launches; 2 s unless changed.
 __device__ unsigned long long g_wait_limit_ns = 2000000000ull;

@@ -205,6 +205,11 @@ template <int NT> constexpr int smem_bytes() {
 }
 }  // namespace ixs
 
+//
+// With `picks` (and the KV cache's block `table`), the row's selection is also
+// published for an attention kernel running concurrently: picks[row][r] is
+// (block id << 32 | page) of rank r, -1 for both past the selection, and
+// kPickPending until written (the row's first CTA resets it every call).
 template <typename T, int NT>
 __global__ void __launch_bounds__(NT) index_stream_select_kernel(
     const T* __restrict__ q_c, const T* __restrict__ k_c, int S, int nb_max, int bs,
@@ -212,7 +217,8 @@ __global__ void __launch_bounds__(NT) index_stream_select_kernel(
     int chunk_blocks, int cta_blocks, int ncta, int nchunks, float* __restrict__ scores,
     uint32_t* __restrict__ chunk_max, unsigned int* __restrict__ counters,
     int32_t* __restrict__ ids, unsigned int* __restrict__ ready,
-    const int32_t* __restrict__ page_table, int num_pages) {
+    const int32_t* __restrict__ page_table, int num_pages,
+    const int32_t* __restrict__ table, unsigned long long* __restrict__ picks) {
     constexpr int NW = NT / 32;
     constexpr int KV = ixs::kRowBytes / (16 * 32);  // 16-byte pieces per lane of a key
     constexpr int kStageBytes = NW * ixs::kRowBytes;
@@ -223,18 +229,19 @@ __global__ void __launch_bounds__(NT) index_stream_select_kernel(
     __shared__ int s_last;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int row = blockIdx.x / ncta, part = blockIdx.x - row * ncta;
-    // The row's publication flag starts every call cleared (see the kernel above).
-    if (ready != nullptr && part == 0) {
-        if (tid == 0) {
-            ready[row] = 0u;
-            __threadfence();
-        }
+    const int b = row / S, s = row - b * S;
+    const int qs = __ldg(&q_start[b]), cl = __ldg(&ctx_len[b]);  // in flight during the clear
+    // The row's publication flag (or picks) starts every call cleared (see the
+    // kernel above).
+    if (part == 0 && (ready != nullptr || picks != nullptr)) {
+        if (ready != nullptr && tid == 0) ready[row] = 0u;
+        if (picks != nullptr)
+            for (int r = tid; r < topk; r += NT) picks[(size_t)row * topk + r] = kPickPending;
+        __threadfence();
         __syncthreads();
     }
     pdl_trigger();
-    const int b = row / S, s = row - b * S;
-    const long long p = (long long)__ldg(&q_start[b]) + s;
-    const int vis = visible_blocks(p, __ldg(&ctx_len[b]), bs, nb_max);
+    const int vis = visible_blocks((long long)qs + s, cl, bs, nb_max);
     const int j0 = part * cta_blocks;
     const int j1 = min(j0 + cta_blocks, vis);
     const int nst = j0 < j1 ? (j1 - j0 + NW - 1) / NW : 0;  // stages of work
@@ -298,25 +305,38 @@ __global__ void __launch_bounds__(NT) index_stream_select_kernel(
         const int u0 = j0 / chunk_blocks, nu = (j1 - j0 + chunk_blocks - 1) / chunk_blocks;
         for (int u = tid; u < nu; u += NT) chunk_max[(size_t)row * nchunks + u0 + u] = s_umax[u];
     }
-    __threadfence();
-    __syncthreads();
+    __syncthreads();  // this CTA's scores and chunk maxima are written
     if (tid == 0) {
-        const unsigned prev = atomicAdd(&counters[row], 1u);
+        // the arrival releases them; the row's last arrival acquires every
+        // earlier arrival's (the CTA barriers carry both to the other threads)
+        const unsigned prev = atom_add_acq_rel_gpu(&counters[row], 1u);
         s_last = (prev == (unsigned)(ncta - 1));
     }
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
     if (tid == 0) counters[row] = 0u;
     SelectSmem& sel = *reinterpret_cast<SelectSmem*>(dyn_smem);
+    int32_t* row_ids = ids + (size_t)row * topk;
+    if (picks != nullptr) {
+        // the table row is warm in L2 by the time the ranks are known
+        const int32_t* trow = table + (size_t)b * nb_max;
+        for (int l = tid * 32; l < nb_max; l += NT * 32) prefetch_l2(trow + l);
+        unsigned long long* row_picks = picks + (size_t)row * topk;
+        cta_topk_select<NT>(
+            row_scores, chunk_max + (size_t)row * nchunks, vis, chunk_blocks, topk,
+            [=](int rank, int id) {
+                row_ids[rank] = id;
+                const int page = id >= 0 ? __ldg(trow + id) : -1;
+                row_picks[rank] = ((unsigned long long)(unsigned)id << 32) | (unsigned)page;
+            },
+            sel);
+        return;
+    }
     cta_topk_select<NT>(row_scores, chunk_max + (size_t)row * nchunks, vis, chunk_blocks, topk,
-                        ids + (size_t)row * topk, sel);
+                        row_ids, sel);
     if (ready != nullptr) {  // publish the row to a consumer running concurrently
-        __syncthreads();
-        if (tid == 0) {
-            __threadfence();
-            st_release_gpu(ready + row, 1u);
-        }
+        __syncthreads();      // every id is written
+        if (tid == 0) st_release_gpu(ready + row, 1u);
     }
 }
 

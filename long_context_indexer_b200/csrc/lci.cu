@@ -176,7 +176,8 @@ lci_status launch_index_stream(const void* q_c, const void* k_c, int32_t batch, 
                                int32_t bs, int32_t nb_max, const int32_t* ctx_len,
                                const int32_t* q_start, int32_t topk, int32_t* ids, void* ws,
                                const IndexPlan& pl, cudaStream_t st, unsigned int* ready,
-                               const int32_t* page_table, int32_t num_pages) {
+                               const int32_t* page_table, int32_t num_pages, const int32_t* table,
+                               unsigned long long* picks) {
     const long long rows = (long long)batch * S;
     const int slots = index_stream_slots<T>();
     if (slots <= 0) return fail(LCI_ERR_CUDA, "index_select: device query failed");
@@ -196,7 +197,8 @@ lci_status launch_index_stream(const void* q_c, const void* k_c, int32_t batch, 
             static_cast<const T*>(q_c), static_cast<const T*>(k_c), S, nb_max, bs, ctx_len, q_start,
             topk, pl.s_chunk, cta_blocks, ncta, pl.s_nchunks,
             reinterpret_cast<float*>(w + pl.off_scores), reinterpret_cast<uint32_t*>(w + pl.off_chunk_max),
-            reinterpret_cast<unsigned int*>(w + pl.off_counters), ids, ready, page_table, num_pages);
+            reinterpret_cast<unsigned int*>(w + pl.off_counters), ids, ready, page_table, num_pages,
+            table, picks);
     return check_launch("index_select");
 }
 
@@ -205,10 +207,11 @@ lci_status launch_index_gemv(const void* q_c, const void* k_c, int32_t batch, in
                              int32_t bs, int32_t nb_max, const int32_t* ctx_len,
                              const int32_t* q_start, int32_t topk, int32_t* ids, void* ws,
                              const IndexPlan& pl, cudaStream_t st, unsigned int* ready = nullptr,
-                             const int32_t* page_table = nullptr, int32_t num_pages = 0) {
+                             const int32_t* page_table = nullptr, int32_t num_pages = 0,
+                             const int32_t* table = nullptr, unsigned long long* picks = nullptr) {
     if (pl.stream)
         return launch_index_stream<T>(q_c, k_c, batch, S, bs, nb_max, ctx_len, q_start, topk, ids,
-                                      ws, pl, st, ready, page_table, num_pages);
+                                      ws, pl, st, ready, page_table, num_pages, table, picks);
     constexpr int KV = 2048 / (16 * 32);
     auto kern = pl.qreg ? lci::index_gemv_select_kernel<T, kIndexThreads, KV>
                         : lci::index_gemv_select_kernel<T, kIndexThreads, 0>;
@@ -466,7 +469,7 @@ lci_status launch_attn_decode(const void* q, int32_t batch, int32_t S, int32_t H
                               const int32_t* ids, int32_t topk, const int32_t* ctx_len,
                               const int32_t* q_start, float scale, void* out, cudaStream_t st,
                               const unsigned int* ready = nullptr, bool early_start = true,
-                              float* lse = nullptr) {
+                              float* lse = nullptr, const unsigned long long* picks = nullptr) {
     CUtensorMap tm_k, tm_v;
     lci_status s = pool_maps(t, k_pool, v_pool, &tm_k, &tm_v);
     if (s != LCI_OK) return s;
@@ -506,7 +509,7 @@ lci_status launch_attn_decode(const void* q, int32_t batch, int32_t S, int32_t H
     cudaError_t e = cudaLaunchKernelEx(
         &cfg, kern, tm_k, tm_v, static_cast<const __nv_bfloat16*>(q),
         t->d_table, t->max_blocks, t->num_pages, t->num_kv_heads, t->block_size, S, H_q, ids, topk,
-        ctx_len, q_start, scale_log2, static_cast<__nv_bfloat16*>(out), nsplit, ready, lse);
+        ctx_len, q_start, scale_log2, static_cast<__nv_bfloat16*>(out), nsplit, ready, lse, picks);
     if (e != cudaSuccess) return fail(LCI_ERR_CUDA, "sparse_attn: %s", cudaGetErrorString(e));
     return check_launch("sparse_attn");
 }
@@ -1099,6 +1102,7 @@ struct DecodePlan {
     bool fused;                 // the one-launch persistent kernel
     int nsplit;                 // attention splits per (row, KV head) pair (fused)
     size_t off_ready;           // publication flags of the two-kernel form (0 / 1)
+    size_t off_picks;           // published (block id, page) picks of the two-kernel form
     size_t off_pready;          // publication flags of the one-launch form (call epochs)
     size_t off_split, off_sync, off_part, bytes;
 };
@@ -1117,7 +1121,8 @@ DecodePlan plan_decode(int32_t batch, int32_t S, int32_t K, int32_t nb_max, size
     d.fused = fused;
     const size_t rows = (size_t)batch * S;
     d.off_ready = align_up(d.ix.bytes);
-    size_t end = d.off_ready + align_up(rows * sizeof(unsigned int));
+    d.off_picks = d.off_ready + align_up(rows * sizeof(unsigned int));
+    size_t end = d.off_picks + align_up(rows * (size_t)topk * sizeof(unsigned long long));
     if (fused) {
         // splits: about two attention items per SM, at least two 64-token tiles each
         const long long pairs = (long long)rows * t->num_kv_heads;
@@ -1244,7 +1249,20 @@ static lci_status sparse_decode_impl(const void* q_c, const void* k_c, lci_dtype
         return launch_decode_fused(q_c, k_c, batch, S, nb_max, d_ctx_len, d_q_start, topk, q, H_q,
                                    k_pool, v_pool, table, scale, d_ids, out, w, pl, cs);
     if (dtype == LCI_BF16 && decode_kernel_fits(table, H_q, k_pool, v_pool)) {
-        // rows are published one by one and attended as soon as they are ready
+        // rows are published one by one and attended as soon as they are ready:
+        // as (block id, page) picks from the streaming index kernel, else as a
+        // flag per row
+        if (pl.ix.stream) {
+            unsigned long long* picks = reinterpret_cast<unsigned long long*>(w + pl.off_picks);
+            st = launch_index_gemv<__nv_bfloat16>(q_c, k_c, batch, S, K, table->block_size, nb_max,
+                                                  d_ctx_len, d_q_start, topk, d_ids, workspace,
+                                                  pl.ix, cs, nullptr, nullptr, 0, table->d_table,
+                                                  picks);
+            if (st != LCI_OK) return st;
+            return launch_attn_decode(q, batch, S, H_q, k_pool, v_pool, table, d_ids, topk,
+                                      d_ctx_len, d_q_start, scale, out, cs, nullptr, true, nullptr,
+                                      picks);
+        }
         unsigned int* ready = reinterpret_cast<unsigned int*>(w + pl.off_ready);
         st = launch_index_gemv<__nv_bfloat16>(q_c, k_c, batch, S, K, table->block_size, nb_max,
                                               d_ctx_len, d_q_start, topk, d_ids, workspace, pl.ix,

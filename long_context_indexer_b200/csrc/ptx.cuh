@@ -138,9 +138,52 @@ __device__ __forceinline__ unsigned int ld_relaxed_gpu(const unsigned int* p) {
 __device__ __forceinline__ void st_release_gpu(unsigned int* p, unsigned int v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+// Atomic add with acquire-release semantics at GPU scope: publishes what this
+// CTA wrote before its barrier and, for the last arrival, acquires what the
+// earlier arrivals published. Returns the old value.
+__device__ __forceinline__ unsigned int atom_add_acq_rel_gpu(unsigned int* p, unsigned int v) {
+    unsigned int old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
 
-// Wait until *flag is nonzero (acquire), polling with a growing sleep so that
-// waiting CTAs do not flood L2, for at most g_wait_limit_ns. On time-out it
+__device__ __forceinline__ unsigned long long ld_relaxed_gpu_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Wait until *slot differs from `pending` (the value is the data itself, no
+// other memory is read on its strength), polling back to back for 4 us and then
+// with sleeps, for at most g_wait_limit_ns. On time-out it raises
+// kStatusTimeout and returns `fallback`.
+__device__ __forceinline__ unsigned long long wait_slot(const unsigned long long* slot,
+                                                        unsigned long long pending,
+                                                        unsigned long long fallback) {
+    unsigned long long v = ld_relaxed_gpu_u64(slot);
+    if (v != pending) return v;
+    const unsigned long long t0 = global_ns();
+    const unsigned long long limit = g_wait_limit_ns;
+    unsigned int sleep_ns = 32;
+    for (;;) {
+        const unsigned long long waited = global_ns() - t0;
+        if (waited > 4000ull) {
+            __nanosleep(sleep_ns);
+            sleep_ns = sleep_ns < 256 ? 2 * sleep_ns : 256;
+        }
+        v = ld_relaxed_gpu_u64(slot);
+        if (v != pending) return v;
+        if (waited > limit) {
+            raise_status(kStatusTimeout);
+            return fallback;
+        }
+    }
+}
+
+// Wait until *flag is nonzero (acquire), for at most g_wait_limit_ns. The
+// first 4 us poll back to back (one load in flight per waiting CTA: a flag set
+// meanwhile is seen within about one L2 round trip); after that the polls
+// sleep, growing to 256 ns, so long waits do not flood L2. On time-out it
 // raises kStatusTimeout and returns false.
 __device__ __forceinline__ bool wait_flag_set(const unsigned int* flag) {
     if (ld_acquire_gpu(flag) != 0u) return true;
@@ -148,13 +191,16 @@ __device__ __forceinline__ bool wait_flag_set(const unsigned int* flag) {
     const unsigned long long limit = g_wait_limit_ns;
     unsigned int sleep_ns = 32;
     for (;;) {
-        __nanosleep(sleep_ns);
+        const unsigned long long waited = global_ns() - t0;
+        if (waited > 4000ull) {
+            __nanosleep(sleep_ns);
+            sleep_ns = sleep_ns < 256 ? 2 * sleep_ns : 256;
+        }
         if (ld_acquire_gpu(flag) != 0u) return true;
-        if (global_ns() - t0 > limit) {
+        if (waited > limit) {
             raise_status(kStatusTimeout);
             return false;
         }
-        sleep_ns = sleep_ns < 512 ? 2 * sleep_ns : 512;
     }
 }
 

@@ -302,9 +302,9 @@ __device__ void radix_select_global(const float* scores, int n, int k, SelectSme
 // Rank of every winner among the k winners by (key desc, id asc), one warp
 // per winner (lanes compare 32 at once, a ballot counts those ahead); writes
 // out[rank] = id.
-template <int NT>
+template <int NT, typename Pick>
 __device__ __forceinline__ void rank_winners(const uint32_t* keys, const int32_t* ids, int k,
-                                             int32_t* out) {
+                                             Pick pick) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int e = warp; e < k; e += NT / 32) {
         const uint32_t ke = keys[e];
@@ -319,26 +319,26 @@ __device__ __forceinline__ void rank_winners(const uint32_t* keys, const int32_t
             }
             rank += __popc(__ballot_sync(0xffffffffu, ahead));
         }
-        if (lane == 0) out[rank] = ie;
+        if (lane == 0) pick(rank, ie);
     }
 }
 
 // All NT (<= 256) threads of the CTA call this. scores[0..n) are the row's
 // scores and chunk_max[0..ceil(n/chunk)) the maximum key of every chunk of
-// `chunk` consecutive blocks, both in global memory (L2). Writes
-// out[0..topk): the selected block ids in rank order, then -1. Requires
-// topk <= kMaxTopk.
-template <int NT>
+// `chunk` consecutive blocks, both in global memory (L2). Calls pick(rank, id)
+// once for every rank in [0, topk): the selected block ids in rank order,
+// then -1. Requires topk <= kMaxTopk.
+template <int NT, typename Pick>
 __device__ void cta_topk_select(const float* scores, const uint32_t* chunk_max, int n, int chunk,
-                                int topk, int32_t* out, SelectSmem& sm) {
+                                int topk, Pick pick, SelectSmem& sm) {
     static_assert(NT % 32 == 0 && NT <= 256, "up to 8 warps");
     constexpr int NW = NT / 32;
     constexpr int kPass = NW * 128;  // candidates one sorted-list pass holds
     const int tid = threadIdx.x;
     const int k = n < topk ? n : topk;
-    for (int i = k + tid; i < topk; i += NT) out[i] = -1;
+    for (int i = k + tid; i < topk; i += NT) pick(i, -1);
     if (k <= 0) return;
-    auto emit_id = [&](int rank, uint64_t x) { out[rank] = composite_id(x); };
+    auto emit_id = [&](int rank, uint64_t x) { pick(rank, composite_id(x)); };
     if (k <= kSortMaxK && n <= kPass) {
         sorted_topk<NT>(n, k, [&](int i) { return compose(load_key(scores, i), i); }, sm.lists,
                         emit_id);
@@ -384,7 +384,16 @@ __device__ void cta_topk_select(const float* scores, const uint32_t* chunk_max, 
         __syncthreads();  // the radix pass reuses the list memory
     }
     radix_select_global<NT>(scores, n, k, sm);
-    rank_winners<NT>(sm.rad.win_key, sm.rad.win_id, k, out);
+    rank_winners<NT>(sm.rad.win_key, sm.rad.win_id, k, pick);
+}
+
+// The common case: write the ids to out[0..topk).
+template <int NT>
+__device__ __forceinline__ void cta_topk_select(const float* scores, const uint32_t* chunk_max,
+                                                int n, int chunk, int topk, int32_t* out,
+                                                SelectSmem& sm) {
+    cta_topk_select<NT>(scores, chunk_max, n, chunk, topk, [=](int rank, int id) { out[rank] = id; },
+                        sm);
 }
 
 }  // namespace lci
