@@ -41,14 +41,14 @@ constexpr int kTile = 64;          // tokens per unit
 // one SM when the grid has about one CTA per SM
 constexpr int kStagesShallow = 3;
 constexpr int kStagesDeep = 6;
-constexpr int kConsumers = 4;      // consumer warps, 16 tokens each
-constexpr int kThreads = (kConsumers + 1) * 32;
+constexpr int kConsumers = 4;      // consumer warps of a group, 16 tokens each
+constexpr int kThreads = (kConsumers + 1) * 32;  // one group and the producer
+__host__ __device__ constexpr int threads(int groups) { return (kConsumers * groups + 1) * 32; }
 constexpr int kBox = 64 * 64 * 2;  // one 64x64 bf16 box = 8 KiB
 constexpr int kStageBytes = 4 * kBox;  // K: 2 boxes, V: 2 boxes
 constexpr int kMaxSplit = 8;
 constexpr int kRows = 16;          // query heads per MMA (padded)
 constexpr int kSlots = 64;         // fp32 accumulators per consumer thread
-constexpr int kWoStride = 68;      // floats per lane of a warp partial (16-byte access, no conflicts)
 constexpr int kMetaBytes = 256;    // barriers and unit info after the ring
 // Slots of one cluster CTA's slice of the output (a multiple of 4), and the
 // padded per-lane pitch of a received slice (4 mod 8 floats: 16-byte
@@ -72,27 +72,31 @@ constexpr int smem_bytes(int stages) {
     return stages * kStageBytes + 1024 /*align*/ + kMetaBytes +
            (kRecvFloats + kMaxSplit * kRows * 2) * 4;
 }
-static_assert(kConsumers * (32 * kWoStride + 2 * kRows) * 4 <= 3 * kStageBytes,
-              "warp partials fit in the ring");
+
 }  // namespace dec
 
 __device__ __forceinline__ int tok_perm(int x) { return x ^ ((x & 1) << 2); }
 
-// Four consecutive bf16 outputs: one 8-byte store when the output is 8-byte
-// aligned, else four 2-byte stores.
-__device__ __forceinline__ void store_bf16x4(__nv_bfloat16* p, float a, float b, float c, float d,
-                                             bool vec) {
-    if (vec) {
-        uint2 w;
-        w.x = pack_bf16x2(a, b);
-        w.y = pack_bf16x2(c, d);
-        *reinterpret_cast<uint2*>(p) = w;
-    } else {
-        p[0] = __float2bfloat16_rn(a);
-        p[1] = __float2bfloat16_rn(b);
-        p[2] = __float2bfloat16_rn(c);
-        p[3] = __float2bfloat16_rn(d);
+// N (2 or 4) consecutive bf16 outputs: one 4- or 8-byte store when the output
+// allows it, else N 2-byte stores.
+template <int N>
+__device__ __forceinline__ void store_bf16_run(__nv_bfloat16* p, const float (&v)[N], bool vec) {
+    if constexpr (N == 4) {
+        if (vec) {
+            uint2 w;
+            w.x = pack_bf16x2(v[0], v[1]);
+            w.y = pack_bf16x2(v[2], v[3]);
+            *reinterpret_cast<uint2*>(p) = w;
+            return;
+        }
+    } else if constexpr (N == 2) {
+        if (vec) {
+            *reinterpret_cast<uint32_t*>(p) = pack_bf16x2(v[0], v[1]);
+            return;
+        }
     }
+#pragma unroll
+    for (int j = 0; j < N; ++j) p[j] = __float2bfloat16_rn(v[j]);
 }
 
 // Byte offset of (row r, 16-byte chunk c of the 128-dim row) inside one K or V
@@ -104,13 +108,15 @@ __device__ __forceinline__ uint32_t tile_off(int r, int c) {
 // One 64-token K/V tile (two 64x64 boxes of K then of V, 128-byte swizzle, at
 // shared address kbase) for consumer warp w, which takes tokens 16w..16w+15:
 // S = Q K^T with mma.m16n8k16, the online softmax update of (m, l) for the
-// fragment's two head rows, and O += P V. t0 is the tile's first token;
-// tokens after `last` are masked (their V is never read into the MMA).
+// fragment's two head rows, and O += P V for NH of the two 64-dim halves of the
+// output, starting at half h0. t0 is the tile's first token; tokens after
+// `last` are masked (their V is never read into the MMA).
+template <int NH>
 __device__ __forceinline__ void dec_consume_tile(uint32_t kbase, int w, int g8, int q4, int t0,
                                                  long long last, float scale_log2,
                                                  const uint4 (&qa)[4], const uint4 (&qb)[4],
                                                  float& m_a, float& m_b, float& l_a, float& l_b,
-                                                 float (&o)[2][8][4]) {
+                                                 float (&o)[NH][8][4], int h0 = 0) {
     using namespace dec;
     const long long wt0 = (long long)t0 + 16 * w;  // first token of this warp
     if (wt0 <= last) {
@@ -164,7 +170,7 @@ __device__ __forceinline__ void dec_consume_tile(uint32_t kbase, int w, int g8, 
         l_a = l_a * corr_a + (pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1]);
         l_b = l_b * corr_b + (pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3]);
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
+        for (int h = 0; h < NH; ++h)
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 o[h][i][0] *= corr_a;
@@ -182,7 +188,8 @@ __device__ __forceinline__ void dec_consume_tile(uint32_t kbase, int w, int g8, 
         const bool z0 = partial && wt0 + c0 > last, z1 = partial && wt0 + c1 > last;
         const bool z2 = partial && wt0 + 8 + c0 > last, z3 = partial && wt0 + 8 + c1 > last;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int hh = 0; hh < NH; ++hh) {
+            const int h = h0 + hh;
             uint4 va = lds128(vbase + tile_off(r0, 8 * h + g8));
             uint4 vb = lds128(vbase + tile_off(r1, 8 * h + g8));
             uint4 vc = lds128(vbase + tile_off(r2, 8 * h + g8));
@@ -198,14 +205,17 @@ __device__ __forceinline__ void dec_consume_tile(uint32_t kbase, int w, int g8, 
                 const uint32_t sel = (i & 1) ? 0x7632u : 0x5410u;
                 const uint32_t b0 = __byte_perm(wa[i >> 1], wb[i >> 1], sel);
                 const uint32_t b1 = __byte_perm(wc[i >> 1], wd[i >> 1], sel);
-                mma_bf16_16816(o[h][i], pa0, pa1, pa2, pa3, b0, b1);
+                mma_bf16_16816(o[hh][i], pa0, pa1, pa2, pa3, b0, b1);
             }
         }
     }
 }
 
-template <int kStages>
-__global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
+// kGroups consumer groups of kConsumers warps take alternate ring stages, each
+// with its own softmax state (two groups when the CTA has an SM to itself: the
+// latency of one tile's MMA and softmax chain hides under the other's).
+template <int kStages, int kGroups>
+__global__ void __launch_bounds__(dec::threads(kGroups)) sparse_attn_decode_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ table, int nb_max,
     int num_pages, int H_kv, int bs, int S, int H_q, const int32_t* __restrict__ ids, int topk,
@@ -214,6 +224,13 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
     float* __restrict__ lse, const unsigned long long* __restrict__ picks) {
     using namespace dec;
     namespace cg = cooperative_groups;
+    constexpr int kCW = kConsumers * kGroups;    // consumer warps; warp kCW produces
+    constexpr int kWoS = kSlots + 4;             // partial row pitch (4 mod 8 floats: no conflicts)
+    constexpr int kSlotsPer = kSlots / kCW;      // accumulator slots each thread merges
+    constexpr int kNT = threads(kGroups);
+    static_assert(kGroups == 1 || kGroups == 2, "one or two groups");
+    static_assert(kCW * (32 * kWoS + 2 * kRows) * 4 <= kStages * kStageBytes,
+                  "warp partials fit in the ring");
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -239,7 +256,7 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
         }
         fence_mbar_init();
     }
-    if (warp == kConsumers && lane == 0) {
+    if (warp == kCW && lane == 0) {
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
     }
@@ -253,7 +270,7 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
 
     // Query rows of this pair (independent of the previous kernel's output).
     uint4 qa[4], qb[4];
-    if (warp < kConsumers) {
+    if (warp < kCW) {
         const int ha = g8, hb = g8 + 8;
         const __nv_bfloat16* qrow = q + ((size_t)row * H_q + (size_t)g * G) * kHD;
 #pragma unroll
@@ -271,7 +288,7 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
     const long long p = (long long)q_start[b] + s;
     const long long ctx = ctx_len[b];
     const long long last = p < ctx - 1 ? p : ctx - 1;
-    if (warp == kConsumers) {
+    if (warp == kCW) {
         const int32_t* trow = table + (size_t)b * nb_max;
         const int nlines = min(nb_max, 8192) / 32;  // 128-byte lines of the row
         for (int l = lane; l < nlines; l += 32) prefetch_l2(trow + l * 32);
@@ -305,7 +322,7 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
 #pragma unroll
             for (int e = 0; e < 4; ++e) o[h][i][e] = 0.f;
 
-    if (warp == kConsumers) {
+    if (warp == kCW) {
         // ---------------- producer ----------------
         // Lanes resolve 32 units at a time (block id -> page -> TMA row), so the
         // dependent id and table loads overlap; lane 0 then issues the copies.
@@ -368,14 +385,16 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
         }
     } else {
         // ---------------- consumers ----------------
-        const int w = warp;
-        for (int u = u0, it = 0; u < u1; ++u, ++it) {
+        // group grp takes the stages it = grp, grp + kGroups, ...; warp w of
+        // the group takes tokens 16w..16w+15 of each tile
+        const int grp = warp / kConsumers, w = warp - grp * kConsumers;
+        for (int u = u0 + grp, it = grp; u < u1; u += kGroups, it += kGroups) {
             const int st = it % kStages;
             const bool ok = mbar_wait(&full_bar[st], (it / kStages) & 1);
             const int t0 = info[st];
             if (ok && t0 >= 0)
-                dec_consume_tile(smem_u32(smem + st * kStageBytes), w, g8, q4, t0, last, scale_log2,
-                                 qa, qb, m_a, m_b, l_a, l_b, o);
+                dec_consume_tile(smem_u32(smem + st * kStageBytes), w, g8, q4, t0, last,
+                                 scale_log2, qa, qb, m_a, m_b, l_a, l_b, o);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty_bar[st]);
         }
@@ -392,14 +411,14 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
     //    stores every slice of its partial into the CTA owning that slice
     //    (distributed shared memory), one cluster barrier publishes the stores,
     //    and every owner merges its slice over the cluster from its own memory.
-    float* wo = reinterpret_cast<float*>(smem);             // [warp][lane][kWoStride]
-    float* wm = wo + kConsumers * 32 * kWoStride;           // [warp][16] running max
-    float* wl = wm + kConsumers * kRows;                    // [warp][16] running sum
+    float* wo = reinterpret_cast<float*>(smem);             // [warp][lane][kWoS]
+    float* wm = wo + kCW * 32 * kWoS;                       // [warp][16] running max
+    float* wl = wm + kCW * kRows;                           // [warp][16] running sum
     float* ro = reinterpret_cast<float*>(smem + kStages * kStageBytes + kMetaBytes);
     float* rml = ro + kRecvFloats;                          // [source CTA][16][max, sum]
     __nv_bfloat16* orow = out + ((size_t)row * H_q + (size_t)g * G) * kHD;
     const bool vec_out = (reinterpret_cast<uintptr_t>(out) & 7u) == 0u;
-    if (warp < kConsumers) {
+    if (warp < kCW) {
         l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
         l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
         l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
@@ -410,7 +429,7 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
             wl[warp * kRows + g8] = l_a;
             wl[warp * kRows + g8 + 8] = l_b;
         }
-        float4* dst = reinterpret_cast<float4*>(wo + (warp * 32 + lane) * kWoStride);
+        float4* dst = reinterpret_cast<float4*>(wo + (warp * 32 + lane) * kWoS);
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -420,32 +439,34 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
     __syncthreads();
     const int sp = slice_slots(nsplit), pitch = slice_pitch(sp);
     if (nsplit > 1) cluster_wait();  // every CTA of the cluster has started
-    if (warp < kConsumers) {
+    if (warp < kCW) {
         // heads of this lane's slots: e = 0, 1 -> ha; e = 2, 3 -> hb
+        constexpr int NJ = kSlotsPer / 4;  // float4 groups this thread merges
         const int ha = g8, hb = g8 + 8;
         float Ma = -INFINITY, Mb = -INFINITY;
 #pragma unroll
-        for (int w2 = 0; w2 < kConsumers; ++w2) {
+        for (int w2 = 0; w2 < kCW; ++w2) {
             Ma = fmaxf(Ma, wm[w2 * kRows + ha]);
             Mb = fmaxf(Mb, wm[w2 * kRows + hb]);
         }
         const float ba = Ma == -INFINITY ? 0.f : Ma, bb = Mb == -INFINITY ? 0.f : Mb;
-        float fa[kConsumers], fb[kConsumers], La = 0.f, Lb = 0.f;
+        float fa[kCW], fb[kCW], La = 0.f, Lb = 0.f;
 #pragma unroll
-        for (int w2 = 0; w2 < kConsumers; ++w2) {
+        for (int w2 = 0; w2 < kCW; ++w2) {
             fa[w2] = exp2f(wm[w2 * kRows + ha] - ba);
             fb[w2] = exp2f(wm[w2 * kRows + hb] - bb);
             La += fa[w2] * wl[w2 * kRows + ha];
             Lb += fb[w2] * wl[w2 * kRows + hb];
         }
-        float4 acc[4];
+        float4 acc[NJ];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < NJ; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int w2 = 0; w2 < kConsumers; ++w2) {
-            const float4* src = reinterpret_cast<const float4*>(wo + (w2 * 32 + lane) * kWoStride) + 4 * warp;
+        for (int w2 = 0; w2 < kCW; ++w2) {
+            const float4* src =
+                reinterpret_cast<const float4*>(wo + (w2 * 32 + lane) * kWoS) + NJ * warp;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < NJ; ++j) {
                 const float4 v = src[j];
                 acc[j].x += fa[w2] * v.x;
                 acc[j].y += fa[w2] * v.y;
@@ -454,21 +475,30 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
             }
         }
         if (nsplit == 1) {
-            // slots 16w + 4j + e: h = w >> 1, i = (4w + j) & 7, so group j of
-            // component e lands on dim 64h + 16*q4 + 8*(e&1) + ((4w) & 7) + j
+            // slots kSlotsPer*warp + 4j + e: h = slot >> 5, i = (slot >> 2) & 7,
+            // so group j of component e lands on dim 64h + 16*q4 + 8*(e&1) + i0 + j
             const float ia = La > 0.f ? 1.f / La : 0.f, ib = Lb > 0.f ? 1.f / Lb : 0.f;
-            const int d0 = 64 * (warp >> 1) + 16 * q4 + ((4 * warp) & 7);
+            const int slot0 = kSlotsPer * warp;
+            const int d0 = 64 * (slot0 >> 5) + 16 * q4 + ((slot0 >> 2) & 7);
             if (ha < G) {
-                store_bf16x4(orow + ha * kHD + d0, acc[0].x * ia, acc[1].x * ia, acc[2].x * ia,
-                             acc[3].x * ia, vec_out);
-                store_bf16x4(orow + ha * kHD + d0 + 8, acc[0].y * ia, acc[1].y * ia, acc[2].y * ia,
-                             acc[3].y * ia, vec_out);
+                float vx[NJ], vy[NJ];
+#pragma unroll
+                for (int j = 0; j < NJ; ++j) {
+                    vx[j] = acc[j].x * ia;
+                    vy[j] = acc[j].y * ia;
+                }
+                store_bf16_run<NJ>(orow + ha * kHD + d0, vx, vec_out);
+                store_bf16_run<NJ>(orow + ha * kHD + d0 + 8, vy, vec_out);
             }
             if (hb < G) {
-                store_bf16x4(orow + hb * kHD + d0, acc[0].z * ib, acc[1].z * ib, acc[2].z * ib,
-                             acc[3].z * ib, vec_out);
-                store_bf16x4(orow + hb * kHD + d0 + 8, acc[0].w * ib, acc[1].w * ib, acc[2].w * ib,
-                             acc[3].w * ib, vec_out);
+                float vz[NJ], vw[NJ];
+#pragma unroll
+                for (int j = 0; j < NJ; ++j) {
+                    vz[j] = acc[j].z * ib;
+                    vw[j] = acc[j].w * ib;
+                }
+                store_bf16_run<NJ>(orow + hb * kHD + d0, vz, vec_out);
+                store_bf16_run<NJ>(orow + hb * kHD + d0 + 8, vw, vec_out);
             }
             // log2-sum-exp2 of the scaled logits, for combining partial results
             if (lse != nullptr && warp == 0 && q4 == 0) {
@@ -480,8 +510,8 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
             namespace cg = cooperative_groups;
             cg::cluster_group cluster = cg::this_cluster();
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int slot = 16 * warp + 4 * j;
+            for (int j = 0; j < NJ; ++j) {
+                const int slot = kSlotsPer * warp + 4 * j;
                 const int owner = slot / sp;
                 float* dst = cluster.map_shared_rank(ro, owner) +
                              (size_t)(split * 32 + lane) * pitch + (slot - owner * sp);
@@ -502,7 +532,7 @@ __global__ void __launch_bounds__(dec::kThreads) sparse_attn_decode_kernel(
     // This CTA owns slots [split*sp, split*sp + sp) of every lane.
     const int s0 = split * sp;
     const int ngroups = s0 < kSlots ? (min(kSlots, s0 + sp) - s0) / 4 : 0;
-    for (int e = tid; e < ngroups * 32; e += kThreads) {
+    for (int e = tid; e < ngroups * 32; e += kNT) {
         const int ln = e & 31, gq = e >> 5;
         const int slot = s0 + 4 * gq;
         const int ha = ln >> 2, hb = ha + 8;

@@ -443,7 +443,8 @@ struct DecodeShape {
 
 DecodeShape decode_shape(long long pairs, int units) {
     // When the pairs fill the SMs with clusters of 2-4 CTAs, give each SM one
-    // CTA with a deep ring; otherwise two shallow CTAs per SM and up to 8 splits.
+    // CTA with the deep ring (and two consumer groups); otherwise two shallow
+    // CTAs per SM and up to 8 splits.
     const long long per_sm = 148 / pairs;
     if (per_sm >= 2 && per_sm <= 4 && units >= 2 * per_sm) return {(int)per_sm, true};
     long long want = (2 * 148 + pairs - 1) / pairs;
@@ -452,17 +453,21 @@ DecodeShape decode_shape(long long pairs, int units) {
     return {want < 1 ? 1 : (int)want, false};
 }
 
-template <int ST>
+template <int ST, int GR>
 cudaError_t decode_kernel_attr() {
     static std::once_flag once;
     static cudaError_t err = cudaSuccess;
     std::call_once(once, [] {
-        err = cudaFuncSetAttribute(lci::sparse_attn_decode_kernel<ST>,
+        err = cudaFuncSetAttribute(lci::sparse_attn_decode_kernel<ST, GR>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    lci::dec::smem_bytes(ST));
     });
     return err;
 }
+
+// The deep ring runs one CTA per SM with two consumer groups, the shallow one
+// two CTAs per SM with one group each.
+constexpr int kDeepGroups = 2, kShallowGroups = 1;
 
 lci_status launch_attn_decode(const void* q, int32_t batch, int32_t S, int32_t H_q,
                               const void* k_pool, const void* v_pool, const lci_block_table* t,
@@ -479,12 +484,13 @@ lci_status launch_attn_decode(const void* q, int32_t batch, int32_t S, int32_t H
     const int nsplit = shape.nsplit;
     const int stages = shape.deep ? lci::dec::kStagesDeep : lci::dec::kStagesShallow;
     const cudaError_t attr_err =
-        shape.deep ? decode_kernel_attr<lci::dec::kStagesDeep>() : decode_kernel_attr<lci::dec::kStagesShallow>();
+        shape.deep ? decode_kernel_attr<lci::dec::kStagesDeep, kDeepGroups>()
+                   : decode_kernel_attr<lci::dec::kStagesShallow, kShallowGroups>();
     if (attr_err != cudaSuccess)
         return fail(LCI_ERR_CUDA, "sparse_attn: %s", cudaGetErrorString(attr_err));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)pairs, (unsigned)nsplit, 1);
-    cfg.blockDim = dim3(lci::dec::kThreads, 1, 1);
+    cfg.blockDim = dim3(lci::dec::threads(shape.deep ? kDeepGroups : kShallowGroups), 1, 1);
     cfg.dynamicSmemBytes = lci::dec::smem_bytes(stages);
     cfg.stream = st;
     cudaLaunchAttribute attrs[2];
@@ -504,8 +510,8 @@ lci_status launch_attn_decode(const void* q, int32_t batch, int32_t S, int32_t H
     cfg.attrs = attrs;
     cfg.numAttrs = na;
     const float scale_log2 = scale * 1.4426950408889634f;
-    auto kern = shape.deep ? lci::sparse_attn_decode_kernel<lci::dec::kStagesDeep>
-                           : lci::sparse_attn_decode_kernel<lci::dec::kStagesShallow>;
+    auto kern = shape.deep ? lci::sparse_attn_decode_kernel<lci::dec::kStagesDeep, kDeepGroups>
+                           : lci::sparse_attn_decode_kernel<lci::dec::kStagesShallow, kShallowGroups>;
     cudaError_t e = cudaLaunchKernelEx(
         &cfg, kern, tm_k, tm_v, static_cast<const __nv_bfloat16*>(q),
         t->d_table, t->max_blocks, t->num_pages, t->num_kv_heads, t->block_size, S, H_q, ids, topk,

@@ -353,13 +353,16 @@ def test_decode_attention_deep_ring_uneven_splits(B, H_kv):
 
 
 @pytest.mark.parametrize("B,H_kv,topk", [(300, 1, 3), (150, 1, 4), (100, 1, 4), (40, 1, 4),
-                                         (1, 1, 5), (3, 2, 5), (1, 1, 6), (1, 1, 7), (2, 1, 9)])
+                                         (50, 1, 7), (40, 1, 9), (1, 1, 5), (3, 2, 5), (1, 1, 6),
+                                         (1, 1, 7), (2, 1, 9)])
 def test_decode_attention_every_cluster_size(B, H_kv, topk):
     """Decode shapes that split each (row, KV head) pair over 1 to 8 CTAs of a
     cluster (the split count follows from the pairs and the units per pair):
-    300 pairs run one CTA each, 150 and 100 pairs clusters of 2 and 3, 40 pairs
-    of 4, and single rows with 5, 6, 7 or 9 units clusters of 5 to 8, whose
-    output slices are uneven. H_kv = 2 leaves half of the 16 MMA rows unused."""
+    300 pairs run one CTA each, 150, 100 and 40 pairs two-CTA-per-SM clusters
+    of 2, 3 and 4; 50 and 40 pairs with 7 and 9 units one-CTA-per-SM clusters
+    of 2 and 3 (two consumer groups on alternate tiles, odd unit counts), and
+    single rows with 5, 6, 7 or 9 units clusters of 5 to 8, whose output slices
+    are uneven. H_kv = 2 leaves half of the 16 MMA rows unused."""
     cfg = CONFIGS["decode"].replace(name="splits", B=B, H_kv=H_kv, ctx=1000, q_start=999,
                                     topk=topk, spare_pages=4)
     w = generate(cfg)
