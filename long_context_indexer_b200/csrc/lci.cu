@@ -161,7 +161,10 @@ int index_stream_slots() {
     if (dev < 0 || dev >= 64) return 0;
     if (slots[dev] == 0) {
         int sms = 0, per_sm = 0;
-        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        if (cudaFuncSetAttribute(lci::index_stream_select_kernel<T, kIndexThreads>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 lci::ixs::smem_bytes<kIndexThreads>()) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(
                 &per_sm, lci::index_stream_select_kernel<T, kIndexThreads>, kIndexThreads,
                 lci::ixs::smem_bytes<kIndexThreads>()) != cudaSuccess)
