@@ -541,7 +541,7 @@ def config_entry(cfg, r, pk):
     ti, ta = r["t_index_ms"] * 1e-3, r["t_attn_ms"] * 1e-3
     e = {
         "ms_step": r["t_step_ms"], "ms_index": r["t_index_ms"], "ms_attn": r["t_attn_ms"],
-        "ms_step_one_launch": r["t_persistent_ms"],
+        "ms_step_one_launch": r.get("t_persistent_ms"),
         "tokens_per_s": rows / (r["t_step_ms"] * 1e-3),
         "index_gbs": a["index_bytes"] / ti / 1e9,
         "index_tflops": a["index_flops"] / ti / 1e12,
