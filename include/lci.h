@@ -380,14 +380,18 @@ LCI_API lci_status lci_sparse_decode_workspace_size(int32_t batch, int32_t S, in
  * latency. The indexer publishes each query row as soon as its block ids are
  * final, and the attention kernel, launched behind it (programmatic dependent
  * launch), starts on a row as soon as that row is published, while later rows
- * are still being scored.
+ * are still being scored. For 2 KiB block keys (H_i*d_c*element size = 2048)
+ * a row is published as its picks, (block id, page) pairs in the workspace
+ * that the attention's producer polls one by one and turns straight into tile
+ * loads; for other key sizes as a flag per row.
  * Arguments are those of the two calls; k_c's nb_max must equal the table's
  * max_blocks and all floating inputs share one dtype. The workspace holds the
- * scratch, per-row publication flags and the per-call counters: zero-fill it
+ * scratch, the per-row publications and the per-call counters: zero-fill it
  * before its first call and again before using it with other sizes or after a
  * call that failed on the device; every successful call leaves it ready for
- * the next. A flag left set by an earlier call is never taken for a new
- * publication. Calls sharing a workspace must not overlap in time.
+ * the next. A publication left by an earlier call is never taken for a new
+ * one (the indexer resets it before the attention kernel can start). Calls
+ * sharing a workspace must not overlap in time.
  */
 LCI_API lci_status lci_sparse_decode(const void* q_c, const void* k_c, lci_dtype dtype,
                                      int32_t batch, int32_t S, int32_t H_i, int32_t d_c,
