@@ -599,10 +599,36 @@ class SparseDecodeStep:
             _dev(self.out, "out", q_c.dtype, 4), _dev(self.ws, "workspace"),
             ctypes.c_size_t(self.ws.numel() * self.ws.element_size()), self._stream)
 
-    def __call__(self) -> None:
-        rc = self._fn(*self._args)
+    def __call__(self, stream=None) -> None:
+        """Launch the step on its stream, or on `stream` if given (e.g. the
+        stream a CUDA graph is being captured on)."""
+        args = self._args if stream is None else self._args[:-1] + (_stream(stream),)
+        rc = self._fn(*args)
         if rc != LCI_OK:
             _check(rc, self._name)
+
+    def capture(self, h2d=(), d2h=()) -> "torch.cuda.CUDAGraph":
+        """The step with its transfers as one CUDA graph, for a serving loop
+        that replays it every step: the copies ``dst.copy_(src)`` of ``h2d``
+        (device tensors filled from pinned host tensors), this step, then the
+        copies of ``d2h`` (pinned host tensors filled from device tensors). The
+        graph reads and writes the same buffers on every replay; the caller
+        refills the host inputs and reads the host outputs between replays
+        (after synchronising). Call the step once before capturing it."""
+        for dst, src in list(h2d) + list(d2h):
+            host = dst if dst.device.type == "cpu" else src
+            if not host.is_pinned():
+                raise ValueError("lci: graph transfers need pinned host tensors")
+        g = torch.cuda.CUDAGraph()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g):
+            for dst, src in h2d:
+                dst.copy_(src, non_blocking=True)
+            self(torch.cuda.current_stream())  # the capturing stream
+            for dst, src in d2h:
+                dst.copy_(src, non_blocking=True)
+        torch.cuda.synchronize()
+        return g
 
 
 def get_device_status(stream=None) -> None:

@@ -424,6 +424,38 @@ def test_prepared_decode_step_matches_the_plain_call():
         assert torch.equal(step.out, out)
 
 
+def test_prepared_decode_step_graph_with_transfers():
+    """SparseDecodeStep.capture: host-to-device copies of the inputs, the step
+    and device-to-host copies of ids and out, replayed as one CUDA graph; each
+    replay sees the host inputs' current contents and matches the plain call."""
+    cfg = CONFIGS["decode"].replace(B=8, ctx=8192, q_start=8191, spare_pages=8)
+    w = generate(cfg)
+    d = upload(w)
+    bt = lci.create_block_table(d["block_table"], d["k_pool"])
+    h_qc = w["q_c"].clone().pin_memory()
+    h_q = w["q"].clone().pin_memory()
+    step = lci.SparseDecodeStep(d["q_c"], d["k_c"], d["ctx_len"], d["q_start"], cfg.topk, d["q"],
+                                d["k_pool"], d["v_pool"], bt)
+    h_ids = torch.empty(step.ids.shape, dtype=step.ids.dtype).pin_memory()
+    h_out = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    step()
+    g = step.capture(h2d=[(d["q_c"], h_qc), (d["q"], h_q)], d2h=[(h_ids, step.ids), (h_out, step.out)])
+    for flip in (False, True):
+        if flip:
+            h_qc.copy_(torch.flip(w["q_c"], dims=[0]))
+            h_q.copy_(torch.flip(w["q"], dims=[0]))
+        g.replay()
+        torch.cuda.synchronize()
+        ids, out = lci.sparse_decode(h_qc.cuda(), d["k_c"], d["ctx_len"], d["q_start"], cfg.topk,
+                                     h_q.cuda(), d["k_pool"], d["v_pool"], bt)
+        torch.cuda.synchronize()
+        lci.get_device_status()
+        assert torch.equal(h_ids, ids.cpu())
+        assert torch.equal(h_out, out.cpu())
+    with pytest.raises(ValueError):
+        step.capture(h2d=[(d["q_c"], w["q_c"])])  # pageable host memory
+
+
 def test_both_decode_forms_share_one_workspace():
     """The two-kernel and the one-launch decode forms alternate on one
     workspace: neither takes the other's publication flags for its own."""
