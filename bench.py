@@ -101,9 +101,9 @@ def peaks():
 # sources the capture ran. Once those sources change the figure no longer
 # describes the kernel and the bench reports traffic as null.
 PROFILED_TRAFFIC = {
-    ("decode", "index_select"): (33683200, "29249c0d5d426974"),
-    ("decode", "sparse_attn"): (33798400, "29249c0d5d426974"),
-    ("1m_chunk", "index_select"): (25226496, "29249c0d5d426974"),
+    ("decode", "index_select"): (33751808, "4867c66070ea45ff"),
+    ("decode", "sparse_attn"): (33830656, "4867c66070ea45ff"),
+    ("1m_chunk", "index_select"): (25250816, "4867c66070ea45ff"),
 }
 
 
