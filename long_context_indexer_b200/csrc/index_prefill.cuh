@@ -170,7 +170,6 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
     int32_t* __restrict__ part_id, unsigned int* __restrict__ counters,
     unsigned int* __restrict__ row_bound, int32_t* __restrict__ ids) {
     using namespace pre;
-    constexpr int kThreads = Cfg<KT>::kThreads;
     constexpr int kParts = Epi<KT>::kParts;        // epilogue warps per TMEM lane quarter
     constexpr int kEW = 4 * kParts;                // epilogue warps
     constexpr int kGroup = 32;                    // TMEM columns per load
@@ -183,7 +182,8 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
     uint64_t* empty_bar = full_bar + kStages;
     uint64_t* tfull_bar = empty_bar + kStages;
     uint64_t* tempty_bar = tfull_bar + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + 2);
+    uint64_t* merge_bar = tempty_bar + 2;    // the split lists' bulk copies
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(merge_bar + 1);
     int* s_last = reinterpret_cast<int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -209,6 +209,7 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
             mbar_init(&tfull_bar[i], 1);
             mbar_init(&tempty_bar[i], kEW);  // one arrive per epilogue warp
         }
+        mbar_init(merge_bar, 1);
         fence_mbar_init();
     }
     if (warp == 1) {  // the whole warp allocates the two accumulators
@@ -417,29 +418,32 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
     if (n_split == 1) return;
 
     // ---------------- merge the split candidates (last CTA of the m-tile) ----------------
-    __threadfence();
-    __syncthreads();
+    __syncthreads();  // this CTA's lists are written
     if (tid == 0) {
+        // the arrival releases them; the m-tile's last arrival acquires the others'
         unsigned int* ctr = counters + (size_t)b * m_tiles + mt;
-        const unsigned prev = atomicAdd(ctr, 1u);
+        const unsigned prev = atom_add_acq_rel_gpu(ctr, 1u);
         *s_last = prev == (unsigned)(n_split - 1);
         if (*s_last) *ctr = 0u;  // ready for the next call
     }
     __syncthreads();
     if (!*s_last) return;
-    __threadfence();
-    // Copy the m-tile's candidate lists [128 rows][n_split][topk] into the
-    // (idle) stage memory with coalesced loads, then merge per row.
+    // Copy the m-tile's candidate lists [128 rows][n_split][topk] (keys, then
+    // ids: two contiguous ranges) into the idle stage memory with two bulk
+    // copies, then merge per row.
     const int per_row = n_split * topk;
     const size_t base = ((size_t)b * m_tiles + mt) * kBM * per_row;
     uint32_t* mk = reinterpret_cast<uint32_t*>(smem);
     int32_t* mi = reinterpret_cast<int32_t*>(smem) + kBM * per_row;
-#pragma unroll 4
-    for (int e = tid; e < kBM * per_row; e += kThreads) {
-        mk[e] = __ldcg(part_key + base + e);
-        mi[e] = __ldcg(part_id + base + e);
+    if (tid == 0) {
+        const uint32_t bytes = (uint32_t)(kBM * per_row * 4);
+        fence_proxy_async_global();  // the acquired lists, then the copies that read them
+        fence_proxy_async_smem();    // this CTA's earlier reads of the stage memory, then the copies
+        mbar_arrive_expect_tx(merge_bar, 2u * bytes);
+        bulk_load(mk, part_key + base, bytes, merge_bar);
+        bulk_load(mi, part_id + base, bytes, merge_bar);
     }
-    __syncthreads();
+    if (!mbar_wait(merge_bar, 0)) return;  // time-out: status raised, ids left unwritten
     if (warp < 2 || warp >= 6) return;  // one thread per row merges
     const int r = (warp & 3) * 32 + lane;
     const int s = row0 + r;
