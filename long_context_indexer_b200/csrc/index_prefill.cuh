@@ -296,13 +296,15 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
         uint32_t gk = 0u;
         float gthr = -INFINITY;
         auto flush = [&]() {
+            // Branch-free: a lane past its own candidates inserts key 0, and a
+            // key at or below the list's last entry changes nothing either
+            // (the network moves an entry only for a strictly larger key).
             const int m = __reduce_max_sync(0xffffffffu, nc);
+            uint2 e = cbuf[0];
             for (int q = 0; q < m; ++q) {
-                if (q < nc) {
-                    const uint2 e = cbuf[q * kEpiThreads];
-                    const uint32_t k = score_key(__uint_as_float(e.x));
-                    if (k > top.threshold()) top.insert(k, (int32_t)e.y);
-                }
+                const uint2 next = cbuf[min(q + 1, kBuf - 1) * kEpiThreads];  // loaded ahead
+                top.insert(q < nc ? score_key(__uint_as_float(e.x)) : 0u, (int32_t)e.y);
+                e = next;
             }
             nc = 0;
             if (top.full() && top.threshold() > gk && bound != nullptr) {
