@@ -309,7 +309,7 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
             nc = 0;
             if (top.full() && top.threshold() > gk && bound != nullptr) {
                 gk = top.threshold();
-                gthr = float_below(key_score(gk));
+                gthr = fmaxf(gthr, float_below(key_score(gk)));
                 atomicMax(bound, gk);
             }
         };
@@ -321,6 +321,33 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
             if (ok) {
                 const uint32_t lane_base =
                     tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kBN);
+                if (t == 0 && __all_sync(0xffffffffu, n0 + kBN <= vis)) {
+                    // First tile, empty list, every column visible to the warp's
+                    // rows: a lower bound of this part's KT-th
+                    // best score from the tile itself. Its columns fall into KT
+                    // runs of kSub; every run's maximum is a score of the part, so
+                    // with L the smallest run maximum, KT scores are >= L and a
+                    // score below L never enters the list.
+                    constexpr int kSub = kBN / kParts / KT;
+                    static_assert(kSub >= 1 && kGroup % kSub == 0, "runs tile a group");
+                    float lmin = INFINITY;
+#pragma unroll 1
+                    for (int c = 0; c < kGroupsPerPart; ++c) {
+                        const int col = (c * kParts + part) * kGroup;
+                        uint32_t raw[kGroup];
+                        __syncwarp();
+                        tmem_ld32(lane_base + (uint32_t)col, raw);
+#pragma unroll
+                        for (int g0 = 0; g0 < kGroup; g0 += kSub) {
+                            float mrun = -INFINITY;
+#pragma unroll
+                            for (int i = 0; i < kSub; ++i)
+                                if (n0 + col + g0 + i < vis) mrun = fmaxf(mrun, __uint_as_float(raw[g0 + i]));
+                            lmin = fminf(lmin, mrun);
+                        }
+                    }
+                    if (lmin > -INFINITY && lmin < INFINITY) gthr = fmaxf(gthr, float_below(lmin));
+                }
 #pragma unroll 1
                 for (int c = 0; c < kGroupsPerPart; ++c) {
                     const int col = (c * kParts + part) * kGroup;  // parts interleave groups
@@ -354,7 +381,7 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
                     }
                     if (gk_next > gk) {
                         gk = gk_next;
-                        gthr = float_below(key_score(gk));
+                        gthr = fmaxf(gthr, float_below(key_score(gk)));
                     }
                 }
                 __syncwarp();
