@@ -408,7 +408,9 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
             int head[kParts];
 #pragma unroll
             for (int q = 0; q < kParts; ++q) head[q] = 0;
-            const size_t prow = (((size_t)b * m_tiles + mt) * kBM + r) * n_split + ns;
+            // split lists of the m-tile: [split][rank][row], rows fastest (the
+            // stores of a warp are contiguous, and so are the merge's reads)
+            const size_t pbase = (((size_t)b * m_tiles + mt) * n_split + ns) * topk * kBM + r;
             int32_t* orow = ids + ((size_t)b * S + s) * topk;
             for (int i = 0; i < topk; ++i) {
                 // the best head: key desc, then id asc; empty entries (id -1) last
@@ -430,8 +432,8 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
                 if (n_split == 1) {
                     if (s < S) orow[i] = bi;
                 } else {
-                    part_key[prow * topk + i] = bk;
-                    part_id[prow * topk + i] = bi;
+                    part_key[pbase + (size_t)i * kBM] = bk;
+                    part_id[pbase + (size_t)i * kBM] = bi;
                 }
             }
         }
@@ -457,7 +459,7 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
     }
     __syncthreads();
     if (!*s_last) return;
-    // Copy the m-tile's candidate lists [128 rows][n_split][topk] (keys, then
+    // Copy the m-tile's candidate lists [n_split][topk][128 rows] (keys, then
     // ids: two contiguous ranges) into the idle stage memory with two bulk
     // copies, then merge per row.
     const int per_row = n_split * topk;
@@ -477,8 +479,8 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
     const int r = (warp & 3) * 32 + lane;
     const int s = row0 + r;
     if (s >= S) return;
-    const uint32_t* rk = mk + r * per_row;
-    const int32_t* ri = mi + r * per_row;
+    const uint32_t* rk = mk + r;  // entry (split q, rank h) at [(q * topk + h) * kBM]
+    const int32_t* ri = mi + r;
     // k-way merge of the n_split sorted lists: (key desc, id asc)
     int head[8];
 #pragma unroll
@@ -492,8 +494,8 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
             if (q >= n_split || head[q] >= topk) continue;
-            const uint32_t kq = rk[q * topk + head[q]];
-            const int32_t iq = ri[q * topk + head[q]];
+            const uint32_t kq = rk[(q * topk + head[q]) * kBM];
+            const int32_t iq = ri[(q * topk + head[q]) * kBM];
             if (iq < 0) continue;  // sentinel: that list is exhausted
             if (best < 0 || kq > bk || (kq == bk && iq < bi)) {
                 best = q;
