@@ -47,6 +47,7 @@ constexpr int kBBytes = kBN * kBK * 2;   // 32 KiB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kTmemCols = 2 * kBN;       // two accumulators
 constexpr int kCandBytes = 32 * 1024;            // per-thread candidate buffers (score, id)
+static_assert(64 * kBM * 4 <= kCandBytes, "the staged output rows (topk <= 64) fit the candidate area");
 constexpr int kSmemBytes = kStages * kStageBytes + kCandBytes + 1024 /*align*/ + 256 /*barriers*/;
 // Epilogue warps: kParts per TMEM lane quarter, each taking every kParts-th
 // 32-column group of every tile with its own list. More parts hide more
@@ -162,6 +163,66 @@ __device__ __forceinline__ float float_below(float x) {
     return __uint_as_float(x > 0.f ? u - 1u : u + 1u);
 }
 
+// Best of N composites c[base .. base+N) by a tournament (depth log2 N):
+// the winner's value and index.
+template <int N> struct Tournament {
+    static __device__ __forceinline__ void run(const uint64_t* c, int base, uint64_t& best,
+                                               int& at) {
+        uint64_t c1;
+        int a1;
+        Tournament<N / 2>::run(c, base, best, at);
+        Tournament<N - N / 2>::run(c, base + N / 2, c1, a1);
+        const bool t = c1 > best;
+        best = t ? c1 : best;
+        at = t ? a1 : at;
+    }
+};
+template <> struct Tournament<1> {
+    static __device__ __forceinline__ void run(const uint64_t* c, int base, uint64_t& best,
+                                               int& at) {
+        best = c[base];
+        at = base;
+    }
+};
+
+// k-way merge of one row's NS sorted split lists into its top `topk`. The
+// lists sit in shared memory at (shared-window) addresses keys / ids, entry
+// (list q, rank h) at byte offset ((q * topk + h) * pre::kBM) * 4; output rank
+// i is stored at out + 4 * out_slot(i). An entry's composite (key << 32 | ~id)
+// orders key desc then id asc, and an empty entry (key 0, id -1) composes to
+// 0, below every real one. Each list's head entry is held in a register, so a
+// step is one tournament and one refill of the winner's list.
+template <int NS, typename Slot>
+__device__ __forceinline__ void merge_split_lists(uint32_t keys, uint32_t ids, uint32_t out,
+                                                  int topk, Slot out_slot) {
+    uint64_t cur[NS];
+    int head[NS];
+#pragma unroll
+    for (int q = 0; q < NS; ++q) {
+        head[q] = 0;
+        const uint32_t off = (uint32_t)(q * topk * pre::kBM * 4);
+        cur[q] = ((uint64_t)lds32(keys + off) << 32) | (uint32_t)~lds32(ids + off);
+    }
+    for (int i = 0; i < topk; ++i) {
+        uint64_t bc;
+        int best;
+        Tournament<NS>::run(cur, 0, bc, best);
+        sts32(out + 4u * (uint32_t)out_slot(i), bc == 0 ? 0xffffffffu : ~(uint32_t)bc);
+        int h = 0;
+#pragma unroll
+        for (int q = 0; q < NS; ++q) h = q == best ? head[q] : h;
+        ++h;  // the winner's next entry (an exhausted list stays at composite 0)
+        const uint32_t off = (uint32_t)((best * topk + min(h, topk - 1)) * pre::kBM * 4);
+        const uint64_t next =
+            h < topk ? ((uint64_t)lds32(keys + off) << 32) | (uint32_t)~lds32(ids + off) : 0ull;
+#pragma unroll
+        for (int q = 0; q < NS; ++q) {
+            head[q] = q == best ? h : head[q];
+            cur[q] = q == best ? next : cur[q];
+        }
+    }
+}
+
 template <int KT>
 __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, int S,
@@ -227,6 +288,31 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+
+    // The m-tile's output rows are staged in the candidate area once the
+    // epilogue is done with it, entry (rank i, row r) at out_slot(i, r): the
+    // row index XOR the rank keeps both the per-row writes (32 rows, one
+    // rank) and the row-major copy-out (one row, consecutive ranks) free of
+    // bank conflicts. The copy-out then writes the tile's contiguous
+    // rows x topk ids with coalesced stores.
+    int32_t* out_s = reinterpret_cast<int32_t*>(cand);
+    auto out_slot = [&](int i, int r) { return i * kBM + (r ^ (i & 31)); };
+    auto store_rows = [&](int t0, int nt) {
+        const int n = min(kBM, S - row0) * topk;
+        int32_t* dst = ids + ((size_t)b * S + row0) * topk;
+        // entry j is (row j / topk, rank j % topk), stepped without a division
+        const int drow = nt / topk, drank = nt - drow * topk;
+        int rr = t0 / topk, i = t0 - rr * topk;
+        for (int j = t0; j < n; j += nt) {
+            dst[j] = out_s[out_slot(i, rr)];
+            rr += drow;
+            i += drank;
+            if (i >= topk) {
+                i -= topk;
+                ++rr;
+            }
+        }
+    };
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -411,7 +497,6 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
             // split lists of the m-tile: [split][rank][row], rows fastest (the
             // stores of a warp are contiguous, and so are the merge's reads)
             const size_t pbase = (((size_t)b * m_tiles + mt) * n_split + ns) * topk * kBM + r;
-            int32_t* orow = ids + ((size_t)b * S + s) * topk;
             for (int i = 0; i < topk; ++i) {
                 // the best head: key desc, then id asc; empty entries (id -1) last
                 int best = 0;
@@ -430,12 +515,16 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
 #pragma unroll
                 for (int q = 0; q < kParts; ++q) head[q] += (q == best && bi >= 0);
                 if (n_split == 1) {
-                    if (s < S) orow[i] = bi;
+                    out_s[out_slot(i, r)] = bi;
                 } else {
                     part_key[pbase + (size_t)i * kBM] = bk;
                     part_id[pbase + (size_t)i * kBM] = bi;
                 }
             }
+        }
+        if (n_split == 1) {
+            named_barrier_sync(1, 32 * kEW);
+            store_rows(et, 32 * kEW);
         }
     }
     tc_fence_before();
@@ -474,39 +563,27 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
         bulk_load(mk, part_key + base, bytes, merge_bar);
         bulk_load(mi, part_id + base, bytes, merge_bar);
     }
-    if (!mbar_wait(merge_bar, 0)) return;  // time-out: status raised, ids left unwritten
-    if (warp < 2 || warp >= 6) return;  // one thread per row merges
+    // (the barrier makes a time-out, which raises the status, a decision of
+    // the whole CTA: the rows' ids are then left unwritten)
+    if (!__syncthreads_and(mbar_wait(merge_bar, 0))) return;
     const int r = (warp & 3) * 32 + lane;
     const int s = row0 + r;
-    if (s >= S) return;
-    const uint32_t* rk = mk + r;  // entry (split q, rank h) at [(q * topk + h) * kBM]
-    const int32_t* ri = mi + r;
-    // k-way merge of the n_split sorted lists: (key desc, id asc)
-    int head[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) head[q] = 0;
-    row_bound[(size_t)b * S + s] = 0u;  // every CTA of the m-tile has finished with it
-    int32_t* orow = ids + ((size_t)b * S + s) * topk;
-    for (int i = 0; i < topk; ++i) {
-        int best = -1;
-        uint32_t bk = 0;
-        int32_t bi = 0;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            if (q >= n_split || head[q] >= topk) continue;
-            const uint32_t kq = rk[(q * topk + head[q]) * kBM];
-            const int32_t iq = ri[(q * topk + head[q]) * kBM];
-            if (iq < 0) continue;  // sentinel: that list is exhausted
-            if (best < 0 || kq > bk || (kq == bk && iq < bi)) {
-                best = q;
-                bk = kq;
-                bi = iq;
-            }
+    if (warp >= 2 && warp < 6 && s < S) {  // one thread per row merges
+        row_bound[(size_t)b * S + s] = 0u;  // every CTA of the m-tile has finished with it
+        const uint32_t kk = smem_u32(mk + r), ki = smem_u32(mi + r), ko = smem_u32(out_s);
+        auto slot = [&](int i) { return out_slot(i, r); };
+        switch (n_split) {
+            case 2: merge_split_lists<2>(kk, ki, ko, topk, slot); break;
+            case 3: merge_split_lists<3>(kk, ki, ko, topk, slot); break;
+            case 4: merge_split_lists<4>(kk, ki, ko, topk, slot); break;
+            case 5: merge_split_lists<5>(kk, ki, ko, topk, slot); break;
+            case 6: merge_split_lists<6>(kk, ki, ko, topk, slot); break;
+            case 7: merge_split_lists<7>(kk, ki, ko, topk, slot); break;
+            default: merge_split_lists<8>(kk, ki, ko, topk, slot); break;
         }
-        orow[i] = best < 0 ? -1 : bi;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) head[q] += (q == best);
     }
+    __syncthreads();
+    store_rows(tid, Cfg<KT>::kThreads);
 }
 
 }  // namespace lci
