@@ -185,36 +185,39 @@ template <> struct Tournament<1> {
     }
 };
 
-// k-way merge of one row's NS sorted split lists into its top `topk`. The
-// lists sit in shared memory at (shared-window) addresses keys / ids, entry
-// (list q, rank h) at byte offset ((q * topk + h) * pre::kBM) * 4; output rank
-// i is stored at out + 4 * out_slot(i). An entry's composite (key << 32 | ~id)
-// orders key desc then id asc, and an empty entry (key 0, id -1) composes to
-// 0, below every real one. Each list's head entry is held in a register, so a
-// step is one tournament and one refill of the winner's list.
-template <int NS, typename Slot>
-__device__ __forceinline__ void merge_split_lists(uint32_t keys, uint32_t ids, uint32_t out,
-                                                  int topk, Slot out_slot) {
+// k-way merge of one row's NS sorted lists into its best `nout` entries. The
+// lists sit in shared memory from (shared-window) addresses keys / ids: entry
+// (list q, rank h) at byte offset q * list_bytes + h * pre::kBM * 4, each list
+// `len` long. An entry's composite (key << 32 | ~id) orders key desc then id
+// asc, and an empty entry (key 0, id -1) composes to 0, below every real one;
+// emit(i, composite) receives output rank i (an empty one as 0). Each list's
+// head entry is held in a register, so a step is one tournament and one
+// refill of the winner's list.
+template <int NS, typename Emit>
+__device__ __forceinline__ void merge_sorted_lists(uint32_t keys, uint32_t ids,
+                                                   uint32_t list_bytes, int len, int nout,
+                                                   Emit emit) {
+    constexpr uint32_t kRank = pre::kBM * 4;
     uint64_t cur[NS];
     int head[NS];
 #pragma unroll
     for (int q = 0; q < NS; ++q) {
         head[q] = 0;
-        const uint32_t off = (uint32_t)(q * topk * pre::kBM * 4);
+        const uint32_t off = (uint32_t)q * list_bytes;
         cur[q] = ((uint64_t)lds32(keys + off) << 32) | (uint32_t)~lds32(ids + off);
     }
-    for (int i = 0; i < topk; ++i) {
+    for (int i = 0; i < nout; ++i) {
         uint64_t bc;
         int best;
         Tournament<NS>::run(cur, 0, bc, best);
-        sts32(out + 4u * (uint32_t)out_slot(i), bc == 0 ? 0xffffffffu : ~(uint32_t)bc);
+        emit(i, bc);
         int h = 0;
 #pragma unroll
         for (int q = 0; q < NS; ++q) h = q == best ? head[q] : h;
         ++h;  // the winner's next entry (an exhausted list stays at composite 0)
-        const uint32_t off = (uint32_t)((best * topk + min(h, topk - 1)) * pre::kBM * 4);
+        const uint32_t off = (uint32_t)best * list_bytes + (uint32_t)min(h, len - 1) * kRank;
         const uint64_t next =
-            h < topk ? ((uint64_t)lds32(keys + off) << 32) | (uint32_t)~lds32(ids + off) : 0ull;
+            h < len ? ((uint64_t)lds32(keys + off) << 32) | (uint32_t)~lds32(ids + off) : 0ull;
 #pragma unroll
         for (int q = 0; q < NS; ++q) {
             head[q] = q == best ? h : head[q];
@@ -491,36 +494,20 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
         // is reset here, otherwise by the CTA that merges the splits
         if (n_split == 1 && part == 0 && bound != nullptr) *bound = 0u;
         if (part == 0) {
-            int head[kParts];
-#pragma unroll
-            for (int q = 0; q < kParts; ++q) head[q] = 0;
             // split lists of the m-tile: [split][rank][row], rows fastest (the
             // stores of a warp are contiguous, and so are the merge's reads)
             const size_t pbase = (((size_t)b * m_tiles + mt) * n_split + ns) * topk * kBM + r;
-            for (int i = 0; i < topk; ++i) {
-                // the best head: key desc, then id asc; empty entries (id -1) last
-                int best = 0;
-                uint32_t bk = 0u;
-                int32_t bi = -1;
-#pragma unroll
-                for (int q = 0; q < kParts; ++q) {
-                    const int h = min(head[q], KT - 1);
-                    const uint32_t kq = head[q] < KT ? xk[(q * KT + h) * kBM + r] : 0u;
-                    const int32_t iq = head[q] < KT ? xi[(q * KT + h) * kBM + r] : -1;
-                    const bool better = iq >= 0 && (bi < 0 || kq > bk || (kq == bk && iq < bi));
-                    best = better ? q : best;
-                    bk = better ? kq : bk;
-                    bi = better ? iq : bi;
-                }
-#pragma unroll
-                for (int q = 0; q < kParts; ++q) head[q] += (q == best && bi >= 0);
+            const uint32_t ko = smem_u32(out_s);
+            auto emit = [&](int i, uint64_t c) {
                 if (n_split == 1) {
-                    out_s[out_slot(i, r)] = bi;
+                    sts32(ko + 4u * (uint32_t)out_slot(i, r), ~(uint32_t)c);
                 } else {
-                    part_key[pbase + (size_t)i * kBM] = bk;
-                    part_id[pbase + (size_t)i * kBM] = bi;
+                    part_key[pbase + (size_t)i * kBM] = (uint32_t)(c >> 32);
+                    part_id[pbase + (size_t)i * kBM] = (int32_t)~(uint32_t)c;
                 }
-            }
+            };
+            merge_sorted_lists<kParts>(smem_u32(xk + r), smem_u32(xi + r),
+                                       (uint32_t)(KT * kBM * 4), KT, topk, emit);
         }
         if (n_split == 1) {
             named_barrier_sync(1, 32 * kEW);
@@ -571,15 +558,18 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
     if (warp >= 2 && warp < 6 && s < S) {  // one thread per row merges
         row_bound[(size_t)b * S + s] = 0u;  // every CTA of the m-tile has finished with it
         const uint32_t kk = smem_u32(mk + r), ki = smem_u32(mi + r), ko = smem_u32(out_s);
-        auto slot = [&](int i) { return out_slot(i, r); };
+        const uint32_t lb = (uint32_t)(topk * kBM * 4);
+        auto emit = [&](int i, uint64_t c) {
+            sts32(ko + 4u * (uint32_t)out_slot(i, r), ~(uint32_t)c);  // id, -1 when empty
+        };
         switch (n_split) {
-            case 2: merge_split_lists<2>(kk, ki, ko, topk, slot); break;
-            case 3: merge_split_lists<3>(kk, ki, ko, topk, slot); break;
-            case 4: merge_split_lists<4>(kk, ki, ko, topk, slot); break;
-            case 5: merge_split_lists<5>(kk, ki, ko, topk, slot); break;
-            case 6: merge_split_lists<6>(kk, ki, ko, topk, slot); break;
-            case 7: merge_split_lists<7>(kk, ki, ko, topk, slot); break;
-            default: merge_split_lists<8>(kk, ki, ko, topk, slot); break;
+            case 2: merge_sorted_lists<2>(kk, ki, lb, topk, topk, emit); break;
+            case 3: merge_sorted_lists<3>(kk, ki, lb, topk, topk, emit); break;
+            case 4: merge_sorted_lists<4>(kk, ki, lb, topk, topk, emit); break;
+            case 5: merge_sorted_lists<5>(kk, ki, lb, topk, topk, emit); break;
+            case 6: merge_sorted_lists<6>(kk, ki, lb, topk, topk, emit); break;
+            case 7: merge_sorted_lists<7>(kk, ki, lb, topk, topk, emit); break;
+            default: merge_sorted_lists<8>(kk, ki, lb, topk, topk, emit); break;
         }
     }
     __syncthreads();
