@@ -429,21 +429,37 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
         int* xok = reinterpret_cast<int*>(xchg + 3 * 2 * 128);      // [2][2][128]
         float m_ref = -INFINITY;  // reference maximum (log2 units), the same in both halves
         float l = 0.f;            // this half's share of the row sum
-        for (int i = 0; i < nstages; ++i) {
-            // this half's unit: its first token, whether the row takes it, and
-            // how many of its 64 tokens the row may see
-            const int u = 2 * i + hf;
-            int t0 = 0, nval = 0;
-            if (u < nunits) {
-                const int blk = u / upb, sub = u - blk * upb;
-                if (upage[blk] >= 0) {
-                    t0 = ublk[blk] * bs + sub * 64;
-                    if ((umask[blk] & qbit) != 0u && (long long)t0 <= last) {
-                        const long long nv = last - t0 + 1;
-                        nval = nv < 64 ? (int)nv : 64;
+        // The stage's two 64-token units (c = 0, 1), read from the union one
+        // stage ahead so that their shared-memory latency hides behind the
+        // previous stage: each unit's first token (-1: past the union or an
+        // absent page; tokens fit 31 bits, nb_max * bs < 2^31) and how many of
+        // this half's unit's tokens the row takes. (nb, nsub) walk the units in
+        // order without a division by the units per block.
+        int nb = 0, nsub = 0;
+        auto load_units = [&](int i, int& t0a, int& t0b, int& nv) {
+            nv = 0;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                int t = -1;
+                if (2 * i + c < nunits && upage[nb] >= 0) {
+                    t = ublk[nb] * bs + nsub * 64;
+                    if (c == hf && (umask[nb] & qbit) != 0u && (long long)t <= last) {
+                        const long long n = last - t + 1;
+                        nv = n < 64 ? (int)n : 64;
                     }
                 }
+                if (c == 0) t0a = t; else t0b = t;
+                if (++nsub == upb) {
+                    nsub = 0;
+                    ++nb;
+                }
             }
+        };
+        int nt0a = -1, nt0b = -1, nnv = 0;
+        if (nstages > 0) load_units(0, nt0a, nt0b, nnv);
+        for (int i = 0; i < nstages; ++i) {
+            const int ut0a = nt0a, ut0b = nt0b, nval = nnv;
+            if (i + 1 < nstages) load_units(i + 1, nt0a, nt0b, nnv);
             const bool waited = mbar_wait(&sfull[i & 1], (i >> 1) & 1);
             const int my_ok = waited && !*s_abort;
             tc_fence_after();
@@ -528,29 +544,13 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
             // V rows of an absent unit and of tokens past the context length
             // must be zero before the P V MMA reads them (this thread: token row
             // r of the stage, dims 64*hf .. 64*hf+63)
-            bool v_absent[2];
-            long long v_t0[2];
-            bool stage_tail = false;  // the same for every thread
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                const int uv = 2 * i + c;
-                v_absent[c] = true;
-                v_t0[c] = 0;
-                if (uv < nunits) {
-                    const int blk = uv / upb, sub = uv - blk * upb;
-                    if (upage[blk] >= 0) {
-                        v_absent[c] = false;
-                        v_t0[c] = (long long)ublk[blk] * bs + sub * 64;
-                    }
-                }
-                stage_tail = stage_tail || v_absent[c] || v_t0[c] + 64 > ctx;
-            }
+            const bool stage_tail =  // the same for every thread
+                ut0a < 0 || ut0b < 0 || ut0a + 64LL > ctx || ut0b + 64LL > ctx;
             if (stage_tail) {
                 const int vs = i % kVStages;
                 if (!mbar_wait(&vfull[vs], (i / kVStages) & 1)) *s_abort = 1;
-                const bool mine_absent = (r >> 6) ? v_absent[1] : v_absent[0];
-                const long long mine_t0 = (r >> 6) ? v_t0[1] : v_t0[0];
-                if (mine_absent || mine_t0 + (r & 63) >= ctx) {
+                const int mine_t0 = (r >> 6) ? ut0b : ut0a;
+                if (mine_t0 < 0 || (long long)mine_t0 + (r & 63) >= ctx) {
                     unsigned char* vt = smem + kOffV + vs * kTileBytes;
 #pragma unroll
                     for (int cc = 8 * hf; cc < 8 * hf + 8; ++cc)

@@ -526,12 +526,13 @@ lci_status launch_attn_decode(const void* q, int32_t batch, int32_t S, int32_t H
 // The tensor-core prefill schedule (attn_prefill.cuh): the decode kernel's
 // shape limits, 4, 8 or 16 query heads per KV head (32, 16 or 8 queries per
 // 128-row tile), at most 16384 blocks per sequence and 1024 selected blocks per
-// tile.
+// tile, token positions below 2^31.
 bool prefill_attn_fits(const lci_block_table* t, int32_t H_q, int32_t topk, const void* k_pool,
                        const void* v_pool) {
     if (!decode_kernel_fits(t, H_q, k_pool, v_pool)) return false;
     const int G = H_q / t->num_kv_heads;
     return (G == 4 || G == 8 || G == 16) && t->max_blocks <= 32 * lci::pfa::kMaxWords &&
+           (long long)t->max_blocks * t->block_size < (1LL << 31) &&
            (long long)(lci::pfa::kRows / G) * topk <= lci::pfa::kMaxUnion;
 }
 
