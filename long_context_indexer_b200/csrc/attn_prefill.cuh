@@ -429,37 +429,46 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
         int* xok = reinterpret_cast<int*>(xchg + 3 * 2 * 128);      // [2][2][128]
         float m_ref = -INFINITY;  // reference maximum (log2 units), the same in both halves
         float l = 0.f;            // this half's share of the row sum
-        // The stage's two 64-token units (c = 0, 1), read from the union one
+        // The stage's two 64-token units (c = 0, 1) come from the union
+        // entries (page, block, query mask) of blocks nb and nb + 1, loaded one
         // stage ahead so that their shared-memory latency hides behind the
-        // previous stage: each unit's first token (-1: past the union or an
-        // absent page; tokens fit 31 bits, nb_max * bs < 2^31) and how many of
-        // this half's unit's tokens the row takes. (nb, nsub) walk the units in
-        // order without a division by the units per block.
+        // previous stage; (nb, nsub) walk the units in order without a division
+        // by the units per block. Token positions fit 31 bits (nb_max * bs <
+        // 2^31); an entry past the union is read (in bounds) but not used.
         int nb = 0, nsub = 0;
-        auto load_units = [&](int i, int& t0a, int& t0b, int& nv) {
-            nv = 0;
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                int t = -1;
-                if (2 * i + c < nunits && upage[nb] >= 0) {
-                    t = ublk[nb] * bs + nsub * 64;
-                    if (c == hf && (umask[nb] & qbit) != 0u && (long long)t <= last) {
-                        const long long n = last - t + 1;
-                        nv = n < 64 ? (int)n : 64;
-                    }
-                }
-                if (c == 0) t0a = t; else t0b = t;
-                if (++nsub == upb) {
-                    nsub = 0;
-                    ++nb;
-                }
-            }
+        int pg0, bl0, pg1, bl1;
+        uint32_t mk0, mk1;
+        auto fetch = [&]() {
+            const int b0 = min(nb, kMaxUnion - 1), b1 = min(nb + 1, kMaxUnion - 1);
+            pg0 = upage[b0];
+            bl0 = ublk[b0];
+            mk0 = umask[b0];
+            pg1 = upage[b1];
+            bl1 = ublk[b1];
+            mk1 = umask[b1];
         };
-        int nt0a = -1, nt0b = -1, nnv = 0;
-        if (nstages > 0) load_units(0, nt0a, nt0b, nnv);
+        fetch();
         for (int i = 0; i < nstages; ++i) {
-            const int ut0a = nt0a, ut0b = nt0b, nval = nnv;
-            if (i + 1 < nstages) load_units(i + 1, nt0a, nt0b, nnv);
+            // each unit's first token (-1: past the union or an absent page)
+            const bool same = nsub + 1 < upb;  // unit 1 in the same block as unit 0
+            const int pgb = same ? pg0 : pg1, blb = same ? bl0 : bl1;
+            const uint32_t mkb = same ? mk0 : mk1;
+            const int ut0a = 2 * i < nunits && pg0 >= 0 ? bl0 * bs + nsub * 64 : -1;
+            const int ut0b = 2 * i + 1 < nunits && pgb >= 0 ? blb * bs + (same ? nsub + 1 : 0) * 64 : -1;
+            // this half's unit: whether the row takes it, and how many of its
+            // 64 tokens the row may see
+            const int t0 = hf ? ut0b : ut0a;
+            int nval = 0;
+            if (t0 >= 0 && ((hf ? mkb : mk0) & qbit) != 0u && (long long)t0 <= last) {
+                const long long nv = last - t0 + 1;
+                nval = nv < 64 ? (int)nv : 64;
+            }
+            nsub += 2;
+            while (nsub >= upb) {
+                nsub -= upb;
+                ++nb;
+            }
+            fetch();  // the next stage's entries
             const bool waited = mbar_wait(&sfull[i & 1], (i >> 1) & 1);
             const int my_ok = waited && !*s_abort;
             tc_fence_after();
@@ -503,21 +512,6 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
                 corr = m_ref > -INFINITY ? fast_exp2(m_ref - mrow) : 1.f;
                 m_ref = mrow;
             }
-            if (__any_sync(0xffffffffu, corr != 1.f)) {
-                // O holds earlier stages of this row: rescale this half's
-                // columns once the previous P V has landed
-                if (!mbar_wait(obar, (i - 1) & 1)) *s_abort = 1;
-                tc_fence_after();
-#pragma unroll
-                for (int ch = 0; ch < 2; ++ch) {
-                    uint32_t ov[32];
-                    tmem_ld32(lane_addr + kColO + hf * 64 + ch * 32, ov);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
-                    tmem_st32(lane_addr + kColO + hf * 64 + ch * 32, ov);
-                }
-                l *= corr;
-            }
             // P = 2^(s*c - m) as bf16 pairs; it overwrites the S buffer's first
             // 64 columns (both halves have read their S columns: the barrier above)
             const float neg_m = -m_ref;
@@ -534,12 +528,28 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
                     ps[e & 7] += a + bb;
                     pk[e] = pack_bf16x2(a, bb);
                 }
-                l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+                l = fmaf(l, corr, ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
             } else {
 #pragma unroll
                 for (int e = 0; e < 32; ++e) pk[e] = 0u;
+                l *= corr;
             }
             tmem_st32(lane_addr + kColS + (i & 1) * 128 + hf * 32, pk);
+            if (__any_sync(0xffffffffu, corr != 1.f)) {
+                // O holds earlier stages of this row: rescale this half's
+                // columns once the previous P V has landed (after P, so that
+                // the S registers are free and the wait comes as late as it can)
+                if (!mbar_wait(obar, (i - 1) & 1)) *s_abort = 1;
+                tc_fence_after();
+#pragma unroll 1  // one 32-column chunk in registers at a time
+                for (int ch = 0; ch < 2; ++ch) {
+                    uint32_t ov[32];
+                    tmem_ld32(lane_addr + kColO + hf * 64 + ch * 32, ov);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
+                    tmem_st32(lane_addr + kColO + hf * 64 + ch * 32, ov);
+                }
+            }
             tmem_wait_st();
             // V rows of an absent unit and of tokens past the context length
             // must be zero before the P V MMA reads them (this thread: token row
