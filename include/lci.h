@@ -151,11 +151,13 @@ LCI_API lci_status lci_index_select_workspace_size(int32_t batch, int32_t S, int
  *   d_ctx_len  [batch] int32, d_q_start [batch] int32, device
  *   d_ids      [batch][S][topk] int32, device (output)
  *   workspace  >= lci_index_select_workspace_size bytes, 256-byte aligned.
- *              It holds arrival counters and per-row selection bounds whose
- *              position depends on the sizes (batch, S, nb_max). Zero-fill a
- *              workspace before its first call; every successful call leaves
- *              them at zero again, so later calls with the same sizes need no
- *              clearing. Zero it again before using it with other sizes, and
+ *              It starts with arrival counters and per-row selection bounds
+ *              whose position depends on (batch, S) alone; scratch follows.
+ *              Zero-fill a workspace before its first call; every successful
+ *              call leaves that prefix at zero again, so later calls with the
+ *              same (batch, S) need no clearing, whatever their dtype, topk,
+ *              nb_max or phase (the workspace must still be large enough).
+ *              Zero it again before using it with another (batch, S), and
  *              after a call that failed on the device. Calls that share a
  *              workspace must not overlap in time.
  * Scores are accumulated in fp32. Limits: 1 <= topk <= 256,

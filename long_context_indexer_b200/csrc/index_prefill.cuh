@@ -259,9 +259,20 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
     const long long p_last = (long long)q_start[b] + min(S - 1, row0 + kBM - 1);
     const int vis_max = visible_blocks(p_last, ctx, bs, nb_max);
     const int n_tiles = (vis_max + kBN - 1) / kBN;
-    const int per = (n_tiles + n_split - 1) / n_split;
-    const int t_lo = ns * per;
-    const int t_hi = min(n_tiles, t_lo + per);
+    // Several n-tiles: the CTAs of the m-tile split them. One n-tile: every
+    // CTA computes it and takes a window [c_lo, c_hi) of its visible columns
+    // (whole 32-column groups) into its list.
+    int t_lo = 0, t_hi = 0, c_lo = 0, c_hi = kBN;
+    if (n_tiles == 1 && n_split > 1) {
+        const int cols = ((vis_max + n_split - 1) / n_split + 31) & ~31;
+        c_lo = ns * cols;
+        c_hi = min(kBN, c_lo + cols);
+        t_hi = c_lo < vis_max ? 1 : 0;
+    } else {
+        const int per = (n_tiles + n_split - 1) / n_split;
+        t_lo = ns * per;
+        t_hi = min(n_tiles, t_lo + per);
+    }
     const int my_tiles = max(0, t_hi - t_lo);
 
     if (tid == 0) {
@@ -402,6 +413,10 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
                 atomicMax(bound, gk);
             }
         };
+        // this part's groups c (columns (c * kParts + part) * kGroup ..) inside
+        // the CTA's column window: c_begin <= c < c_end
+        const int c_begin = (c_lo / kGroup - part + kParts - 1) / kParts;
+        const int c_end = (c_hi / kGroup - part + kParts - 1) / kParts;
         for (int t = 0; t < my_tiles; ++t) {
             const int buf = t & 1;
             const bool ok = mbar_wait(&tfull_bar[buf], (t >> 1) & 1);
@@ -438,7 +453,7 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
                     if (lmin > -INFINITY && lmin < INFINITY) gthr = fmaxf(gthr, float_below(lmin));
                 }
 #pragma unroll 1
-                for (int c = 0; c < kGroupsPerPart; ++c) {
+                for (int c = c_begin; c < c_end; ++c) {
                     const int col = (c * kParts + part) * kGroup;  // parts interleave groups
                     // the row's bound as published so far, used from the next group on
                     const uint32_t gk_next = bound != nullptr ? ld_relaxed_gpu(bound) : 0u;

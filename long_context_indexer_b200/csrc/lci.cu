@@ -106,6 +106,18 @@ int index_chunk(long long rows, int32_t K, int32_t nb_max, size_t esz) {
     return chunk;
 }
 
+// Every index_select schedule keeps the state that must start at zero (arrival
+// counters, per-row selection bounds) in one prefix of the workspace whose
+// size depends on (batch, S) alone, and its scratch after it. Each schedule
+// leaves its own zero state at zero after a successful call and writes no
+// scratch inside the prefix, so a workspace serves calls of any dtype, topk
+// or schedule for the same (batch, S) without clearing.
+size_t index_zero_prefix(int32_t batch, int32_t S) {
+    const long long m_tiles = (S + lci::pre::kBM - 1) / lci::pre::kBM;
+    return align_up((size_t)batch * m_tiles * sizeof(unsigned int)) +
+           align_up((size_t)batch * S * sizeof(unsigned int));
+}
+
 IndexPlan plan_index(int32_t batch, int32_t S, int32_t K, int32_t nb_max, size_t esz) {
     IndexPlan pl{};
     const long long rows = (long long)batch * S;
@@ -116,8 +128,8 @@ IndexPlan plan_index(int32_t batch, int32_t S, int32_t K, int32_t nb_max, size_t
     // The layout is sized for the smaller fp32 chunk, so that one workspace
     // size serves both element types.
     const int nchunks_alloc = (nb_max + index_chunk(rows, K, nb_max, 4) - 1) / index_chunk(rows, K, nb_max, 4);
-    pl.off_counters = 0;
-    pl.off_scores = align_up((size_t)rows * sizeof(unsigned int));
+    pl.off_counters = 0;  // rows counters, inside the zero prefix
+    pl.off_scores = index_zero_prefix(batch, S);
     pl.off_chunk_max = pl.off_scores + align_up((size_t)rows * nb_max * sizeof(float));
     pl.bytes = pl.off_chunk_max + align_up((size_t)rows * nchunks_alloc * sizeof(uint32_t));
     pl.qreg = row_bytes == 2048;
@@ -351,21 +363,25 @@ PrefillPlan plan_prefill(int32_t batch, int32_t S, int32_t K, int32_t nb_max, in
     pl.kt = topk <= 16 ? 16 : (topk <= 32 ? 32 : 64);
     const int n_tiles = (nb_max + lci::pre::kBN - 1) / lci::pre::kBN;
     // about one CTA per SM; the merge copies n_split * topk candidates per row
-    // of a 128-row tile into the stage memory
+    // of a 128-row tile into the stage memory. The CTAs of an m-tile split its
+    // n-tiles, or with a single n-tile its visible columns (windows of at
+    // least 64 columns).
     long long split = 148 / ((long long)batch * pl.m_tiles);
     split = split < 1 ? 1 : split;
     split = split > 8 ? 8 : split;
-    split = split > n_tiles ? n_tiles : split;
+    const int split_max = n_tiles == 1 ? lci::pre::kBN / 64 : n_tiles;
+    split = split > split_max ? split_max : split;
     while (split > 1 &&
            (long long)lci::pre::kBM * split * topk * 8 > (long long)lci::pre::kStages * lci::pre::kStageBytes)
         --split;
     pl.n_split = (int)split;
     const long long cand = (long long)batch * pl.m_tiles * lci::pre::kBM * pl.n_split * topk;
+    // counters and row bounds in the zero prefix, then the split lists
     pl.off_counters = 0;
-    pl.off_key = align_up((size_t)batch * pl.m_tiles * sizeof(unsigned int));
+    pl.off_bound = align_up((size_t)batch * pl.m_tiles * sizeof(unsigned int));
+    pl.off_key = index_zero_prefix(batch, S);
     pl.off_id = pl.off_key + align_up((size_t)cand * sizeof(uint32_t));
-    pl.off_bound = pl.off_id + align_up((size_t)cand * sizeof(int32_t));
-    pl.bytes = pl.off_bound + align_up((size_t)batch * S * sizeof(unsigned int));
+    pl.bytes = pl.off_id + align_up((size_t)cand * sizeof(int32_t));
     return pl;
 }
 

@@ -476,3 +476,30 @@ def test_both_decode_forms_share_one_workspace():
         assert torch.equal(ids.cpu().reshape(-1, cfg.topk), ref_ids), persistent
         assert_out_close(out.reshape(-1, cfg.H_q, cfg.hd), ref_out, cfg.torch_dtype,
                          f"persistent={persistent}")
+
+
+def test_one_workspace_serves_every_schedule_dtype_and_topk():
+    """Calls with the same (batch, S) share one workspace without clearing it:
+    the tensor-core schedule with split candidate lists (bf16, two topk
+    values) and the row-wise schedule (f32, and bf16 with phase 'decode')
+    alternate on it, and every call's ids match the oracle."""
+    base = SMALL.replace(S=37, q_start=950, ctx=1000)
+    calls = [("bf16", 3, "prefill"), ("f32", 3, "auto"), ("bf16", 16, "prefill"),
+             ("bf16", 5, "decode"), ("bf16", 3, "prefill"), ("f32", 16, "auto")]
+    need = max(lci.index_select_workspace_size(base.B, base.S, base.H_i, base.d_c, base.NB, k, ph)
+               for _, k, ph in calls)
+    ws = torch.zeros(need + 256, dtype=torch.uint8, device="cuda")
+    off = (-ws.data_ptr()) % 256
+    ws = ws[off:off + need]
+    for dtype, topk, phase in calls:
+        cfg = base.replace(dtype=dtype, topk=topk)
+        w = generate(cfg, with_kv=False)
+        w["ctx_len"] = torch.tensor([1000, 500, 1], dtype=torch.int32)
+        w["q_start"] = torch.tensor([950, 617, 0], dtype=torch.int32)
+        d = upload(w)
+        ids = lci.index_select(d["q_c"], d["k_c"], cfg.bs, d["ctx_len"], d["q_start"], topk,
+                               phase=phase, ws=ws)
+        torch.cuda.synchronize()
+        lci.get_device_status()
+        ref = oracle.index_select(w["q_c"], w["k_c"], cfg.bs, w["ctx_len"], w["q_start"], topk)
+        assert torch.equal(ids.cpu().reshape(-1, topk), ref), (dtype, topk, phase)
