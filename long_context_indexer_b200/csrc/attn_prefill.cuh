@@ -482,14 +482,17 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
                     for (int e = 0; e < 64; ++e)
                         sv[e] = e < nval ? sv[e] : __float_as_uint(-INFINITY);
                 }
-                // eight independent running maxima, then a tree
+                // eight independent running maxima, two new values per
+                // three-input max, then a tree
                 float pm[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) pm[k] = __uint_as_float(sv[k]);
 #pragma unroll
-                for (int e = 8; e < 64; ++e) pm[e & 7] = fmaxf(pm[e & 7], __uint_as_float(sv[e]));
-                mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                           fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+                for (int e = 8; e < 64; e += 2)
+                    pm[(e >> 1) & 7] = fmax3(pm[(e >> 1) & 7], __uint_as_float(sv[e]),
+                                             __uint_as_float(sv[e + 1]));
+                mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]),
+                           fmaxf(pm[6], pm[7]));
             }
             // the row maximum of the stage (raw scores; the scale is positive),
             // and whether both halves may go on: one decision for the pair of
@@ -517,18 +520,25 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
             const float neg_m = -m_ref;
             uint32_t pk[32];
             if (nval > 0) {
-                float ps[8];
+                // the scale and shift, and the row sum, on packed fp32 pairs:
+                // one instruction for two tokens
+                const float2 sc2 = make_float2(scale_log2, scale_log2);
+                const float2 nm2 = make_float2(neg_m, neg_m);
+                float2 ps[4];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) ps[k] = 0.f;
+                for (int k = 0; k < 4; ++k) ps[k] = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     // masked entries hold -inf: 2^-inf = 0
-                    const float a = fast_exp2(fmaf(__uint_as_float(sv[2 * e]), scale_log2, neg_m));
-                    const float bb = fast_exp2(fmaf(__uint_as_float(sv[2 * e + 1]), scale_log2, neg_m));
-                    ps[e & 7] += a + bb;
-                    pk[e] = pack_bf16x2(a, bb);
+                    const float2 x = ffma2(
+                        make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), sc2, nm2);
+                    const float2 pe = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                    ps[e & 3] = fadd2(ps[e & 3], pe);
+                    pk[e] = pack_bf16x2(pe.x, pe.y);
                 }
-                l = fmaf(l, corr, ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
+                const float2 s01 = fadd2(ps[0], ps[1]), s23 = fadd2(ps[2], ps[3]);
+                const float2 st = fadd2(s01, s23);
+                l = fmaf(l, corr, st.x + st.y);
             } else {
 #pragma unroll
                 for (int e = 0; e < 32; ++e) pk[e] = 0u;
