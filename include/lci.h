@@ -343,7 +343,8 @@ LCI_API lci_status lci_attn_merge(const void* d_o, const float* d_lse, lci_dtype
  * whatever the phase. Its scratch is one fixed array of
  * LCI_NOALLOC_SCRATCH_BYTES bytes inside the library, which every GPU that
  * loads the library holds until the process exits. The scratch a call needs is
- *   align256(4*rows) + align256(4*rows*nb_max) + align256(4*rows*nchunks)
+ *   align256(4*batch*ceil(S/128)) + align256(4*rows) + align256(4*rows*nb_max)
+ *   + align256(4*rows*nchunks)
  * bytes (rows = batch*S; nchunks <= nb_max, the chunks a row is scored in),
  * which is exactly what lci_index_select_workspace_size returns for the same
  * sizes with LCI_PHASE_DECODE. Sizes whose scratch exceeds the array return
