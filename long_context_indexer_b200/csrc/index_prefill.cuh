@@ -27,8 +27,9 @@
 // lists of a row grow at the same time, the bound runs only a little ahead of
 // each list's own threshold.
 //
-// n-tiles beyond the last visible block of the m-tile are skipped. When an
-// m-tile's n-tiles are split over several CTAs, each writes its per-row
+// n-tiles beyond the last visible block of the m-tile are skipped. An m-tile
+// may be split over several CTAs: by n-tiles, or, when it has a single n-tile,
+// by windows of that tile's visible columns. Each CTA then writes its per-row
 // candidates (key, id) to the workspace and the last CTA to arrive (atomic
 // counter, no spin-wait) merges them. Ties break to the lower block id.
 #pragma once
