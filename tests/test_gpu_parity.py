@@ -503,3 +503,20 @@ def test_one_workspace_serves_every_schedule_dtype_and_topk():
         lci.get_device_status()
         ref = oracle.index_select(w["q_c"], w["k_c"], cfg.bs, w["ctx_len"], w["q_start"], topk)
         assert torch.equal(ids.cpu().reshape(-1, topk), ref), (dtype, topk, phase)
+
+
+@pytest.mark.parametrize("topk", [32, 64])
+def test_prefill_indexer_column_windows(topk):
+    """Every m-tile has a single 256-block n-tile, so its CTAs (four here) split
+    the tile's visible columns into windows of whole 32-column groups, the last
+    window ragged, and the last CTA merges the windows' lists."""
+    cfg = SMALL.replace(B=1, S=2560, ctx=12800, q_start=12800 - 2560, topk=topk)
+    assert cfg.NB == 200
+    w = generate(cfg, with_kv=False)
+    d = upload(w)
+    ids = lci.index_select(d["q_c"], d["k_c"], cfg.bs, d["ctx_len"], d["q_start"], topk,
+                           phase="prefill")
+    torch.cuda.synchronize()
+    lci.get_device_status()
+    ref = oracle.index_select(w["q_c"], w["k_c"], cfg.bs, w["ctx_len"], w["q_start"], topk)
+    assert torch.equal(ids.cpu().reshape(-1, topk), ref)
