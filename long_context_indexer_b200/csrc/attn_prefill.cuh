@@ -423,6 +423,9 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
         const int qi = r / G, s = s0 + qi;
         const long long p = (long long)q_start[b] + s;
         const long long last = s < S ? (p < ctx - 1 ? p : ctx - 1) : -1;
+        // 32-bit copies for the per-stage tests (token positions fit 31 bits)
+        const int last32 = (int)(last < 0x7fffffffLL ? last : 0x7fffffffLL);
+        const int ctx32 = (int)(ctx < 0x7fffffffLL ? ctx : 0x7fffffffLL);
         const uint32_t qbit = 1u << qi;
         const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
         float* xchg = reinterpret_cast<float*>(smem + kOffXchg);  // [3][2][128]
@@ -459,10 +462,8 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
             // 64 tokens the row may see
             const int t0 = hf ? ut0b : ut0a;
             int nval = 0;
-            if (t0 >= 0 && ((hf ? mkb : mk0) & qbit) != 0u && (long long)t0 <= last) {
-                const long long nv = last - t0 + 1;
-                nval = nv < 64 ? (int)nv : 64;
-            }
+            if (t0 >= 0 && ((hf ? mkb : mk0) & qbit) != 0u && t0 <= last32)
+                nval = last32 - t0 >= 63 ? 64 : last32 - t0 + 1;
             nsub += 2;
             while (nsub >= upb) {
                 nsub -= upb;
@@ -565,12 +566,12 @@ __global__ void __launch_bounds__(pfa::kThreads, 1) sparse_attn_prefill_kernel(
             // must be zero before the P V MMA reads them (this thread: token row
             // r of the stage, dims 64*hf .. 64*hf+63)
             const bool stage_tail =  // the same for every thread
-                ut0a < 0 || ut0b < 0 || ut0a + 64LL > ctx || ut0b + 64LL > ctx;
+                ut0a < 0 || ut0b < 0 || ut0a > ctx32 - 64 || ut0b > ctx32 - 64;
             if (stage_tail) {
                 const int vs = i % kVStages;
                 if (!mbar_wait(&vfull[vs], (i / kVStages) & 1)) *s_abort = 1;
                 const int mine_t0 = (r >> 6) ? ut0b : ut0a;
-                if (mine_t0 < 0 || (long long)mine_t0 + (r & 63) >= ctx) {
+                if (mine_t0 < 0 || mine_t0 + (r & 63) >= ctx32) {
                     unsigned char* vt = smem + kOffV + vs * kTileBytes;
 #pragma unroll
                     for (int cc = 8 * hf; cc < 8 * hf + 8; ++cc)
