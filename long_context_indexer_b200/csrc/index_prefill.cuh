@@ -56,9 +56,12 @@ constexpr int kSmemBytes = kStages * kStageBytes + kCandBytes + 1024 /*align*/ +
 // length KT.
 template <int KT> struct Epi { static constexpr int kParts = KT <= 32 ? 2 : 1; };
 template <int KT> struct Cfg { static constexpr int kThreads = 64 + 128 * Epi<KT>::kParts; };
-// instruction descriptor: D fp32, A/B bf16, both K-major, N = 256, M = 128
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
-                            ((uint32_t)(kBM >> 4) << 24);
+// instruction descriptor: D fp32, A/B bf16, both K-major, M = 128, N = n (a
+// multiple of 16 up to 256: the first n rows of the B tile)
+__host__ __device__ constexpr uint32_t idesc_n(int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+           ((uint32_t)(kBM >> 4) << 24);
+}
 }  // namespace pre
 
 // Shared-memory matrix descriptor of a K-major tile written by TMA with the
@@ -355,6 +358,10 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
                 if (t >= 2) ok = mbar_wait(&tempty_bar[buf], ((t >> 1) - 1) & 1);
                 tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)(buf * kBN);
+                // only the tile's visible columns (and none past the CTA's
+                // window): the epilogue never reads the others
+                const int ncols = min(min(kBN, vis_max - (t_lo + t) * kBN), c_hi);
+                const uint32_t idesc = idesc_n(max(16, (ncols + 15) & ~15));
                 for (int ks = 0; ks < ksteps && ok; ++ks, ++it) {
                     const int st = it % kStages;
                     ok = mbar_wait(&full_bar[st], (it / kStages) & 1);
@@ -363,7 +370,7 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
                     const uint64_t ad = sw128_desc(a), bd = sw128_desc(a + kABytes);
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk)  // +32 bytes per K=16 step
-                        tc_mma(d, ad + 2 * kk, bd + 2 * kk, kIdesc, (ks | kk) != 0);
+                        tc_mma(d, ad + 2 * kk, bd + 2 * kk, idesc, (ks | kk) != 0);
                     tc_commit(&empty_bar[st]);  // the stage is free once these MMAs finish
                 }
                 tc_commit(&tfull_bar[buf]);  // accumulator ready
@@ -426,9 +433,9 @@ __global__ void __launch_bounds__(pre::Cfg<KT>::kThreads, 1) index_prefill_tc_ke
             if (ok) {
                 const uint32_t lane_base =
                     tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kBN);
-                if (t == 0 && __all_sync(0xffffffffu, n0 + kBN <= vis)) {
+                if (t == 0 && c_hi == kBN && __all_sync(0xffffffffu, n0 + kBN <= vis)) {
                     // First tile, empty list, every column visible to the warp's
-                    // rows: a lower bound of this part's KT-th
+                    // rows (and computed: no column window): a lower bound of this part's KT-th
                     // best score from the tile itself. Its columns fall into KT
                     // runs of kSub; every run's maximum is a score of the part, so
                     // with L the smallest run maximum, KT scores are >= L and a

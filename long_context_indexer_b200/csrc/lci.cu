@@ -364,12 +364,11 @@ PrefillPlan plan_prefill(int32_t batch, int32_t S, int32_t K, int32_t nb_max, in
     const int n_tiles = (nb_max + lci::pre::kBN - 1) / lci::pre::kBN;
     // about one CTA per SM; the merge copies n_split * topk candidates per row
     // of a 128-row tile into the stage memory. The CTAs of an m-tile split its
-    // n-tiles, or with a single n-tile its visible columns (windows of at
-    // least 64 columns).
+    // n-tiles, or with a single n-tile its visible columns.
     long long split = 148 / ((long long)batch * pl.m_tiles);
     split = split < 1 ? 1 : split;
     split = split > 8 ? 8 : split;
-    const int split_max = n_tiles == 1 ? lci::pre::kBN / 64 : n_tiles;
+    const int split_max = n_tiles == 1 ? lci::pre::kBN / 64 : n_tiles;  // windows of >= 64 columns
     split = split > split_max ? split_max : split;
     while (split > 1 &&
            (long long)lci::pre::kBM * split * topk * 8 > (long long)lci::pre::kStages * lci::pre::kStageBytes)
