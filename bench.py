@@ -101,9 +101,9 @@ def peaks():
 # sources the capture ran. Once those sources change the figure no longer
 # describes the kernel and the bench reports traffic as null.
 PROFILED_TRAFFIC = {
-    ("decode", "index_select"): (33752064, "348a2e47c2fd0efe"),
-    ("decode", "sparse_attn"): (33811968, "348a2e47c2fd0efe"),
-    ("1m_chunk", "index_select"): (25248512, "348a2e47c2fd0efe"),
+    ("decode", "index_select"): (33751808, "7c06d6f15ea82c7c"),
+    ("decode", "sparse_attn"): (33816576, "7c06d6f15ea82c7c"),
+    ("1m_chunk", "index_select"): (25255680, "7c06d6f15ea82c7c"),
 }
 
 
