@@ -424,15 +424,23 @@ def time_graph(g, reps, warmup):
     return e0.elapsed_time(e1) / reps
 
 
-def e2e_graph(pipes):
-    """The R replicas' steps as one CUDA graph of a pipelined serving loop over
-    independent batches: every step copies its inputs in from pinned host
-    memory (one stream), runs the library's prepared decode step (another) and
-    copies its results back to pinned host memory (a third), so a step's
-    copies overlap its neighbours' kernels; each step's kernels wait for its
-    own inputs and its copy back waits for its kernels."""
+E2E_PASSES = 4  # passes over the replicas in one end-to-end graph
+
+
+def e2e_graph(pipes, passes=E2E_PASSES):
+    """`passes` rounds over the R replicas' steps as one CUDA graph of a
+    pipelined serving loop over independent batches: every step copies its
+    inputs in from pinned host memory (one stream), runs the library's prepared
+    decode step (another) and copies its results back to pinned host memory (a
+    third), so a step's copies overlap its neighbours' kernels. Each step's
+    kernels wait for its own inputs and its copy back for its kernels; a step
+    that reuses a replica's buffers also waits, for its upload, until the
+    previous step on that replica has computed, and for its kernels until that
+    step's results have been copied back. Several passes spread the graph's
+    first upload and last download over more steps."""
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     g = torch.cuda.CUDAGraph()
+    R = len(pipes)
     torch.cuda.synchronize()
     with torch.cuda.graph(g):
         cap = torch.cuda.current_stream()
@@ -440,21 +448,28 @@ def e2e_graph(pipes):
         start.record(cap)
         s_in.wait_event(start)
         s_out.wait_event(start)
-        ev_in = []
-        with torch.cuda.stream(s_in):
-            for p in pipes:
+        ev_comp, ev_out = [], []
+        for i in range(R * passes):
+            p = pipes[i % R]
+            with torch.cuda.stream(s_in):
+                if i >= R:
+                    s_in.wait_event(ev_comp[i - R])
                 p._d_in.copy_(p._h_in, non_blocking=True)
-                e = torch.cuda.Event()
-                e.record(s_in)
-                ev_in.append(e)
-        for p, e in zip(pipes, ev_in):
-            cap.wait_event(e)
+                e_in = torch.cuda.Event()
+                e_in.record(s_in)
+            cap.wait_event(e_in)
+            if i >= R:
+                cap.wait_event(ev_out[i - R])
             p._prepared(cap)
             k = torch.cuda.Event()
             k.record(cap)
+            ev_comp.append(k)
             s_out.wait_event(k)
             with torch.cuda.stream(s_out):
                 p._h_out.copy_(p._d_out, non_blocking=True)
+                o = torch.cuda.Event()
+                o.record(s_out)
+            ev_out.append(o)
         done = torch.cuda.Event()
         done.record(s_out)
         cap.wait_event(done)
@@ -474,9 +489,11 @@ def time_e2e(pipes, steps, warmup):
     R = len(pipes)
     g = e2e_graph(pipes) if all(p._prepared is not None for p in pipes) else None
 
+    per_graph = R * E2E_PASSES
+
     def run(n):
         if g is not None:
-            for _ in range(-(-n // R)):
+            for _ in range(-(-n // per_graph)):
                 g.replay()
             return
         for i in range(n):
@@ -496,7 +513,7 @@ def time_e2e(pipes, steps, warmup):
     torch.cuda.synchronize()
     if SAMPLER is not None:
         SAMPLER.active = False
-    n_done = -(-steps // R) * R if g is not None else steps
+    n_done = -(-steps // per_graph) * per_graph if g is not None else steps
     return e0.elapsed_time(e1) * steps / n_done
 
 
