@@ -520,3 +520,22 @@ def test_prefill_indexer_column_windows(topk):
     lci.get_device_status()
     ref = oracle.index_select(w["q_c"], w["k_c"], cfg.bs, w["ctx_len"], w["q_start"], topk)
     assert torch.equal(ids.cpu().reshape(-1, topk), ref)
+
+
+def test_prefill_indexer_sequence_without_context():
+    """The tensor-core schedule with a sequence whose context is empty (no
+    visible block in any of its m-tiles, every CTA's window empty) beside one
+    whose m-tiles split their columns: the empty one gets -1 everywhere."""
+    cfg = SMALL.replace(B=2, S=256, ctx=3000, q_start=3000 - 256, topk=8)
+    w = generate(cfg, with_kv=False)
+    w["ctx_len"] = torch.tensor([3000, 0], dtype=torch.int32)
+    w["q_start"] = torch.tensor([3000 - 256, 0], dtype=torch.int32)
+    d = upload(w)
+    ids = lci.index_select(d["q_c"], d["k_c"], cfg.bs, d["ctx_len"], d["q_start"], cfg.topk,
+                           phase="prefill")
+    torch.cuda.synchronize()
+    lci.get_device_status()
+    ref = oracle.index_select(w["q_c"], w["k_c"], cfg.bs, w["ctx_len"], w["q_start"], cfg.topk)
+    got = ids.cpu().reshape(-1, cfg.topk)
+    assert torch.equal(got, ref)
+    assert (got[cfg.S:] == -1).all()
